@@ -1,0 +1,218 @@
+/*
+ * nvfp4pw.h -- C ABI of the B200 (sm_100a) NVFP4 GPTQ + Schur Replay layer solve.
+ *
+ * Method: "Replay the Curvature: Accurate and Scalable NVFP4 Quantization for
+ * Large Language Model Inference" (arXiv 2609.36654v1), Abstract:
+ *   - NVFP4: every 16 consecutive E2M1 weights share one E4M3 block scale
+ *     (Abstract, sentence defining NVFP4); a per-tensor fp32 global scale sits
+ *     on top (s_g = amax|W| / (6 * 448)).
+ *   - GPTQ: quantizing one column updates the columns that follow it (Abstract,
+ *     sentence on why the scale choice is hard); second-order state H = X^T X
+ *     is accumulated from calibration activations (Abstract, sentence on
+ *     second-order state).
+ *   - Schur Replay: each candidate block scale is scored by replaying the
+ *     in-block GPTQ updates it causes and measuring the block error left after
+ *     compensation from the still-unquantized columns (Abstract, sentence
+ *     introducing Schur Replay).
+ *
+ * Conventions for every call
+ *   - All array pointers are DEVICE pointers unless the argument says "host".
+ *     The caller owns every buffer; the library allocates no device memory
+ *     (scratch comes from a caller-provided workspace whose size the
+ *     *_workspace_size() calls return).
+ *   - Matrices are row-major and densely packed (leading dimension = columns).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns a host-side status at once.  Conditions that
+ *     only the GPU can see (non-finite input, a non-positive pivot) are written
+ *     to a sticky status word at the start of the workspace; read it with
+ *     nvfp4_workspace_status() after the stream's work is done.  No kernel
+ *     traps or spins without a bound.
+ *   - Sizes are int64_t; negative sizes are NVFP4_ERR_INVALID_ARG.  The
+ *     quantized dimension (d, d_in) must be a multiple of 16.
+ */
+#ifndef NVFP4PW_H
+#define NVFP4PW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call and stored in the device status word. */
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum        */
+  NVFP4_ERR_SHAPE = 2,       /* d or d_in not a multiple of 16, or too large */
+  NVFP4_ERR_WORKSPACE = 3,   /* workspace null or smaller than required      */
+  NVFP4_ERR_NONFINITE = 4,   /* NaN/Inf met in W or H (device-detected)      */
+  NVFP4_ERR_NOT_PD = 5,      /* damped H not positive definite (device)      */
+  NVFP4_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (device)       */
+  NVFP4_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed         */
+  NVFP4_ERR_UNSUPPORTED = 8  /* parameter value this build does not support  */
+} nvfp4_status;
+
+/* Element type of an input or output array. */
+typedef enum { NVFP4_BF16 = 0, NVFP4_F32 = 1 } nvfp4_dtype;
+
+/* Opaque stream handle, layout-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+/* Solve parameters.  Only the defaults below are supported by this build
+ * (n_candidates = 16, cand_lo = -8, lazy_batch = 128); other values return
+ * NVFP4_ERR_UNSUPPORTED.  The candidate window is the n_candidates
+ * consecutive E4M3 codes starting at k0 + cand_lo, shifted into 1..126,
+ * where k0 = e4m3_rn(amax_block / (6 s_g)) (at least 1). */
+typedef struct {
+  int n_candidates; /* 16 */
+  int cand_lo;      /* -8 */
+  int lazy_batch;   /* 128: columns per batch of the trailing update */
+  int reserved;     /* 0 */
+} nvfp4_solve_params;
+
+/* Fills *p with the defaults above. */
+void nvfp4_default_params(nvfp4_solve_params* p);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* Synchronizes `stream`, then returns the device status word that the
+ * prepare / quantize calls keep at the start of their workspace `ws`
+ * (NVFP4_OK if nothing was flagged).  Returns NVFP4_ERR_CUDA if the copy
+ * fails.  The word is sticky: it is cleared at the start of the next call
+ * that uses the same workspace. */
+nvfp4_status nvfp4_workspace_status(const void* ws, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* a1  Hessian: H (+)= X^T X over calibration tokens                          */
+/* "Replay the Curvature", Abstract (second-order state from calibration     */
+/* activations).                                                             */
+/* ------------------------------------------------------------------------ */
+/* H     : d x d fp32, full symmetric matrix (both triangles written).
+ * X     : n_tok x d, bf16 or fp32 (x_dtype), one token per row.
+ * beta  : 0 -> H = X^T X, 1 -> H += X^T X (accumulate over token chunks).
+ * d must be a multiple of 16; n_tok >= 0 (0 with beta = 0 zeroes H).
+ * bf16 products are exact in fp32 and are summed in fp32 on the tensor cores;
+ * fp32 inputs are multiplied and summed in fp32.  No workspace. */
+nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dtype,
+                                      int64_t n_tok, int64_t d, int beta,
+                                      nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* a2-a4  damping + upper Cholesky factor of the damped inverse              */
+/* ------------------------------------------------------------------------ */
+/* Bytes of workspace nvfp4_gptq_prepare needs for dimension d. */
+size_t nvfp4_prepare_workspace_size(int64_t d);
+
+/* H       : d x d fp32 symmetric (read only).
+ * damp    : lambda = damp * mean(diag H) is added to the diagonal (0.01).
+ *           A column with H_ii == 0 is dead: H_ii := 1 before damping.
+ * U       : d x d fp32 out; upper triangular with positive diagonal and
+ *           (H + lambda I)^-1 = U^T U; the strict lower triangle is written 0.
+ * dead    : optional (may be NULL) d bytes out, 1 where column i is dead.
+ * lambda_out : optional (may be NULL) device fp32 scalar out, lambda.
+ * ws/ws_bytes : workspace of at least nvfp4_prepare_workspace_size(d) bytes,
+ *           256-byte aligned.  A non-positive pivot sets NVFP4_ERR_NOT_PD and
+ *           a non-finite H sets NVFP4_ERR_NONFINITE in the status word; U is
+ *           then unspecified. */
+nvfp4_status nvfp4_gptq_prepare(const float* H, int64_t d, float damp, float* U,
+                                uint8_t* dead, float* lambda_out, void* ws,
+                                size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* a5-a8  GPTQ with Schur Replay block-scale selection                       */
+/* ------------------------------------------------------------------------ */
+/* Bytes of workspace nvfp4_gptq_schur_replay_quantize needs. */
+size_t nvfp4_quantize_workspace_size(int64_t d_out, int64_t d_in,
+                                     const nvfp4_solve_params* params);
+
+/* W       : d_out x d_in, bf16 or fp32 (w_dtype), read only.
+ * U       : d_in x d_in fp32 upper factor from nvfp4_gptq_prepare (several
+ *           weight matrices with the same input, e.g. q/k/v, share one U).
+ * params  : NULL for the defaults.
+ * dead    : optional d_in bytes from nvfp4_gptq_prepare; dead columns of W
+ *           are treated as zero.
+ * codes   : d_out x d_in/2 bytes out; byte c of a row packs column 2c in the
+ *           low nibble and column 2c+1 in the high nibble; nibble bit 3 is the
+ *           sign, bits 2..0 index {0, 0.5, 1, 1.5, 2, 3, 4, 6}; zero is +0.
+ * scales  : d_out x d_in/16 bytes out, E4M3 (fn) codes; 0 for an all-zero
+ *           block.
+ * global_scale : device fp32 scalar out, s_g = amax|W| / 2688 (1 if W == 0).
+ * err_out : optional (may be NULL) device fp64 scalar out, sum of delta^2 =
+ *           tr((W-Q)(H + lambda I)(W-Q)^T) up to rounding.
+ * ws/ws_bytes : workspace (256-byte aligned) of at least
+ *           nvfp4_quantize_workspace_size() bytes; holds the fp64 working copy
+ *           of W (8 bytes per weight) and the fp64 deltas of one lazy batch.
+ *           Non-finite W sets NVFP4_ERR_NONFINITE in its status word.
+ * d_out is at most 2^22 and d_in at most 2^17 (NVFP4_ERR_SHAPE beyond).
+ * The working copy and the replay are fp64: the codes are discrete decisions
+ * taken on values that every earlier column's update has moved, so they need
+ * more than fp32 precision to match an exact-arithmetic solve. */
+nvfp4_status nvfp4_gptq_schur_replay_quantize(
+    const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in, const float* U,
+    const nvfp4_solve_params* params, const uint8_t* dead, uint8_t* codes,
+    uint8_t* scales, float* global_scale, double* err_out, void* ws, size_t ws_bytes,
+    nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* a9  dequantization: Q = e2m1(code) * e4m3(scale) * s_g                    */
+/* "Replay the Curvature", Abstract (NVFP4 format).                          */
+/* ------------------------------------------------------------------------ */
+/* codes/scales/global_scale as written by the quantize call.
+ * out     : d_out x d_in, fp32 or bf16 (out_dtype).  The product
+ *           e2m1 * e4m3 is exact; the result is the exactly rounded
+ *           (round-to-nearest-even) value of the full product in out_dtype. */
+nvfp4_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales,
+                           const float* global_scale, int64_t d_out, int64_t d_in,
+                           void* out, nvfp4_dtype out_dtype, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* a10  layer error tr((W - Q) H (W - Q)^T) (measurement)                   */
+/* ------------------------------------------------------------------------ */
+size_t nvfp4_layer_error_workspace_size(int64_t d_out, int64_t d_in);
+
+/* W, w_dtype : the original weights (dead columns contribute 0 because their
+ *           H row is 0).  codes/scales/global_scale from the quantize call.
+ * H       : d_in x d_in fp32, undamped.
+ * err_out : device fp64 scalar out.
+ * ws      : at least nvfp4_layer_error_workspace_size() bytes. */
+nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t* codes,
+                               const uint8_t* scales, const float* global_scale,
+                               const float* H, int64_t d_out, int64_t d_in,
+                               double* err_out, void* ws, size_t ws_bytes,
+                               nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics: launch accounting and per-phase device timing                */
+/* (measurement support; the paper has no counterpart)                       */
+/* ------------------------------------------------------------------------ */
+/* Number of kernels this library has launched since it was loaded (all
+ * threads, all devices).  Host-only; never fails. */
+long long nvfp4_launch_count(void);
+
+/* Phases reported by nvfp4_profile_end, in this order. */
+enum {
+  NVFP4_PHASE_HESSIAN = 0, /* nvfp4_hessian_accumulate                      */
+  NVFP4_PHASE_PREPARE = 1, /* nvfp4_gptq_prepare                            */
+  NVFP4_PHASE_REPLAY = 2,  /* Schur Replay batch kernels of the quantize call */
+  NVFP4_PHASE_UPDATE = 3,  /* trailing-update GEMMs of the quantize call    */
+  NVFP4_PHASE_DEQUANT = 4, /* nvfp4_dequant                                 */
+  NVFP4_PHASE_OTHER = 5,   /* everything else (prologues, reductions)       */
+  NVFP4_NUM_PHASES = 6
+};
+
+/* Starts a profiling window: from now on every phase above records a CUDA
+ * event pair on its launching stream.  Resets the per-phase launch counts. */
+nvfp4_status nvfp4_profile_begin(void);
+
+/* Ends the window: waits for the recorded events and writes, for phases
+ * 0..n_phases-1, the summed device time in ms (ms[]) and the number of kernel
+ * launches (launches[]).  NVFP4_OTHER's time is not measured (0).  Returns
+ * NVFP4_ERR_CUDA if an event could not be read. */
+nvfp4_status nvfp4_profile_end(double* ms, long long* launches, int n_phases);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4PW_H */

@@ -1,0 +1,160 @@
+"""ctypes binding of libnvfp4pw.so: the C-ABI calls under the same names.
+
+Argument marshalling only -- every step of the solve runs in the library's CUDA
+kernels.  torch provides device memory and streams.  If the library is not
+built, importing the calls raises: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4pw.so")
+
+NVFP4_BF16 = 0
+NVFP4_F32 = 1
+
+_STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace",
+    4: "non-finite input", 5: "not positive definite", 6: "timeout", 7: "CUDA error",
+    8: "unsupported parameter",
+}
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, call, code):
+        self.code = int(code)
+        super().__init__(f"{call}: status {code} ({_STATUS.get(int(code), 'unknown')})")
+
+
+class SolveParams(ctypes.Structure):
+    _fields_ = [("n_candidates", ctypes.c_int), ("cand_lo", ctypes.c_int),
+                ("lazy_batch", ctypes.c_int), ("reserved", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m nvfp4_post_weight_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        f32 = ctypes.c_float
+        sig = {
+            "nvfp4_status_string": ([i32], ctypes.c_char_p),
+            "nvfp4_workspace_status": ([vp, vp], i32),
+            "nvfp4_default_params": ([ctypes.POINTER(SolveParams)], None),
+            "nvfp4_hessian_accumulate": ([vp, vp, i32, i64, i64, i32, vp], i32),
+            "nvfp4_prepare_workspace_size": ([i64], sz),
+            "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
+            "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
+            "nvfp4_gptq_schur_replay_quantize": (
+                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, sz,
+                 vp], i32),
+            "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
+            "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
+            "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(call, code):
+    if code != 0:
+        raise Nvfp4Error(call, code)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return NVFP4_BF16
+    if t.dtype == torch.float32:
+        return NVFP4_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device byte buffer of at least nbytes."""
+    buf = torch.empty(int(nbytes) + 256, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 256
+    return buf[off:off + int(nbytes)]
+
+
+def default_params() -> SolveParams:
+    p = SolveParams()
+    lib().nvfp4_default_params(ctypes.byref(p))
+    return p
+
+
+def nvfp4_workspace_status(ws, stream=None) -> int:
+    return int(lib().nvfp4_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def nvfp4_hessian_accumulate(H, X, beta=0, stream=None):
+    n_tok, d = X.shape
+    _check("nvfp4_hessian_accumulate", lib().nvfp4_hessian_accumulate(
+        _ptr(H), _ptr(X), _dtype_code(X), n_tok, d, int(beta), _stream(stream)))
+
+
+def nvfp4_prepare_workspace_size(d) -> int:
+    return int(lib().nvfp4_prepare_workspace_size(int(d)))
+
+
+def nvfp4_gptq_prepare(H, damp, U, dead=None, lambda_out=None, ws=None, stream=None):
+    d = H.shape[0]
+    _check("nvfp4_gptq_prepare", lib().nvfp4_gptq_prepare(
+        _ptr(H), d, float(damp), _ptr(U), _ptr(dead), _ptr(lambda_out), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def nvfp4_quantize_workspace_size(d_out, d_in, params=None) -> int:
+    p = params if params is not None else default_params()
+    return int(lib().nvfp4_quantize_workspace_size(int(d_out), int(d_in), ctypes.byref(p)))
+
+
+def nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, global_scale, err_out=None,
+                                     dead=None, ws=None, params=None, stream=None):
+    d_out, d_in = W.shape
+    p = params if params is not None else default_params()
+    _check("nvfp4_gptq_schur_replay_quantize", lib().nvfp4_gptq_schur_replay_quantize(
+        _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
+        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def nvfp4_dequant(codes, scales, global_scale, out, stream=None):
+    d_out, d_in = out.shape
+    _check("nvfp4_dequant", lib().nvfp4_dequant(
+        _ptr(codes), _ptr(scales), _ptr(global_scale), d_out, d_in, _ptr(out),
+        _dtype_code(out), _stream(stream)))
+
+
+def nvfp4_layer_error_workspace_size(d_out, d_in) -> int:
+    return int(lib().nvfp4_layer_error_workspace_size(int(d_out), int(d_in)))
+
+
+def nvfp4_layer_error(W, codes, scales, global_scale, H, err_out, ws, stream=None):
+    d_out, d_in = W.shape
+    _check("nvfp4_layer_error", lib().nvfp4_layer_error(
+        _ptr(W), _dtype_code(W), _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(H),
+        d_out, d_in, _ptr(err_out), _ptr(ws), ws.numel(), _stream(stream)))

@@ -1,0 +1,146 @@
+// C-ABI entry points: argument validation, then the kernel launchers.
+#include <string.h>
+
+#include "common.cuh"
+
+using namespace nvfp4;
+
+namespace nvfp4 {
+nvfp4_status launch_hessian_simt(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
+                                 int64_t d, int beta, cudaStream_t st);
+}
+
+namespace {
+
+bool params_ok(const nvfp4_solve_params* p) {
+  if (!p) return true;
+  return p->n_candidates == kCand && p->cand_lo == -8 && p->lazy_batch == kLazyBatch &&
+         p->reserved == 0;
+}
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+// Largest dimension this build accepts; keeps every int index below 2^31.
+constexpr int64_t kMaxDim = 1 << 17;
+// Largest row count (output channels) accepted; keeps grid.y within 65535 tiles.
+constexpr int64_t kMaxRows = 1 << 22;
+
+}  // namespace
+
+extern "C" {
+
+void nvfp4_default_params(nvfp4_solve_params* p) {
+  if (!p) return;
+  p->n_candidates = kCand;
+  p->cand_lo = -8;
+  p->lazy_batch = kLazyBatch;
+  p->reserved = 0;
+}
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_SHAPE: return "unsupported shape (dimension must be a multiple of 16)";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case NVFP4_ERR_NONFINITE: return "non-finite value in the input";
+    case NVFP4_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case NVFP4_ERR_TIMEOUT: return "bounded device wait timed out";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported parameter value";
+  }
+  return "unknown status";
+}
+
+nvfp4_status nvfp4_workspace_status(const void* ws, nvfp4_stream_t stream) {
+  if (!ws) return NVFP4_ERR_INVALID_ARG;
+  int v = 0;
+  NVFP4_CUDA_TRY(cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, as_cuda(stream)));
+  NVFP4_CUDA_TRY(cudaStreamSynchronize(as_cuda(stream)));
+  return static_cast<nvfp4_status>(v);
+}
+
+nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dtype,
+                                      int64_t n_tok, int64_t d, int beta,
+                                      nvfp4_stream_t stream) {
+  if (!H || n_tok < 0 || d < 0 || (n_tok > 0 && !X)) return NVFP4_ERR_INVALID_ARG;
+  if (x_dtype != NVFP4_BF16 && x_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (beta != 0 && beta != 1) return NVFP4_ERR_INVALID_ARG;
+  if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (d == 0) return NVFP4_OK;
+  ProfileScope ps(kPhaseHessian, as_cuda(stream));
+  return launch_hessian_simt(H, X, x_dtype, n_tok, d, beta, as_cuda(stream));
+}
+
+size_t nvfp4_prepare_workspace_size(int64_t d) {
+  if (d < 0) return 0;
+  return prepare_ws_bytes(d);
+}
+
+nvfp4_status nvfp4_gptq_prepare(const float* H, int64_t d, float damp, float* U,
+                                uint8_t* dead, float* lambda_out, void* ws, size_t ws_bytes,
+                                nvfp4_stream_t stream) {
+  if (!H || !U || d < 0 || !(damp >= 0.f)) return NVFP4_ERR_INVALID_ARG;
+  if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (!ws || !aligned256(ws) || ws_bytes < prepare_ws_bytes(d)) return NVFP4_ERR_WORKSPACE;
+  if (d == 0) return NVFP4_OK;
+  ProfileScope ps(kPhasePrepare, as_cuda(stream));
+  return launch_prepare(H, d, damp, U, dead, lambda_out, ws, as_cuda(stream));
+}
+
+size_t nvfp4_quantize_workspace_size(int64_t d_out, int64_t d_in,
+                                     const nvfp4_solve_params* params) {
+  (void)params;
+  if (d_out < 0 || d_in < 0) return 0;
+  return quantize_ws_bytes(d_out, d_in);
+}
+
+nvfp4_status nvfp4_gptq_schur_replay_quantize(
+    const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in, const float* U,
+    const nvfp4_solve_params* params, const uint8_t* dead, uint8_t* codes, uint8_t* scales,
+    float* global_scale, double* err_out, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+  if (d_out < 0 || d_in < 0 || !global_scale) return NVFP4_ERR_INVALID_ARG;
+  if (d_out > 0 && d_in > 0 && (!W || !U || !codes || !scales)) return NVFP4_ERR_INVALID_ARG;
+  if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!params_ok(params)) return NVFP4_ERR_UNSUPPORTED;
+  if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
+  if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(d_out, d_in))
+    return NVFP4_ERR_WORKSPACE;
+  return launch_quantize(W, w_dtype, d_out, d_in, U, dead, codes, scales, global_scale,
+                         err_out, ws, as_cuda(stream));
+}
+
+nvfp4_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales,
+                           const float* global_scale, int64_t d_out, int64_t d_in, void* out,
+                           nvfp4_dtype out_dtype, nvfp4_stream_t stream) {
+  if (d_out < 0 || d_in < 0) return NVFP4_ERR_INVALID_ARG;
+  if (d_out > 0 && d_in > 0 && (!codes || !scales || !global_scale || !out))
+    return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_BF16 && out_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (d_in % 16) return NVFP4_ERR_SHAPE;
+  ProfileScope ps(kPhaseDequant, as_cuda(stream));
+  return launch_dequant(codes, scales, global_scale, d_out, d_in, out, out_dtype,
+                        as_cuda(stream));
+}
+
+size_t nvfp4_layer_error_workspace_size(int64_t d_out, int64_t d_in) {
+  if (d_out < 0 || d_in < 0) return 0;
+  return layer_error_ws_bytes(d_out, d_in);
+}
+
+nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t* codes,
+                               const uint8_t* scales, const float* global_scale,
+                               const float* H, int64_t d_out, int64_t d_in, double* err_out,
+                               void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+  if (d_out < 0 || d_in < 0 || !err_out) return NVFP4_ERR_INVALID_ARG;
+  if (d_out > 0 && d_in > 0 && (!W || !codes || !scales || !global_scale || !H))
+    return NVFP4_ERR_INVALID_ARG;
+  if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
+  if (!ws || !aligned256(ws) || ws_bytes < layer_error_ws_bytes(d_out, d_in))
+    return NVFP4_ERR_WORKSPACE;
+  return launch_layer_error(W, w_dtype, codes, scales, global_scale, H, d_out, d_in, err_out,
+                            ws, as_cuda(stream));
+}
+
+}  // extern "C"

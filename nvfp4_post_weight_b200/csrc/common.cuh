@@ -1,0 +1,104 @@
+// Shared host/device helpers of the NVFP4 GPTQ library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nvfp4pw.h"
+
+namespace nvfp4 {
+
+constexpr int kBlock = 16;        // weights per E4M3 block scale
+constexpr int kCand = 16;         // candidate scales per block
+constexpr int kLazyBatch = 128;   // columns per lazy batch
+constexpr int kNumSMs = 148;      // B200
+
+// Workspace header: the sticky device status word lives in the first 256 bytes.
+constexpr size_t kWsHeader = 256;
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Records the first non-OK status in the sticky word (device side).
+__device__ __forceinline__ void flag_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+inline cudaStream_t as_cuda(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---- launch accounting and optional per-phase event timing (runtime.cu) ----
+enum Phase {
+  kPhaseHessian = 0,
+  kPhasePrepare = 1,
+  kPhaseReplay = 2,
+  kPhaseUpdate = 3,
+  kPhaseDequant = 4,
+  kPhaseOther = 5,
+  kNumPhases = 6
+};
+// Adds n to the library's kernel-launch counter (and to the open phase's).
+void count_launches(int n);
+// While profiling is on, records a CUDA event pair around its lifetime on
+// `st` and charges the launches counted meanwhile to `phase`.
+struct ProfileScope {
+  ProfileScope(int phase, cudaStream_t st);
+  ~ProfileScope();
+  int slot;
+  int prev_phase;
+  cudaStream_t st;
+};
+
+#define NVFP4_LAUNCH_CHECK()                                   \
+  do {                                                         \
+    if (cudaPeekAtLastError() != cudaSuccess) {                \
+      cudaGetLastError();                                      \
+      return NVFP4_ERR_CUDA;                                   \
+    }                                                          \
+  } while (0)
+
+#define NVFP4_CUDA_TRY(x)                                      \
+  do {                                                         \
+    if ((x) != cudaSuccess) {                                  \
+      cudaGetLastError();                                      \
+      return NVFP4_ERR_CUDA;                                   \
+    }                                                          \
+  } while (0)
+
+// ---- kernel launchers implemented in the .cu files -------------------------
+nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
+                            int64_t d, int beta, cudaStream_t st);
+nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,
+                            uint8_t* dead, float* lambda_out, void* ws, cudaStream_t st);
+size_t prepare_ws_bytes(int64_t d);
+nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
+                             const float* U, const uint8_t* dead, uint8_t* codes,
+                             uint8_t* scales, float* sg, double* err, void* ws,
+                             cudaStream_t st);
+size_t quantize_ws_bytes(int64_t d_out, int64_t d_in);
+nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* sg,
+                            int64_t d_out, int64_t d_in, void* out, nvfp4_dtype ot,
+                            cudaStream_t st);
+nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* codes,
+                                const uint8_t* scales, const float* sg, const float* H,
+                                int64_t d_out, int64_t d_in, double* err, void* ws,
+                                cudaStream_t st);
+size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in);
+
+// C = alpha * op(A) * op(B) + beta * C in fp32 on the CUDA cores.  Row-major;
+// op(A) is M x K, op(B) is K x N.  ta/tb: 1 -> the stored matrix is transposed.
+// tri: 0 full; 1 only output tiles on or below the diagonal (row >= col block);
+//      2 only tiles on or above it.
+nvfp4_status sgemm_simt_batched(int M, int N, int K, float alpha, const float* A,
+                                int64_t lda, int64_t sA, int ta, const float* B,
+                                int64_t ldb, int64_t sB, int tb, float beta, float* C,
+                                int64_t ldc, int64_t sC, int tri, int batch,
+                                cudaStream_t st);
+// C -= A B with C, A fp64 and B fp32 (widened exactly), on the CUDA cores.
+// Row-major: A is M x K (lda), B is K x N (ldb), C is M x N (ldc).
+nvfp4_status dgemm_update(int M, int N, int K, const double* A, int64_t lda, const float* B,
+                          int64_t ldb, double* C, int64_t ldc, cudaStream_t st);
+
+nvfp4_status sgemm_simt(int M, int N, int K, float alpha, const float* A, int64_t lda,
+                        int ta, const float* B, int64_t ldb, int tb, float beta, float* C,
+                        int64_t ldc, int tri, cudaStream_t st);
+
+}  // namespace nvfp4

@@ -1,0 +1,357 @@
+// a5-a8: global scale, working copy, Schur Replay block-scale selection inside
+// GPTQ, and the lazy-batch trailing update.
+//
+// "Replay the Curvature" (arXiv 2609.36654v1), Abstract: GPTQ quantizes the
+// columns in order and each quantized column updates the columns after it, so
+// a block scale changes the values the rest of its block is quantized from.
+// Schur Replay scores every candidate scale by replaying those in-block
+// updates and measuring the block error that remains after compensation from
+// the still-unquantized columns; the best candidate is kept.
+//
+// With U the upper factor of H_d^-1 (H_d^-1 = U^T U), quantizing column j of
+// a row leaves delta_j = (v_j - q_j) / U_jj and the later columns absorb
+// delta_j * U[j, i].  delta_j^2 = (v_j - q_j)^2 / U_jj^2 where 1/U_jj^2 is the
+// Schur complement of column j given the columns after it, and the block's
+// sum of delta_j^2 is its exact share of tr((W-Q) H_d (W-Q)^T).
+//
+// Precision: the working copy W~ is kept in fp64 and the replay runs in fp64.
+// The codes are discrete decisions (nearest E2M1 value, argmin over scales)
+// and one flipped code changes every later update of its row, so the values
+// they are taken on must carry more than fp32's 24 bits; the factor U itself
+// is fp32 (its rounding moves no decision on the workloads measured).
+//
+// Layout of the work: columns go in lazy batches of 128.  For one batch the
+// replay kernel walks the batch's 8 blocks for every row (a half-warp per row,
+// lane = candidate scale) with the row's 128 batch values in shared memory,
+// and applies each chosen block's deltas to the rest of the batch; it writes
+// the batch's deltas.  The trailing update then applies the whole batch to
+// every later column at once: W~[:, e:] -= Delta U[batch, e:].
+#include <math.h>
+
+#include "common.cuh"
+#include "nvfp4_format.cuh"
+
+namespace nvfp4 {
+namespace {
+
+struct QuantHeader {   // workspace header (first 256 bytes)
+  int status;
+  unsigned amax_bits;  // max |W| as fp32 bits (non-negative floats order as uints)
+};
+
+struct QuantLayout {
+  QuantHeader* hdr;
+  double* Wt;      // d_out x d_in working copy
+  double* Delta;   // d_out x 128
+  double* rowerr;  // d_out
+};
+
+QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in) {
+  char* p = static_cast<char*>(ws);
+  QuantLayout L;
+  L.hdr = reinterpret_cast<QuantHeader*>(p);
+  size_t off = kWsHeader;
+  L.Wt = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * d_out * d_in);
+  L.Delta = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * d_out * kLazyBatch);
+  L.rowerr = reinterpret_cast<double*>(p + off);
+  return L;
+}
+
+// a5 + a6: W~ = fp64(W) with dead columns zeroed, amax |W~|, non-finite check.
+// Eight consecutive elements per thread step (d_in is a multiple of 16).
+template <typename T>
+__global__ void wprep_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_in,
+                             const uint8_t* __restrict__ dead, double* __restrict__ Wt,
+                             double* __restrict__ rowerr, QuantHeader* hdr) {
+  const int64_t n8 = d_out * d_in / 8;
+  float m = 0.f;
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float v[8];
+    if constexpr (sizeof(T) == 2) {
+      const uint4 raw = reinterpret_cast<const uint4*>(W)[i];
+      const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(u[k] << 16);
+        v[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+      }
+    } else {
+      const float4 a = reinterpret_cast<const float4*>(W)[2 * i];
+      const float4 b = reinterpret_cast<const float4*>(W)[2 * i + 1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    if (dead) {
+      const int64_t c = (i * 8) % d_in;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (dead[c + k]) v[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      bad |= !isfinite(v[k]);
+      m = fmaxf(m, fabsf(v[k]));
+    }
+    double2* o = reinterpret_cast<double2*>(Wt + 8 * i);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] = make_double2(v[2 * k], v[2 * k + 1]);
+  }
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < d_out;
+       r += (int64_t)gridDim.x * blockDim.x)
+    rowerr[r] = 0.0;
+  if (__any_sync(0xffffffffu, bad)) {
+    if ((threadIdx.x & 31) == 0) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&hdr->amax_bits, __float_as_uint(m));
+}
+
+// s_g = amax / (6 * 448) correctly rounded to fp32, 1 when W == 0.
+__global__ void global_scale_kernel(QuantHeader* hdr, float* __restrict__ sg) {
+  const float amax = __uint_as_float(hdr->amax_bits);
+  *sg = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+constexpr int kReplayThreads = 256;                 // 8 warps = 16 rows in flight
+constexpr int kRowsPerCta = kReplayThreads / 16;
+constexpr int kNb = kLazyBatch / kBlock;            // blocks per batch (8)
+constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a batch (36)
+
+// Index of the upper tile (p, q), q >= p, in the packed tile array.
+__device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p) / 2 + q; }
+
+// One candidate's replay of the in-block GPTQ updates (fp64).  v holds the
+// block's 16 current values and is consumed.  Ud points at the block's
+// diagonal 16x16 tile (row-major), invd at its 1/U_jj.  Returns the score
+// sum delta_j^2; delta and the packed code nibbles are written out.
+__device__ __forceinline__ double replay(double (&v)[16], double s, double inv_s,
+                                         const double* __restrict__ Ud,
+                                         const double* __restrict__ invd, double (&dl)[16],
+                                         uint64_t& packed) {
+  double score = 0.0;
+  uint64_t pk = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const double x = __dmul_rn(v[j], inv_s);
+    const double r = e2m1_round_mag(fabs(x));
+    const uint32_t idx = e2m1_index(r);
+    const double sr = x < 0.0 ? -r : r;
+    const uint32_t nib = idx | ((x < 0.0 && idx) ? 8u : 0u);
+    pk |= (uint64_t)nib << (4 * j);
+    const double res = __fma_rn(-sr, s, v[j]);       // v_j - q_j, one rounding
+    const double d = __dmul_rn(res, invd[j]);
+    dl[j] = d;
+    score = __fma_rn(d, d, score);
+#pragma unroll
+    for (int i = j + 1; i < 16; ++i) v[i] = __fma_rn(-d, Ud[j * 16 + i], v[i]);
+  }
+  packed = pk;
+  return score;
+}
+
+// One lazy batch of Schur Replay.  Half-warp = one row; lane hl = candidate hl
+// of the current block.  The batch's upper block-triangular part of U lives in
+// shared memory as 16x16 fp64 tiles, the rows' batch values next to it.
+__global__ void __launch_bounds__(kReplayThreads)
+    schur_replay_batch_kernel(double* __restrict__ Wt, const float* __restrict__ U,
+                              int64_t d_out, int64_t d_in, int c0, int bw,
+                              const float* __restrict__ sg_ptr, uint8_t* __restrict__ codes,
+                              uint8_t* __restrict__ scales, double* __restrict__ Delta,
+                              double* __restrict__ rowerr) {
+  extern __shared__ double4 smem_d4[];
+  double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
+  double* invd = Ut + kUTiles * 256;                         // 128
+  double* rows = invd + kLazyBatch;                          // kRowsPerCta x 128
+  const int nblk = bw / kBlock;
+  for (int idx = threadIdx.x; idx < kUTiles * 256; idx += blockDim.x) {
+    const int t = idx >> 8, e = idx & 255;
+    // recover (p, q) of tile t
+    int p = 0;
+    while (p + 1 < kNb && utile(p + 1, p + 1) <= t) ++p;
+    const int q = p + (t - utile(p, p));
+    const int i = e >> 4, j = e & 15;
+    const int gi = 16 * p + i, gj = 16 * q + j;
+    double u = 0.0;
+    if (p < nblk && q < nblk && gj >= gi) u = (double)U[(int64_t)(c0 + gi) * d_in + c0 + gj];
+    Ut[idx] = u;
+  }
+  for (int i = threadIdx.x; i < bw; i += blockDim.x)
+    invd[i] = 1.0 / (double)U[(int64_t)(c0 + i) * d_in + c0 + i];
+  __syncthreads();
+
+  const double sg = (double)*sg_ptr;
+  const double six_sg = 6.0 * sg;
+  const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
+  const int warp = threadIdx.x >> 5;
+  const int rloc = warp * 2 + half;
+  double* row = rows + rloc * kLazyBatch;
+  const unsigned FULL = 0xffffffffu;
+
+  for (int64_t rb = (int64_t)blockIdx.x * kRowsPerCta; rb < d_out;
+       rb += (int64_t)gridDim.x * kRowsPerCta) {
+    const int64_t r = rb + rloc;
+    const bool valid = r < d_out;
+    // stage the row's batch values
+    for (int c = hl; c < bw; c += 16) row[c] = valid ? Wt[r * d_in + c0 + c] : 0.0;
+    __syncwarp();
+    double rowsum = 0.0;
+
+    for (int b = 0; b < nblk; ++b) {
+      double v[16];
+      double amax = 0.0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        v[i] = row[16 * b + i];
+        amax = fmax(amax, fabs(v[i]));
+      }
+      const int k0 = max(e4m3_code_rn(amax / six_sg), 1);
+      const int lo = min(max(k0 - 8, 1), 127 - kCand);
+      const double s = e4m3_value(lo + hl) * sg;   // exact: 4 + 24 significant bits
+      const double inv_s = 1.0 / s;
+      const double* Ud = Ut + utile(b, b) * 256;
+      const double* idb = invd + 16 * b;
+
+      double dl[16];
+      uint64_t pk;
+      const double score = replay(v, s, inv_s, Ud, idb, dl, pk);
+
+      // argmin over the 16 candidates, ties to the lower code
+      double best = score;
+      int bl = hl;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const double os = __shfl_xor_sync(FULL, best, o, 16);
+        const int ol = __shfl_xor_sync(FULL, bl, o, 16);
+        if (os < best || (os == best && ol < bl)) {
+          best = os;
+          bl = ol;
+        }
+      }
+      const bool live = amax > 0.0;
+      __syncwarp();
+      if (hl == bl) {
+        // the winner publishes its deltas in place of the block's values
+#pragma unroll
+        for (int j = 0; j < 16; ++j) row[16 * b + j] = live ? dl[j] : 0.0;
+        if (valid) {
+          *reinterpret_cast<uint64_t*>(codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
+              live ? pk : 0ull;
+          scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
+        }
+      }
+      if (live) rowsum += best;
+      __syncwarp();
+      // later columns of the batch absorb the chosen block's deltas
+      if (b + 1 < nblk) {
+        double d[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) d[j] = row[16 * b + j];
+        for (int q = b + 1; q < nblk; ++q) {
+          const double* Uq = Ut + utile(b, q) * 256 + hl;
+          double acc = row[16 * q + hl];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc = __fma_rn(-d[j], Uq[16 * j], acc);
+          row[16 * q + hl] = acc;
+        }
+      }
+      __syncwarp();
+    }
+    if (valid) {
+      for (int c = hl; c < bw; c += 16) Delta[r * kLazyBatch + c] = row[c];
+      if (hl == 0) rowerr[r] += rowsum;
+    }
+    __syncwarp();
+  }
+}
+
+__global__ void sum_rows_kernel(const double* __restrict__ rowerr, int64_t n,
+                                double* __restrict__ out) {
+  __shared__ double part[32];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += rowerr[i];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    s = (threadIdx.x < (blockDim.x >> 5)) ? part[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x == 0) *out = s;
+  }
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  return (int)(b < 8 * kNumSMs ? (b < 1 ? 1 : b) : 8 * kNumSMs);
+}
+
+constexpr size_t kReplaySmem =
+    sizeof(double) * (kUTiles * 256 + kLazyBatch + kRowsPerCta * kLazyBatch);
+
+}  // namespace
+
+size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
+  return kWsHeader + align256(sizeof(double) * d_out * d_in) +
+         align256(sizeof(double) * d_out * kLazyBatch) + align256(sizeof(double) * d_out);
+}
+
+nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
+                             const float* U, const uint8_t* dead, uint8_t* codes,
+                             uint8_t* scales, float* sg, double* err, void* ws,
+                             cudaStream_t st) {
+  QuantLayout L = quant_layout(ws, d_out, d_in);
+  NVFP4_CUDA_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(QuantHeader), st));
+  if (d_out == 0 || d_in == 0) {
+    global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, sg);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(1);
+    if (err) NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
+    return NVFP4_OK;
+  }
+  const int g = grid_for(d_out * d_in / 8, 256);
+  if (wt == NVFP4_BF16)
+    wprep_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), d_out, d_in,
+                                              dead, L.Wt, L.rowerr, L.hdr);
+  else
+    wprep_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), d_out, d_in, dead,
+                                           L.Wt, L.rowerr, L.hdr);
+  NVFP4_LAUNCH_CHECK();
+  global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, sg);
+  NVFP4_LAUNCH_CHECK();
+  count_launches(2);
+
+  NVFP4_CUDA_TRY(cudaFuncSetAttribute(schur_replay_batch_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kReplaySmem));
+  const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
+  const int rgrid = (int)(row_groups < 2 * kNumSMs ? row_groups : 2 * kNumSMs);
+  for (int64_t c0 = 0; c0 < d_in; c0 += kLazyBatch) {
+    const int bw = (int)((d_in - c0) < kLazyBatch ? (d_in - c0) : kLazyBatch);
+    {
+      ProfileScope ps(kPhaseReplay, st);
+      schur_replay_batch_kernel<<<rgrid, kReplayThreads, kReplaySmem, st>>>(
+          L.Wt, U, d_out, d_in, (int)c0, bw, sg, codes, scales, L.Delta, L.rowerr);
+      NVFP4_LAUNCH_CHECK();
+      count_launches(1);
+    }
+    const int64_t e = c0 + bw;
+    if (e < d_in) {
+      ProfileScope ps(kPhaseUpdate, st);
+      // W~[:, e:] -= Delta[:, :bw] U[c0:c0+bw, e:]
+      nvfp4_status s = dgemm_update((int)d_out, (int)(d_in - e), bw, L.Delta, kLazyBatch,
+                                    U + c0 * d_in + e, d_in, L.Wt + e, d_in, st);
+      if (s != NVFP4_OK) return s;
+    }
+  }
+  if (err) {
+    sum_rows_kernel<<<1, 1024, 0, st>>>(L.rowerr, d_out, err);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(1);
+  }
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4

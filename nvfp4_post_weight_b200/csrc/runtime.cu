@@ -1,0 +1,128 @@
+// Launch accounting and optional per-phase CUDA-event timing.
+//
+// Every kernel launch of the library is counted (nvfp4_launch_count), so a
+// caller can check how many of the library's kernels a piece of work ran.
+// While profiling is on, each launcher's ProfileScope records a CUDA event
+// pair on the launching stream; nvfp4_profile_end() waits for the events and
+// returns, per phase, the summed device time and the number of launches.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+struct Record {
+  int phase;
+  cudaEvent_t a, b;
+};
+
+std::mutex g_mu;
+std::atomic<long long> g_launches{0};
+std::atomic<long long> g_phase_launches[kNumPhases];
+std::atomic<bool> g_profiling{false};
+std::vector<Record> g_records;
+std::vector<cudaEvent_t> g_pool;
+thread_local int t_phase = -1;
+
+cudaEvent_t get_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+}  // namespace
+
+void count_launches(int n) {
+  g_launches.fetch_add(n, std::memory_order_relaxed);
+  const int p = t_phase >= 0 ? t_phase : kPhaseOther;
+  g_phase_launches[p].fetch_add(n, std::memory_order_relaxed);
+}
+
+ProfileScope::ProfileScope(int phase, cudaStream_t s) : slot(-1), prev_phase(t_phase), st(s) {
+  t_phase = phase;
+  if (!g_profiling.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Record r{phase, get_event(), get_event()};
+  if (!r.a || !r.b) return;
+  if (cudaEventRecord(r.a, st) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  slot = (int)g_records.size();
+  g_records.push_back(r);
+}
+
+ProfileScope::~ProfileScope() {
+  t_phase = prev_phase;
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (slot < (int)g_records.size() && cudaEventRecord(g_records[slot].b, st) != cudaSuccess) {
+    cudaGetLastError();
+    g_records[slot].phase = -1;
+  }
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+long long nvfp4_launch_count(void) { return g_launches.load(); }
+
+nvfp4_status nvfp4_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& r : g_records) {
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_records.clear();
+  for (int p = 0; p < kNumPhases; ++p) g_phase_launches[p].store(0);
+  g_profiling.store(true);
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_profile_end(double* ms, long long* launches, int n_phases) {
+  if (n_phases < 0 || (n_phases > 0 && (!ms || !launches))) return NVFP4_ERR_INVALID_ARG;
+  g_profiling.store(false);
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int p = 0; p < n_phases; ++p) {
+    ms[p] = 0.0;
+    launches[p] = p < kNumPhases ? g_phase_launches[p].load() : 0;
+  }
+  nvfp4_status st = NVFP4_OK;
+  for (auto& r : g_records) {
+    if (r.phase < 0) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) {
+      cudaGetLastError();
+      st = NVFP4_ERR_CUDA;
+      continue;
+    }
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      st = NVFP4_ERR_CUDA;
+      continue;
+    }
+    if (r.phase < n_phases) ms[r.phase] += (double)t;
+  }
+  for (auto& r : g_records) {
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_records.clear();
+  return st;
+}
+
+}  // extern "C"
