@@ -1,0 +1,373 @@
+"""Benchmark of the per-layer NVFP4 GPTQ + Schur Replay solve on B200.
+
+One step = one whole solve of a synthetic layer through the C ABI, inputs
+already resident in HBM: Hessian H = X^T X, damping + upper Cholesky factor of
+H_d^-1, global scale + Schur Replay GPTQ (codes, E4M3 scales, sum delta^2),
+dequantization to bf16 and the layer error tr((W-Q) H (W-Q)^T).
+
+Prints ONE JSON line (rank 0).  `value` is weights quantized per second over
+the whole step, summed over ranks (each rank solves its own layer: weak
+scaling, no collective on the data path).  `--impl reference` times the fp64
+CPU oracle instead, on a bounded row sample of the same workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GPTQ+Schur Replay layer solve ms & weights/s; Hessian TFLOP/s"
+UNIT = "weights/s"
+DEFAULT_WORKLOAD = "attn_massive_4096x4096"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+N_SM = 148
+FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def workload(name):
+    from nvfp4_post_weight_b200 import synth
+    if name == "attn_massive_4096x4096":
+        return synth.attn_massive()
+    if name == "small_outlier_256x256":
+        return synth.small_outlier()
+    if name == "mlp_down_silu_4096x14336":
+        return synth.mlp_down_silu()
+    raise SystemExit(f"unknown workload {name}")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v
+                          and "Not" not in v})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def phase_work(d_out, d_in, n_tok):
+    """Algorithmic work per phase of one step (flops or bytes)."""
+    upd = 0
+    for c0 in range(0, d_in, 128):
+        e = min(c0 + 128, d_in)
+        upd += 2 * d_out * (e - c0) * (d_in - e)
+    return {
+        "hessian_flops": n_tok * d_in * (d_in + 1),          # symmetric half, 2 flops per MAC
+        "prepare_flops": 2 * d_in ** 3 // 3,
+        "update_flops": upd,
+        "replay_bytes": d_out * d_in * (8 + 8 + 0.5) + d_out * d_in / 16,
+        "dequant_bytes": d_out * d_in * (0.5 + 2) + d_out * d_in / 16,
+    }
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from nvfp4_post_weight_b200 import binding as B
+    from nvfp4_post_weight_b200.layer import LayerSolver
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    W, X = workload(args.workload)
+    d_out, d_in = W.shape
+    n_tok = X.shape[0]
+    Wd, Xd = W.to(dev), X.to(dev)
+    solver = LayerSolver(d_out, d_in, dev, out_dtype=torch.bfloat16)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        solver.step(Wd, Xd)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    st = solver.status()
+    if st != (0, 0):
+        raise SystemExit(f"device status after warm-up: {st}")
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        tdist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    n0 = B.lib().nvfp4_launch_count()
+    B.lib().nvfp4_profile_begin()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    import ctypes
+    ms_ph = (ctypes.c_double * 6)()
+    ln_ph = (ctypes.c_longlong * 6)()
+    B.lib().nvfp4_profile_end(ms_ph, ln_ph, 6)
+    launches = B.lib().nvfp4_launch_count() - n0
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    if dist:
+        t = torch.tensor([step_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        step_ms = float(t.item())
+        tdist.barrier()
+
+    # end to end through the C ABI from pinned host buffers: H2D of W and X,
+    # the solve, D2H of codes, scales and the global scale
+    Wh, Xh = W.pin_memory(), X.pin_memory()
+    codes_h = torch.empty(solver.codes.shape, dtype=torch.uint8).pin_memory()
+    scales_h = torch.empty(solver.scales.shape, dtype=torch.uint8).pin_memory()
+    sg_h = torch.empty(1, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        Wd.copy_(Wh, non_blocking=True)
+        Xd.copy_(Xh, non_blocking=True)
+        step()
+        codes_h.copy_(solver.codes, non_blocking=True)
+        scales_h.copy_(solver.scales, non_blocking=True)
+        sg_h.copy_(solver.s_g, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev2[i][0].record(stream)
+        e2e_step()
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    wk = phase_work(d_out, d_in, n_tok)
+    names = ["hessian", "prepare", "replay", "update", "dequant", "other"]
+    ph_ms = {n: ms_ph[i] / args.steps for i, n in enumerate(names[:5])}
+    ph_launch = {n: ln_ph[i] // args.steps for i, n in enumerate(names)}
+    sm_ghz = peaks.get("sm_max_mhz", 1965.0) / 1e3
+    fp64_peak = N_SM * FP64_LANES_PER_SM * 2 * sm_ghz / 1e3    # TFLOP/s
+    fp32_peak = N_SM * FP32_LANES_PER_SM * 2 * sm_ghz / 1e3
+    bf16_peak = peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+    # per-phase roofline (what bounds each phase in this build)
+    rl = {
+        "hessian": ("alu", wk["hessian_flops"] / (ph_ms["hessian"] * 1e9), fp32_peak, "TFLOP/s"),
+        "prepare": ("alu", wk["prepare_flops"] / (ph_ms["prepare"] * 1e9), fp32_peak, "TFLOP/s"),
+        "update": ("alu", wk["update_flops"] / (ph_ms["update"] * 1e9), fp64_peak, "TFLOP/s"),
+        "replay": ("hbm", wk["replay_bytes"] / (ph_ms["replay"] * 1e6), hbm, "GB/s"),
+        "dequant": ("hbm", wk["dequant_bytes"] / (ph_ms["dequant"] * 1e6), hbm, "GB/s"),
+    }
+    dom = max(rl, key=lambda n: ph_ms[n])
+    bound, ach, peak, unit = rl[dom]
+    solve_ms = ph_ms["prepare"] + ph_ms["replay"] + ph_ms["update"]
+    weights = d_out * d_in
+    out = {
+        "metric": METRIC, "value": world * weights / (step_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in; f32 H and U; f64 solve", "data": "synthetic",
+        "config": {"workload": args.workload, "d_out": d_out, "d_in": d_in, "n_tok": n_tok,
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "parallelism": f"{world} independent layer solves (one per GPU)"},
+        "layer_solve_ms": solve_ms,
+        "solve_weights_per_s": weights / (solve_ms / 1e3),
+        "hessian_tflops": {"algorithmic_syrk_half": wk["hessian_flops"] / (ph_ms["hessian"] * 1e9),
+                           "conventional_2Nd2": 2 * n_tok * d_in * d_in / (ph_ms["hessian"] * 1e9)},
+        "phase_ms": ph_ms, "phase_launches": ph_launch,
+        "phase_roofline": {n: {"bound": b, "achieved": a, "peak": p, "unit": u, "frac": a / p}
+                           for n, (b, a, p, u) in rl.items()},
+        "roofline": {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                     "frac": ach / peak, "traffic": None,
+                     "peak_source": peaks["source"] if unit == "GB/s" else
+                     "derived: 148 SMs x lanes x 2 x max SM clock"},
+        "e2e": {"value": world * weights / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": W.numel() * W.element_size() + X.numel() * X.element_size(),
+                "d2h_bytes_per_step": codes_h.numel() + scales_h.numel() + 4},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_step(W64, X64, rows):
+    """One bounded oracle sample: the full Hessian and factor, the solve and
+    dequant of `rows`.  Returns (seconds, seconds scaled to the whole layer)."""
+    import oracle as O
+    t0 = time.perf_counter()
+    H = O.hessian(X64)
+    Hd, dead, lam = O.damp(H)
+    U = O.inverse_cholesky_upper(Hd)
+    sg = O.global_scale(W64)
+    t1 = time.perf_counter()
+    res = O.schur_replay_gptq(W64[rows], U, sg, dead)
+    O.dequant(res["codes"], res["scales"], sg, "bf16")
+    t2 = time.perf_counter()
+    full = (t1 - t0) + (t2 - t1) * W64.shape[0] / len(rows)
+    return t2 - t0, full
+
+
+def oracle_inputs(name, n_rows):
+    W, X = workload(name)
+    W64 = W.double().numpy()
+    X64 = X.double().numpy()
+    rows = np.sort(np.random.default_rng(7).choice(W64.shape[0], min(n_rows, W64.shape[0]),
+                                                   replace=False))
+    return W64, X64, rows
+
+
+def cpu_baseline(name, n_rows=128):
+    W64, X64, rows = oracle_inputs(name, n_rows)
+    wall, full = oracle_step(W64, X64, rows)
+    return {"value": W64.size / full, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"full fp64 Hessian and factor; solve + dequant of {len(rows)} of "
+                       f"{W64.shape[0]} rows, scaled by rows ({wall:.1f} s wall)")}
+
+
+def run_reference(args):
+    W64, X64, rows = oracle_inputs(args.workload, args.ref_rows)
+    for _ in range(args.warmup):
+        oracle_step(W64, X64, rows)
+    fulls = [oracle_step(W64, X64, rows)[1] for _ in range(args.steps)]
+    full = float(np.mean(fulls))
+    v = W64.size / full
+    d_out, d_in = W64.shape
+    return {
+        "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": args.workload, "d_out": d_out, "d_in": d_in,
+                   "n_tok": X64.shape[0], "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": (f"each step: full fp64 Hessian and factor; solve + dequant "
+                                    f"of {len(rows)} of {d_out} rows, scaled by rows")},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -29,6 +29,8 @@
  *     traps or spins without a bound.
  *   - Sizes are int64_t; negative sizes are NVFP4_ERR_INVALID_ARG.  The
  *     quantized dimension (d, d_in) must be a multiple of 16.
+ *   - Alignment: W and dequant's `out` 16 bytes, packed codes 8 bytes,
+ *     workspaces 256 bytes (NVFP4_ERR_INVALID_ARG / _WORKSPACE otherwise).
  */
 #ifndef NVFP4PW_H
 #define NVFP4PW_H

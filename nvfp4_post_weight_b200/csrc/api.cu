@@ -19,6 +19,7 @@ bool params_ok(const nvfp4_solve_params* p) {
 }
 
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Largest dimension this build accepts; keeps every int index below 2^31.
 constexpr int64_t kMaxDim = 1 << 17;
@@ -101,6 +102,7 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
     float* global_scale, double* err_out, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
   if (d_out < 0 || d_in < 0 || !global_scale) return NVFP4_ERR_INVALID_ARG;
   if (d_out > 0 && d_in > 0 && (!W || !U || !codes || !scales)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 8)) return NVFP4_ERR_INVALID_ARG;
   if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
   if (!params_ok(params)) return NVFP4_ERR_UNSUPPORTED;
   if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
@@ -116,6 +118,7 @@ nvfp4_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales,
   if (d_out < 0 || d_in < 0) return NVFP4_ERR_INVALID_ARG;
   if (d_out > 0 && d_in > 0 && (!codes || !scales || !global_scale || !out))
     return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 8) || !aligned(out, 16)) return NVFP4_ERR_INVALID_ARG;
   if (out_dtype != NVFP4_BF16 && out_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
   if (d_in % 16) return NVFP4_ERR_SHAPE;
   ProfileScope ps(kPhaseDequant, as_cuda(stream));
@@ -135,6 +138,7 @@ nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t
   if (d_out < 0 || d_in < 0 || !err_out) return NVFP4_ERR_INVALID_ARG;
   if (d_out > 0 && d_in > 0 && (!W || !codes || !scales || !global_scale || !H))
     return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 8)) return NVFP4_ERR_INVALID_ARG;
   if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
   if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
   if (!ws || !aligned256(ws) || ws_bytes < layer_error_ws_bytes(d_out, d_in))

@@ -1,0 +1,304 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Every comparison feeds both sides the same seeded inputs.  Discrete outputs
+(E2M1 codes, E4M3 scales, the global scale) must match bit for bit on small
+layers and follow the near-tie rule of tests/parity.py on large ones; the
+Hessian must be within 1e-4 relative Frobenius and the layer error
+tr((W-Q) H (W-Q)^T) within 1e-4 relative.
+
+Method: "Replay the Curvature: Accurate and Scalable NVFP4 Quantization for
+Large Language Model Inference", Abstract (NVFP4 format, GPTQ column updates,
+Schur Replay block-scale selection).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_post_weight_b200 import binding as B
+from nvfp4_post_weight_b200 import synth
+from nvfp4_post_weight_b200.layer import LayerSolver
+from parity import classify, unpack_codes, pack_codes
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def rel_frob(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def f64(t):
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def gpu_quantize(W, U32):
+    """Quantize W (torch CPU tensor, bf16/fp32) with a given fp32 U on the GPU."""
+    d_out, d_in = W.shape
+    Wd = W.to(DEV)
+    Ud = torch.as_tensor(U32, dtype=torch.float32).to(DEV)
+    codes = torch.empty((d_out, d_in // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((d_out, d_in // 16), dtype=torch.uint8, device=DEV)
+    sg = torch.empty(1, dtype=torch.float32, device=DEV)
+    err = torch.empty(1, dtype=torch.float64, device=DEV)
+    ws = B.workspace(B.nvfp4_quantize_workspace_size(d_out, d_in), DEV)
+    B.nvfp4_gptq_schur_replay_quantize(Wd, Ud, codes, scales, sg, err, None, ws)
+    torch.cuda.synchronize()
+    assert B.nvfp4_workspace_status(ws) == 0
+    return (unpack_codes(codes.cpu().numpy()), scales.cpu().numpy().astype(np.int64),
+            float(sg.item()), float(err.item()))
+
+
+def gpu_solve(W, X, out_dtype=torch.float32):
+    d_out, d_in = W.shape
+    s = LayerSolver(d_out, d_in, DEV, out_dtype=out_dtype)
+    Wd, Xd = W.to(DEV), X.to(DEV)
+    s.step(Wd, Xd)
+    torch.cuda.synchronize()
+    assert s.status() == (0, 0)
+    return s
+
+
+# --------------------------------------------------------------------------
+# a9 dequant: bit-exact against the exact product rounded once
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d_out,d_in", [(1, 16), (37, 48), (256, 4096)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_dequant_bitexact(d_out, d_in, out):
+    rng = np.random.default_rng(d_out * 7 + d_in)
+    codes = rng.integers(0, 16, size=(d_out, d_in))
+    scales = rng.integers(0, 127, size=(d_out, d_in // 16))
+    for sg in (np.float32(1.0), np.float32(3.7e-5), np.float32(rng.uniform(1e-6, 1e3)),
+               np.float32(1e-30)):
+        c = torch.from_numpy(pack_codes(codes)).to(DEV)
+        s = torch.from_numpy(scales.astype(np.uint8)).to(DEV)
+        g = torch.tensor([sg], dtype=torch.float32, device=DEV)
+        dt = torch.float32 if out == "f32" else torch.bfloat16
+        Q = torch.empty((d_out, d_in), dtype=dt, device=DEV)
+        B.nvfp4_dequant(c, s, g, Q)
+        want = O.dequant(codes, scales, sg, np.float32 if out == "f32" else "bf16")
+        got = Q.float().cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), (sg, out)
+
+
+# --------------------------------------------------------------------------
+# a1 Hessian
+# --------------------------------------------------------------------------
+def test_hessian_fp32_small_outlier():
+    W, X = synth.small_outlier()
+    H = torch.empty((256, 256), dtype=torch.float32, device=DEV)
+    B.nvfp4_hessian_accumulate(H, X.to(DEV), 0)
+    torch.cuda.synchronize()
+    Href = O.hessian(X.double().numpy())
+    assert rel_frob(H.cpu().numpy(), Href) < 1e-5
+    assert np.array_equal(H.cpu().numpy(), H.cpu().numpy().T)
+
+
+@pytest.mark.parametrize("n_tok,d", [(1000, 208), (1, 16), (333, 512)])
+def test_hessian_bf16_ragged_and_accumulate(n_tok, d):
+    rng = np.random.default_rng(n_tok + d)
+    X1 = torch.from_numpy(rng.standard_normal((n_tok, d)).astype(np.float32)).bfloat16()
+    X2 = torch.from_numpy(rng.standard_normal((n_tok // 2 + 1, d)).astype(np.float32)).bfloat16()
+    H = torch.full((d, d), float("nan"), dtype=torch.float32, device=DEV)
+    B.nvfp4_hessian_accumulate(H, X1.to(DEV), 0)
+    B.nvfp4_hessian_accumulate(H, X2.to(DEV), 1)
+    torch.cuda.synchronize()
+    Href = O.hessian(X1.double().numpy()) + O.hessian(X2.double().numpy())
+    assert rel_frob(H.cpu().numpy(), Href) < 1e-5
+
+
+def test_hessian_zero_tokens_zeroes_h():
+    H = torch.full((32, 32), 5.0, dtype=torch.float32, device=DEV)
+    X = torch.empty((0, 32), dtype=torch.bfloat16, device=DEV)
+    B.nvfp4_hessian_accumulate(H, X, 0)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(H).item() == 0
+
+
+# --------------------------------------------------------------------------
+# a2-a4 prepare
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [16, 208, 256, 1040])
+def test_prepare_factor(d):
+    rng = np.random.default_rng(d)
+    n = 2 * d
+    X = rng.standard_normal((n, d)) * rng.lognormal(0.0, 1.0, size=d)
+    H32 = (X.T @ X).astype(np.float32)
+    H = torch.from_numpy(H32).to(DEV)
+    U = torch.full((d, d), float("nan"), dtype=torch.float32, device=DEV)
+    dead = torch.empty(d, dtype=torch.uint8, device=DEV)
+    lam = torch.empty(1, dtype=torch.float32, device=DEV)
+    ws = B.workspace(B.nvfp4_prepare_workspace_size(d), DEV)
+    B.nvfp4_gptq_prepare(H, 0.01, U, dead, lam, ws)
+    torch.cuda.synchronize()
+    assert B.nvfp4_workspace_status(ws) == 0
+    Hd, dd, lam_ref = O.damp(H32.astype(np.float64))
+    Uref = O.inverse_cholesky_upper(Hd)
+    Ug = U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0.0)
+    assert np.all(np.diag(Ug) > 0)
+    assert rel_frob(Ug, Uref) < 1e-4
+    assert abs(lam.item() - lam_ref) <= 1e-6 * lam_ref
+    assert not dead.cpu().numpy().any()
+
+
+def test_prepare_dead_column():
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((64, 48))
+    X[:, 7] = 0.0
+    H32 = (X.T @ X).astype(np.float32)
+    H = torch.from_numpy(H32).to(DEV)
+    U = torch.empty((48, 48), dtype=torch.float32, device=DEV)
+    dead = torch.empty(48, dtype=torch.uint8, device=DEV)
+    ws = B.workspace(B.nvfp4_prepare_workspace_size(48), DEV)
+    B.nvfp4_gptq_prepare(H, 0.01, U, dead, None, ws)
+    torch.cuda.synchronize()
+    Hd, dd, _ = O.damp(H32.astype(np.float64))
+    assert np.array_equal(dead.cpu().numpy().astype(bool), dd)
+    assert rel_frob(U.cpu().numpy(), O.inverse_cholesky_upper(Hd)) < 1e-4
+
+
+def test_prepare_not_pd_sets_status():
+    d = 32
+    H = -torch.eye(d, dtype=torch.float32, device=DEV)
+    U = torch.empty((d, d), dtype=torch.float32, device=DEV)
+    ws = B.workspace(B.nvfp4_prepare_workspace_size(d), DEV)
+    B.nvfp4_gptq_prepare(H, 0.01, U, None, None, ws)
+    assert B.nvfp4_workspace_status(ws) == 5
+
+
+# --------------------------------------------------------------------------
+# a5-a8 quantize, given the oracle's factor (isolates the solve)
+# --------------------------------------------------------------------------
+def test_quantize_given_oracle_factor_bitexact_small_outlier():
+    W, X = synth.small_outlier()
+    W64 = W.double().numpy()
+    H = O.hessian(X.double().numpy())
+    Hd, dead, _ = O.damp(H)
+    U32 = O.inverse_cholesky_upper(Hd).astype(np.float32)
+    sg = O.global_scale(W64)
+    ref = O.schur_replay_gptq(W64, U32.astype(np.float64), sg)
+    codes, scales, sg_gpu, err = gpu_quantize(W, U32)
+    assert np.float32(sg_gpu) == sg
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+    assert abs(err - ref["err_sum"]) <= 1e-9 * ref["err_sum"]
+
+
+@pytest.mark.parametrize("d_out,d_in", [(1, 16), (33, 144), (5, 272), (17, 128)])
+@pytest.mark.parametrize("wdt", [torch.float32, torch.bfloat16])
+def test_quantize_shapes_bitexact(d_out, d_in, wdt):
+    rng = np.random.default_rng(d_out * 1000 + d_in)
+    W = torch.from_numpy(rng.normal(0, 0.02, size=(d_out, d_in)).astype(np.float32)).to(wdt)
+    X = rng.standard_normal((3 * d_in, d_in)) * rng.lognormal(0, 1, size=d_in)
+    Hd, _, _ = O.damp(X.T @ X)
+    U32 = O.inverse_cholesky_upper(Hd).astype(np.float32)
+    W64 = W.double().numpy()
+    sg = O.global_scale(W64)
+    ref = O.schur_replay_gptq(W64, U32.astype(np.float64), sg)
+    codes, scales, sg_gpu, _ = gpu_quantize(W, U32)
+    assert np.float32(sg_gpu) == sg
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+
+
+def test_quantize_zero_rows_blocks_and_all_zero():
+    rng = np.random.default_rng(11)
+    W64 = rng.normal(0, 0.02, size=(6, 64))
+    W64[2] = 0.0
+    W64[4, 16:32] = 0.0
+    W = torch.from_numpy(W64.astype(np.float32))
+    U32 = np.triu(rng.uniform(0.1, 0.3, size=(64, 64))).astype(np.float32)
+    U32[np.diag_indices(64)] = rng.uniform(0.5, 1.5, size=64).astype(np.float32)
+    sg = O.global_scale(W.double().numpy())
+    ref = O.schur_replay_gptq(W.double().numpy(), U32.astype(np.float64), sg)
+    codes, scales, sg_gpu, _ = gpu_quantize(W, U32)
+    assert np.array_equal(scales, ref["scales"]) and np.array_equal(codes, ref["codes"])
+    assert scales[2].sum() == 0 and codes[2].sum() == 0
+    codes, scales, sg_gpu, err = gpu_quantize(torch.zeros((3, 32)), U32[:32, :32])
+    assert sg_gpu == 1.0 and scales.sum() == 0 and codes.sum() == 0 and err == 0.0
+
+
+def test_quantize_empty_rows():
+    U = torch.eye(32, dtype=torch.float32, device=DEV)
+    W = torch.empty((0, 32), dtype=torch.bfloat16, device=DEV)
+    codes = torch.empty((0, 16), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((0, 2), dtype=torch.uint8, device=DEV)
+    sg = torch.zeros(1, dtype=torch.float32, device=DEV)
+    ws = B.workspace(B.nvfp4_quantize_workspace_size(0, 32), DEV)
+    B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws)
+    torch.cuda.synchronize()
+    assert sg.item() == 1.0
+
+
+def test_quantize_errors():
+    U = torch.eye(32, dtype=torch.float32, device=DEV)
+    W = torch.zeros((4, 24), dtype=torch.float32, device=DEV)
+    codes = torch.empty((4, 16), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((4, 2), dtype=torch.uint8, device=DEV)
+    sg = torch.empty(1, dtype=torch.float32, device=DEV)
+    ws = B.workspace(B.nvfp4_quantize_workspace_size(4, 32), DEV)
+    with pytest.raises(B.Nvfp4Error) as e:
+        B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws)
+    assert e.value.code == 2
+    W = torch.zeros((4, 32), dtype=torch.float32, device=DEV)
+    with pytest.raises(B.Nvfp4Error) as e:
+        B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws[:64])
+    assert e.value.code == 3
+    W[1, 3] = float("nan")
+    B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws)
+    assert B.nvfp4_workspace_status(ws) == 4
+
+
+# --------------------------------------------------------------------------
+# whole solve: small layer bit-exact, full-size layer on a row sample
+# --------------------------------------------------------------------------
+def test_solve_small_outlier_bitexact():
+    W, X = synth.small_outlier()
+    ref = O.solve_layer(W.double().numpy(), X.double().numpy())
+    s = gpu_solve(W, X)
+    assert rel_frob(s.H.cpu().numpy(), ref["H"]) < 1e-4
+    assert np.float32(s.s_g.item()) == ref["s_g"]
+    scales = s.scales.cpu().numpy().astype(np.int64)
+    codes = unpack_codes(s.codes.cpu().numpy())
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+    Q = s.Q.cpu().numpy()
+    assert np.array_equal(Q.view(np.uint32), O.dequant(codes, scales, ref["s_g"]).view(np.uint32))
+    L = ref["layer_error"]
+    assert abs(s.layer_err.item() - L) <= 1e-4 * L
+    L_gpu_codes = O.layer_error(ref["W"], O.dequant(codes, scales, ref["s_g"]).astype(np.float64),
+                                ref["H"])
+    assert abs(L_gpu_codes - L) <= 1e-4 * L
+    # the solve's sum of delta^2 is the damped-Hessian error
+    Ld = O.layer_error(ref["W"], ref["q"], ref["H_d"])
+    assert abs(s.err.item() - Ld) <= 1e-4 * Ld
+
+
+def test_solve_attn_4096_row_sample():
+    """Full-size attention-projection layer (4096 x 4096, 4096 tokens), solved
+    whole on the GPU in the benchmark's configuration; the oracle solves a
+    seeded sample of 192 rows (rows are independent given U)."""
+    W, X = synth.attn_massive()
+    s = gpu_solve(W, X, out_dtype=torch.bfloat16)
+    Xn = X.double().numpy()
+    H = O.hessian(Xn)
+    assert rel_frob(s.H.cpu().numpy(), H) < 1e-4
+    Hd, dead, lam = O.damp(H)
+    U = O.inverse_cholesky_upper(Hd)
+    W64 = W.double().numpy()
+    sg = O.global_scale(W64)
+    assert np.float32(s.s_g.item()) == sg
+    rows = np.sort(np.random.default_rng(101).choice(W64.shape[0], 192, replace=False))
+    ref = O.schur_replay_gptq(W64[rows], U, sg, return_diag=True)
+    codes = unpack_codes(s.codes.cpu().numpy()[rows])
+    scales = s.scales.cpu().numpy()[rows].astype(np.int64)
+    c = classify(ref, U, sg, codes, scales, rows)
+    assert c["frac"] <= 1e-3, c
+    assert not c["bad_first"], c
+    Q = O.dequant(codes, scales, sg).astype(np.float64)
+    L_gpu = O.layer_error(W64[rows], Q, H)
+    L_ref = O.layer_error(W64[rows], ref["q"], H)
+    assert abs(L_gpu - L_ref) <= 1e-4 * L_ref
