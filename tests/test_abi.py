@@ -1,0 +1,70 @@
+"""The C-ABI library loads and exports every function its public header
+declares (no GPU needed: nothing here launches a kernel), and the host-side
+argument checks answer without touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_post_weight_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4pw.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    names = re.findall(r"\b([A-Za-z_][A-Za-z0-9_]*)\s*\([^;{}]*\)\s*;", src)
+    return sorted({n for n in names if n.startswith("nvfp4_")})
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("nvfp4_hessian_accumulate", "nvfp4_gptq_prepare",
+              "nvfp4_gptq_schur_replay_quantize", "nvfp4_dequant", "nvfp4_layer_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function():
+    lib = ctypes.CDLL(B._LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_function():
+    lib = B.lib()
+    for n in declared_functions():
+        assert getattr(lib, n).restype is not None or n in (
+            "nvfp4_default_params",), n
+
+
+def test_host_side_checks_need_no_device():
+    L = B.lib()
+    null = None
+    # d_in not a multiple of 16 -> NVFP4_ERR_SHAPE before any device work
+    assert L.nvfp4_gptq_schur_replay_quantize(
+        ctypes.c_void_p(256), 0, 4, 20, ctypes.c_void_p(256), null, null,
+        ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), null,
+        ctypes.c_void_p(256), 1 << 20, null) == 2
+    # negative sizes -> NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_dequant(null, null, null, -1, 16, null, 0, null) == 1
+    # a workspace that is too small -> NVFP4_ERR_WORKSPACE
+    assert L.nvfp4_gptq_prepare(ctypes.c_void_p(256), 32, 0.01, ctypes.c_void_p(256), null,
+                                null, ctypes.c_void_p(256), 16, null) == 3
+    # the allocation-free quantize refuses layers beyond its fixed scratch
+    assert L.nvfp4_gptq_schur_replay_quantize_noalloc(
+        ctypes.c_void_p(256), 0, 4096, 4096, ctypes.c_void_p(256), null, null,
+        ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), null, null,
+        null) == 3
+    assert L.nvfp4_status_string(5) == b"damped Hessian is not positive definite"
+    assert L.nvfp4_prepare_workspace_size(-1) == 0
+
+
+@pytest.mark.parametrize("d_out,d_in", [(0, 0), (1, 16), (4096, 4096)])
+def test_workspace_sizes_grow_with_the_layer(d_out, d_in):
+    q = B.nvfp4_quantize_workspace_size(d_out, d_in)
+    assert q >= 8 * d_out * d_in
+    assert B.nvfp4_prepare_workspace_size(d_in) >= 4 * d_in * d_in
