@@ -157,6 +157,36 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
     uint8_t* scales, float* global_scale, double* err_out, void* ws, size_t ws_bytes,
     nvfp4_stream_t stream);
 
+/* Allocation-free form of nvfp4_gptq_schur_replay_quantize (the paper has no
+ * counterpart; it serves callers that cannot allocate device memory when they
+ * quantize, e.g. an engine that owns all GPU memory through its own fixed pool
+ * and forbids allocations outside it, or a host loop that must not take the
+ * implicit device synchronisation of cudaMalloc/cudaFree).
+ *
+ * Same arguments and results as nvfp4_gptq_schur_replay_quantize, without the
+ * workspace: the scratch is one fixed 16 MiB device array inside the library,
+ * present on every GPU that loads it until the process exits.  The call does
+ * not allocate (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Size limit: the layer must satisfy
+ *     nvfp4_quantize_workspace_size(d_out, d_in, params) <= 16 MiB (about one
+ *     million weights, e.g. 1024 x 1024); larger layers return
+ *     NVFP4_ERR_WORKSPACE without launching anything.
+ *   - status_out: optional device int out; receives the device status word of
+ *     this call (what nvfp4_workspace_status reports for the workspace form).
+ *   - The device current on the calling thread must be the stream's device.
+ *     The first call on a device looks up the array's device address (once
+ *     per device, under a lock); make that first call before any stream
+ *     capture.
+ *   - All calls on one device share the array and it keeps the previous
+ *     call's contents (the call clears what must start at zero itself).  Calls
+ *     whose GPU work overlaps, e.g. on two streams without ordering, race and
+ *     give undefined results: order them on one stream. */
+nvfp4_status nvfp4_gptq_schur_replay_quantize_noalloc(
+    const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in, const float* U,
+    const nvfp4_solve_params* params, const uint8_t* dead, uint8_t* codes,
+    uint8_t* scales, float* global_scale, double* err_out, int* status_out,
+    nvfp4_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* a9  dequantization: Q = e2m1(code) * e4m3(scale) * s_g                    */
 /* "Replay the Curvature", Abstract (NVFP4 format).                          */

@@ -58,6 +58,9 @@ def lib():
             "nvfp4_gptq_schur_replay_quantize": (
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, sz,
                  vp], i32),
+            "nvfp4_gptq_schur_replay_quantize_noalloc": (
+                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
+                 vp], i32),
             "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
             "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
@@ -140,6 +143,20 @@ def nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, global_scale, err_out=
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
         _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def nvfp4_gptq_schur_replay_quantize_noalloc(W, U, codes, scales, global_scale, err_out=None,
+                                             status_out=None, dead=None, params=None,
+                                             stream=None):
+    """The quantize call without a workspace: the library's fixed device
+    scratch array is used instead, for callers that cannot allocate."""
+    d_out, d_in = W.shape
+    p = params if params is not None else default_params()
+    _check("nvfp4_gptq_schur_replay_quantize_noalloc",
+           lib().nvfp4_gptq_schur_replay_quantize_noalloc(
+               _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
+               _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(status_out),
+               _stream(stream)))
 
 
 def nvfp4_dequant(codes, scales, global_scale, out, stream=None):
