@@ -95,11 +95,21 @@ nvfp4_status nvfp4_workspace_status(const void* ws, nvfp4_stream_t stream);
  * X     : n_tok x d, bf16 or fp32 (x_dtype), one token per row.
  * beta  : 0 -> H = X^T X, 1 -> H += X^T X (accumulate over token chunks).
  * d must be a multiple of 16; n_tok >= 0 (0 with beta = 0 zeroes H).
- * bf16 products are exact in fp32 and are summed in fp32 on the tensor cores;
- * fp32 inputs are multiplied and summed in fp32.  No workspace. */
+ * bf16 products are exact in fp32 and are summed in fp32 on the tensor cores
+ * (tcgen05, when d >= 256, n_tok >= 64 and X is 16-byte aligned; otherwise on
+ * the CUDA cores); fp32 inputs are multiplied and summed in fp32 on the CUDA
+ * cores.  With beta = 1 the existing H must be symmetric (as this call writes
+ * it).  No workspace.  The tensor-core kernel's waits are bounded; if one runs
+ * out it sets a library status word that nvfp4_hessian_status() reports. */
 nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dtype,
                                       int64_t n_tok, int64_t d, int beta,
                                       nvfp4_stream_t stream);
+
+/* Synchronizes `stream` and returns, then clears, the status word of the
+ * Hessian calls on the current device: NVFP4_ERR_TIMEOUT if a tensor-core
+ * Hessian kernel gave up on a bounded wait since the last query, NVFP4_OK
+ * otherwise (NVFP4_ERR_CUDA if the word could not be read). */
+nvfp4_status nvfp4_hessian_status(nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* a2-a4  damping + upper Cholesky factor of the damped inverse              */

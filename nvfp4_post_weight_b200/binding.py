@@ -52,6 +52,7 @@ def lib():
             "nvfp4_workspace_status": ([vp, vp], i32),
             "nvfp4_default_params": ([ctypes.POINTER(SolveParams)], None),
             "nvfp4_hessian_accumulate": ([vp, vp, i32, i64, i64, i32, vp], i32),
+            "nvfp4_hessian_status": ([vp], i32),
             "nvfp4_prepare_workspace_size": ([i64], sz),
             "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
@@ -117,6 +118,10 @@ def nvfp4_hessian_accumulate(H, X, beta=0, stream=None):
     n_tok, d = X.shape
     _check("nvfp4_hessian_accumulate", lib().nvfp4_hessian_accumulate(
         _ptr(H), _ptr(X), _dtype_code(X), n_tok, d, int(beta), _stream(stream)))
+
+
+def nvfp4_hessian_status(stream=None) -> int:
+    return int(lib().nvfp4_hessian_status(_stream(stream)))
 
 
 def nvfp4_prepare_workspace_size(d) -> int:

@@ -70,7 +70,13 @@ nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dty
   if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
   if (d == 0) return NVFP4_OK;
   ProfileScope ps(kPhaseHessian, as_cuda(stream));
+  if (hessian_tc_supported(H, X, x_dtype, n_tok, d))
+    return launch_hessian_tc(H, X, n_tok, d, beta, as_cuda(stream));
   return launch_hessian_simt(H, X, x_dtype, n_tok, d, beta, as_cuda(stream));
+}
+
+nvfp4_status nvfp4_hessian_status(nvfp4_stream_t stream) {
+  return static_cast<nvfp4_status>(hessian_tc_take_status(as_cuda(stream)));
 }
 
 size_t nvfp4_prepare_workspace_size(int64_t d) {

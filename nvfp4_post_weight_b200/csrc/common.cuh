@@ -1,6 +1,7 @@
 // Shared host/device helpers of the NVFP4 GPTQ library (sm_100a).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -63,7 +64,20 @@ struct ProfileScope {
     }                                                          \
   } while (0)
 
+// SM count of the current device (cached per device).
+int num_sms();
+// 2-D tiled TMA descriptor: dims[0] innermost (elements), strides[0] = bytes
+// between rows, box in elements; out-of-range elements read as zero.
+bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                    const uint64_t dims[2], const uint64_t strides[1], const uint32_t box[2],
+                    CUtensorMapSwizzle swizzle);
+
 // ---- kernel launchers implemented in the .cu files -------------------------
+bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
+                          int64_t d);
+nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
+                               cudaStream_t st);
+int hessian_tc_take_status(cudaStream_t st);
 nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                             int64_t d, int beta, cudaStream_t st);
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,

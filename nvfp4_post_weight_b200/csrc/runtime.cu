@@ -5,6 +5,8 @@
 // While profiling is on, each launcher's ProfileScope records a CUDA event
 // pair on the launching stream; nvfp4_profile_end() waits for the events and
 // returns, per phase, the summed device time and the number of launches.
+#include <cudaTypedefs.h>
+
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -71,6 +73,50 @@ ProfileScope::~ProfileScope() {
     cudaGetLastError();
     g_records[slot].phase = -1;
   }
+}
+
+// ---- device properties and TMA descriptors ---------------------------------
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return kNumSMs;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = kNumSMs;
+  }
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                    const uint64_t dims[2], const uint64_t strides[1], const uint32_t box[2],
+                    CUtensorMapSwizzle swizzle) {
+  // The driver entry point is looked up at run time, so the library itself does
+  // not link against libcuda.
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      fn = nullptr;
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }();
+  if (!encode) return false;
+  cuuint64_t gd[2] = {dims[0], dims[1]};
+  cuuint64_t gs[1] = {strides[0]};
+  cuuint32_t bd[2] = {box[0], box[1]};
+  cuuint32_t es[2] = {1, 1};
+  return encode(map, dtype, 2, const_cast<void*>(base), gd, gs, bd, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace nvfp4
