@@ -78,6 +78,19 @@ bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t
 nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
                                cudaStream_t st);
 int hessian_tc_take_status(cudaStream_t st);
+
+// TMA descriptors of the tensor-core trailing update: Delta = Dh + Dl
+// (d_out x 128, fp32 each) and the split rows U = Uh + Ul of one batch,
+// transposed (d_in x 128, fp32 each, rows >= e used).
+struct UpdateMaps {
+  CUtensorMap Dh, Dl, Uh, Ul;
+};
+bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
+                      const float* Ul, int64_t d_out, int64_t d_in);
+// W~[:, e:] -= (Dh + Dl)(Uh + Ul)[:, e:] (3xTF32, fp64 W~); a timed-out wait
+// sets NVFP4_ERR_TIMEOUT in *status.
+nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int64_t d_out,
+                              int64_t d_in, int64_t e, int* status, cudaStream_t st);
 nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                             int64_t d, int beta, cudaStream_t st);
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,

@@ -42,7 +42,10 @@ struct QuantHeader {   // workspace header (first 256 bytes)
 struct QuantLayout {
   QuantHeader* hdr;
   double* Wt;      // d_out x d_in working copy
-  double* Delta;   // d_out x 128
+  float* Dh;       // d_out x 128: the batch's deltas, tf32-rounded part
+  float* Dl;       // d_out x 128: remainder (delta - Dh)
+  float* Uh;       // d_in x 128: the batch's rows of U transposed, tf32 part
+  float* Ul;       // d_in x 128: remainder
   double* rowerr;  // d_out
 };
 
@@ -53,8 +56,14 @@ QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in) {
   size_t off = kWsHeader;
   L.Wt = reinterpret_cast<double*>(p + off);
   off += align256(sizeof(double) * d_out * d_in);
-  L.Delta = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * d_out * kLazyBatch);
+  L.Dh = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * d_out * kLazyBatch);
+  L.Dl = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * d_out * kLazyBatch);
+  L.Uh = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * kLazyBatch * d_in);
+  L.Ul = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * kLazyBatch * d_in);
   L.rowerr = reinterpret_cast<double*>(p + off);
   return L;
 }
@@ -124,6 +133,41 @@ constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a ba
 // Index of the upper tile (p, q), q >= p, in the packed tile array.
 __device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p) / 2 + q; }
 
+// x = hi + lo with hi rounded to tf32 (10 explicit mantissa bits, nearest,
+// ties to even) and lo = x - hi; the 3xTF32 update multiplies the pairs.
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
+}
+
+// Uh[j][k] + Ul[j][k] = U[c0 + k][j] for the batch rows k < 128 and the
+// columns j >= e right of the batch: the trailing update's B operand, stored
+// K-contiguous.  32x32 tiles transposed through shared memory.
+__global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restrict__ U,
+                                                           int64_t d_in, int64_t c0, int64_t e,
+                                                           float* __restrict__ Uh,
+                                                           float* __restrict__ Ul) {
+  __shared__ float t[32][33];
+  const int64_t j0 = e + (int64_t)blockIdx.x * 32;
+  const int k0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int64_t j = j0 + tx;
+    t[r][tx] = j < d_in ? U[(c0 + k0 + r) * d_in + j] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int64_t j = j0 + r;
+    if (j < d_in) {
+      const float u = t[tx][r];
+      const float h = tf32_rn(u);
+      Uh[j * kLazyBatch + k0 + tx] = h;
+      Ul[j * kLazyBatch + k0 + tx] = u - h;
+    }
+  }
+}
+
 // One candidate's replay of the in-block GPTQ updates (fp64).  v holds the
 // block's 16 current values and is consumed.  Ud points at the block's
 // diagonal 16x16 tile (row-major), invd at its 1/U_jj.  Returns the score
@@ -160,8 +204,8 @@ __global__ void __launch_bounds__(kReplayThreads)
     schur_replay_batch_kernel(double* __restrict__ Wt, const float* __restrict__ U,
                               int64_t d_out, int64_t d_in, int c0, int bw,
                               const float* __restrict__ sg_ptr, uint8_t* __restrict__ codes,
-                              uint8_t* __restrict__ scales, double* __restrict__ Delta,
-                              double* __restrict__ rowerr) {
+                              uint8_t* __restrict__ scales, float* __restrict__ Dh,
+                              float* __restrict__ Dl, double* __restrict__ rowerr) {
   extern __shared__ double4 smem_d4[];
   double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
   double* invd = Ut + kUTiles * 256;                         // 128
@@ -261,7 +305,12 @@ __global__ void __launch_bounds__(kReplayThreads)
       __syncwarp();
     }
     if (valid) {
-      for (int c = hl; c < bw; c += 16) Delta[r * kLazyBatch + c] = row[c];
+      for (int c = hl; c < bw; c += 16) {
+        const double x = row[c];
+        const float h = tf32_rn((float)x);
+        Dh[r * kLazyBatch + c] = h;
+        Dl[r * kLazyBatch + c] = (float)(x - (double)h);
+      }
       if (hl == 0) rowerr[r] += rowsum;
     }
     __syncwarp();
@@ -295,7 +344,8 @@ constexpr size_t kReplaySmem =
 
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
   return kWsHeader + align256(sizeof(double) * d_out * d_in) +
-         align256(sizeof(double) * d_out * kLazyBatch) + align256(sizeof(double) * d_out);
+         2 * align256(sizeof(float) * d_out * kLazyBatch) +
+         2 * align256(sizeof(float) * kLazyBatch * d_in) + align256(sizeof(double) * d_out);
 }
 
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
@@ -326,6 +376,8 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(schur_replay_batch_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kReplaySmem));
+  UpdateMaps maps;
+  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, d_out, d_in)) return NVFP4_ERR_CUDA;
   const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
   const int rgrid = (int)(row_groups < 2 * kNumSMs ? row_groups : 2 * kNumSMs);
   for (int64_t c0 = 0; c0 < d_in; c0 += kLazyBatch) {
@@ -333,16 +385,19 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
     {
       ProfileScope ps(kPhaseReplay, st);
       schur_replay_batch_kernel<<<rgrid, kReplayThreads, kReplaySmem, st>>>(
-          L.Wt, U, d_out, d_in, (int)c0, bw, sg, codes, scales, L.Delta, L.rowerr);
+          L.Wt, U, d_out, d_in, (int)c0, bw, sg, codes, scales, L.Dh, L.Dl, L.rowerr);
       NVFP4_LAUNCH_CHECK();
       count_launches(1);
     }
     const int64_t e = c0 + bw;
     if (e < d_in) {
       ProfileScope ps(kPhaseUpdate, st);
-      // W~[:, e:] -= Delta[:, :bw] U[c0:c0+bw, e:]
-      nvfp4_status s = dgemm_update((int)d_out, (int)(d_in - e), bw, L.Delta, kLazyBatch,
-                                    U + c0 * d_in + e, d_in, L.Wt + e, d_in, st);
+      // W~[:, e:] -= Delta[:, :bw] U[c0:c0+bw, e:]   (bw = 128 here)
+      split_u_rows_kernel<<<dim3((unsigned)((d_in - e + 31) / 32), kLazyBatch / 32), 256, 0,
+                            st>>>(U, d_in, c0, e, L.Uh, L.Ul);
+      NVFP4_LAUNCH_CHECK();
+      count_launches(1);
+      nvfp4_status s = launch_update_tc(maps, L.Wt, d_in, d_out, d_in, e, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
     }
   }
