@@ -229,6 +229,18 @@ nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t
 /* Diagnostics: launch accounting and per-phase device timing                */
 /* (measurement support; the paper has no counterpart)                       */
 /* ------------------------------------------------------------------------ */
+/* The factorisation's fp32 GEMM building block, exposed so that it can be
+ * tested on its own (the paper has no counterpart):
+ *   C = beta C + alpha P Q^T   on the tensor cores, 3xTF32 (fp32 accuracy),
+ * P: M x K (ldp), Q: N x K (ldq), C: M x N (ldc), fp32 row-major device
+ * arrays; P and Q 16-byte aligned with ldp, ldq multiples of 4.  lower != 0
+ * (M == N): only the 128 x 128 tiles on or below the diagonal are written.
+ * status: device int, 0 on entry; a timed-out wait inside the kernel sets it
+ * to NVFP4_ERR_TIMEOUT. */
+nvfp4_status nvfp4_gemm_nt_f32(int64_t M, int64_t N, int64_t K, float alpha, const float* P,
+                               int64_t ldp, const float* Q, int64_t ldq, float beta, float* C,
+                               int64_t ldc, int lower, int* status, nvfp4_stream_t stream);
+
 /* Number of kernels this library has launched since it was loaded (all
  * threads, all devices).  Host-only; never fails. */
 long long nvfp4_launch_count(void);

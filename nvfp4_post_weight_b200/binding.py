@@ -63,6 +63,8 @@ def lib():
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
                  vp], i32),
             "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
+            "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
+                                   vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
             "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
         }
@@ -180,3 +182,15 @@ def nvfp4_layer_error(W, codes, scales, global_scale, H, err_out, ws, stream=Non
     _check("nvfp4_layer_error", lib().nvfp4_layer_error(
         _ptr(W), _dtype_code(W), _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(H),
         d_out, d_in, _ptr(err_out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def nvfp4_gemm_nt_f32(P, Q, C, alpha=1.0, beta=0.0, lower=False, status=None, stream=None):
+    """C = beta C + alpha P Q^T (3xTF32 on the tensor cores); P, Q, C fp32."""
+    M, K = P.shape
+    N = Q.shape[0]
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=P.device)
+    _check("nvfp4_gemm_nt_f32", lib().nvfp4_gemm_nt_f32(
+        M, N, K, float(alpha), _ptr(P), P.stride(0), _ptr(Q), Q.stride(0), float(beta), _ptr(C),
+        C.stride(0), int(bool(lower)), _ptr(status), _stream(stream)))
+    return status

@@ -153,4 +153,15 @@ nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t
                             ws, as_cuda(stream));
 }
 
+nvfp4_status nvfp4_gemm_nt_f32(int64_t M, int64_t N, int64_t K, float alpha, const float* P,
+                               int64_t ldp, const float* Q, int64_t ldq, float beta, float* C,
+                               int64_t ldc, int lower, int* status, nvfp4_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0 || !status || (lower && M != N)) return NVFP4_ERR_INVALID_ARG;
+  if (M > kMaxRows || N > kMaxRows || K > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!P || !Q || !C || ldp < K || ldq < K || ldc < N) return NVFP4_ERR_INVALID_ARG;
+  return gemm_nt_tc((int)M, (int)N, (int)K, alpha, P, ldp, 0, Q, ldq, 0, beta, C, ldc, 0,
+                    nullptr, 0, 0, 1, lower ? 1 : 0, status, as_cuda(stream));
+}
+
 }  // extern "C"

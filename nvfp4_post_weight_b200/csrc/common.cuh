@@ -71,6 +71,21 @@ int num_sms();
 bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                     const uint64_t dims[2], const uint64_t strides[1], const uint32_t box[2],
                     CUtensorMapSwizzle swizzle);
+// rank-D version: dims[rank], strides[rank-1] (bytes), box[rank].
+bool encode_tmap_nd(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int rank,
+                    const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                    CUtensorMapSwizzle swizzle);
+
+// C = beta C + alpha P Q^T on the tensor cores (3xTF32).  P: M x K, Q: N x K,
+// C: M x N, all fp32 row-major with leading dimensions ld* (multiples of 4)
+// and, for batch > 1, element strides stride* between the batch's matrices.
+// C2 (optional): C^T is also written there.  lower: only the 128 x 128 tiles
+// on or below the diagonal (M == N).  A timed-out wait sets *status.
+nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_t ldp,
+                        int64_t strideP, const float* Q, int64_t ldq, int64_t strideQ,
+                        float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
+                        int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
+                        cudaStream_t st);
 
 // ---- kernel launchers implemented in the .cu files -------------------------
 bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
@@ -109,23 +124,5 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
                                 int64_t d_out, int64_t d_in, double* err, void* ws,
                                 cudaStream_t st);
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in);
-
-// C = alpha * op(A) * op(B) + beta * C in fp32 on the CUDA cores.  Row-major;
-// op(A) is M x K, op(B) is K x N.  ta/tb: 1 -> the stored matrix is transposed.
-// tri: 0 full; 1 only output tiles on or below the diagonal (row >= col block);
-//      2 only tiles on or above it.
-nvfp4_status sgemm_simt_batched(int M, int N, int K, float alpha, const float* A,
-                                int64_t lda, int64_t sA, int ta, const float* B,
-                                int64_t ldb, int64_t sB, int tb, float beta, float* C,
-                                int64_t ldc, int64_t sC, int tri, int batch,
-                                cudaStream_t st);
-// C -= A B with C, A fp64 and B fp32 (widened exactly), on the CUDA cores.
-// Row-major: A is M x K (lda), B is K x N (ldb), C is M x N (ldc).
-nvfp4_status dgemm_update(int M, int N, int K, const double* A, int64_t lda, const float* B,
-                          int64_t ldb, double* C, int64_t ldc, cudaStream_t st);
-
-nvfp4_status sgemm_simt(int M, int N, int K, float alpha, const float* A, int64_t lda,
-                        int ta, const float* B, int64_t ldb, int tb, float beta, float* C,
-                        int64_t ldc, int tri, cudaStream_t st);
 
 }  // namespace nvfp4

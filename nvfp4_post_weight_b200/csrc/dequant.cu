@@ -158,8 +158,11 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
         static_cast<const float*>(W), codes, scales, sg, nb, E);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-  nvfp4_status s = sgemm_simt((int)d_out, (int)d_in, (int)d_in, 1.f, E, d_in, 0, H, d_in, 0,
-                              0.f, EH, d_in, 0, st);
+  // EH = E H^T = E H (H symmetric) on the tensor cores
+  int* status = static_cast<int*>(ws);
+  NVFP4_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  nvfp4_status s = gemm_nt_tc((int)d_out, (int)d_in, (int)d_in, 1.f, E, d_in, 0, H, d_in, 0,
+                              0.f, EH, d_in, 0, nullptr, 0, 0, 1, 0, status, st);
   if (s != NVFP4_OK) return s;
   dot_kernel<<<kDotBlocks, 256, 0, st>>>(E, EH, d_out * d_in, part);
   NVFP4_LAUNCH_CHECK();

@@ -73,58 +73,219 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
   }
 }
 
-// Factors the kb x kb diagonal block at (k, k) of A in fp64: A_kk = L11 L11^T,
-// writes L11 back into A and L11^-1 into the same block of X.
-__global__ void __launch_bounds__(256) chol_diag_block_kernel(float* __restrict__ A, int64_t d,
-                                                              int64_t k, int kb,
-                                                              float* __restrict__ X,
-                                                              PrepHeader* hdr) {
+// One panel of the right-looking Cholesky: columns k .. k+kb-1 of A (lower,
+// already updated by the earlier panels).  Every CTA factors the 64 x 64
+// diagonal block A11 = L11 L11^T and inverts L11 in fp64 (redundantly: no CTA
+// waits for another); CTA 0 then writes L11 into A and X11 = L11^-1,
+// Y11 = X11^T into the diagonal blocks of X and Y, every other CTA solves its
+// own 64-row slice of the panel below, L21 = A21 X11^T, in place.
+//
+// The 64 x 64 block is itself blocked by 16 (a per-column CTA barrier costs
+// far more than the arithmetic of a column):
+//   for each 16-column sub-panel K:
+//     one warp factors and inverts the 16 x 16 diagonal block in registers,
+//       exchanging values by shuffles (lane i holds row i);
+//     all threads solve the rows below it, L[r][K] = S[r][K] inv(L_KK)^T,
+//     and update the trailing lower part, S -= L[:,K] L[:,K]^T;
+//   the inverse of L is assembled from the four 16 x 16 inverses by two
+//   doubling steps, X21 = -X22 (L21 X11), as small products.
+constexpr int kPanelThreads = 256;
+constexpr int kPitch = NB + 1;
+constexpr int kSub = 16;
+
+// 1/p for p > 0: the hardware's approximate fp64 reciprocal refined by two
+// Newton-Raphson steps (x <- x + x (1 - p x)), which square the relative
+// error each time.
+__device__ __forceinline__ double recip_nr(double p) {
+  double x;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(x) : "d"(p));
+  x = fma(x, fma(-p, x, 1.0), x);
+  x = fma(x, fma(-p, x, 1.0), x);
+  return x;
+}
+
+constexpr size_t kPanelSmem = sizeof(double) * (4 * NB * kPitch);
+
+// One warp, lanes 0..15 meaningful: factor the 16 x 16 block at (o, o) of S
+// (lower part), write L_KK back into S and inv(L_KK) into the same block of
+// Xd (lower, zeros above).  A non-positive pivot is flagged and taken as 1.
+__device__ __forceinline__ void factor_invert_16(double (*S)[kPitch], double (*Xd)[kPitch],
+                                                 int o, PrepHeader* hdr) {
+  const int lane = threadIdx.x & 31;
+  const int i = lane & 15;
+  const unsigned full = 0xffffffffu;
+  double r[kSub];   // row i of the block
+#pragma unroll
+  for (int l = 0; l < kSub; ++l) r[l] = (l <= i) ? S[o + i][o + l] : 0.0;
+  double sq[kSub];  // sqrt(pivot_j), the same in every lane
+#pragma unroll
+  for (int j = 0; j < kSub; ++j) {
+    double p = __shfl_sync(full, r[j], j, 16);
+    const bool ok = p > 0.0;
+    if (!ok) {
+      if (lane == 0) flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
+      p = 1.0;
+    }
+    sq[j] = p;   // square root taken below, off the per-column chain
+    const double a = (i > j) ? r[j] * recip_nr(p) : 0.0;
+#pragma unroll
+    for (int l = j + 1; l < kSub; ++l) {
+      const double cl = __shfl_sync(full, r[j], l, 16);   // S[l][j]
+      r[l] = fma(-a, cl, r[l]);
+    }
+  }
+  // L[i][l] = r[l] / sqrt(p_l) (l < i), L[i][i] = sqrt(p_i)
+  double isq[kSub];
+#pragma unroll
+  for (int l = 0; l < kSub; ++l) {
+    sq[l] = sqrt(sq[l]);
+    isq[l] = recip_nr(sq[l]);
+  }
+#pragma unroll
+  for (int l = 0; l < kSub; ++l) r[l] = l < i ? r[l] * isq[l] : (l == i ? sq[i] : 0.0);
+  // column c = i of inv(L): x[m] = -(sum_{l<m} L[m][l] x[l]) / L[m][m] for m > c
+  double x[kSub];
+#pragma unroll
+  for (int m = 0; m < kSub; ++m) {
+    double acc = 0.0;
+#pragma unroll
+    for (int l = 0; l < m; ++l) acc = fma(__shfl_sync(full, r[l], m, 16), x[l], acc);
+    x[m] = m < i ? 0.0 : (m == i ? isq[m] : -acc * isq[m]);
+  }
+  if (lane < kSub) {
+#pragma unroll
+    for (int l = 0; l < kSub; ++l) {
+      S[o + i][o + l] = l <= i ? r[l] : 0.0;
+      Xd[o + l][o + i] = x[l];   // column i of the inverse
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPanelThreads)
+    chol_panel_kernel(float* __restrict__ A, int64_t d, int64_t k, int kb,
+                      float* __restrict__ X, float* __restrict__ Y, PrepHeader* hdr) {
   extern __shared__ double dsm[];
-  double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(dsm);
-  double(*V)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(dsm + NB * (NB + 1));
-  const int tid = threadIdx.x;
-  for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
-    const int i = idx / kb, j = idx % kb;
-    S[i][j] = (j <= i) ? (double)A[(k + i) * d + k + j] : 0.0;
+  double(*S)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm);             // A11 -> L11
+  double(*Xd)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + NB * kPitch);   // X11
+  double(*R)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 2 * NB * kPitch);
+  double(*T)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 3 * NB * kPitch);  // scratch
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t r0 = k + kb + (int64_t)(blockIdx.x - 1) * NB;   // slice rows (CTA >= 1)
+  const int64_t rem = d - r0;
+  const int rows = blockIdx.x == 0 ? 0 : (int)(rem < NB ? rem : NB);
+
+  {   // all global loads of a thread are issued before any is used
+    constexpr int kPer = NB * NB / kPanelThreads;   // 16
+    float a11[kPer], a21[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
+      a11[q] = (i < kb && l <= i) ? A[(k + i) * d + k + l] : 0.f;
+      a21[q] = (i < rows && l < kb) ? A[(r0 + i) * d + k + l] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
+      S[i][l] = (i < kb && l < kb) ? (double)a11[q] : (i == l ? 1.0 : 0.0);
+      Xd[i][l] = 0.0;
+      R[i][l] = (double)a21[q];
+    }
   }
   __syncthreads();
-  for (int j = 0; j < kb; ++j) {
-    if (tid == 0) {
-      double p = S[j][j];
-      if (!(p > 0.0)) {           // also catches NaN
-        flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
-        p = 1.0;
-      }
-      S[j][j] = sqrt(p);
-    }
+
+  // ---- factor, 16 columns at a time
+  for (int K = 0; K < NB / kSub; ++K) {
+    const int o = K * kSub;
+    if (warp == 0) factor_invert_16(S, Xd, o, hdr);
     __syncthreads();
-    const double piv = S[j][j];
-    for (int i = j + 1 + tid; i < kb; i += blockDim.x) S[i][j] /= piv;
-    __syncthreads();
-    const int w = kb - j - 1;
-    for (int idx = tid; idx < w * w; idx += blockDim.x) {
-      const int i = j + 1 + idx / w, l = j + 1 + idx % w;
-      if (l <= i) S[i][l] -= S[i][j] * S[l][j];
-    }
-    __syncthreads();
-  }
-  // inverse of the lower triangle, one column per thread (forward substitution)
-  if (tid < kb) {
-    const int c = tid;
-    for (int i = 0; i < c; ++i) V[i][c] = 0.0;
-    V[c][c] = 1.0 / S[c][c];
-    for (int i = c + 1; i < kb; ++i) {
+    // rows below the sub-block: T[r][c] = sum_{l <= c} S[r][o+l] inv(L_KK)[c][l]
+    const int nb = NB - o - kSub;   // rows below (0, 16, 32 or 48)
+    for (int idx = tid; idx < nb * kSub; idx += blockDim.x) {
+      const int rr = o + kSub + idx / kSub, c = idx % kSub;
       double acc = 0.0;
-      for (int l = c; l < i; ++l) acc += S[i][l] * V[l][c];
-      V[i][c] = -acc / S[i][i];
+#pragma unroll
+      for (int l = 0; l < kSub; ++l) acc = fma(S[rr][o + l], Xd[o + c][o + l], acc);
+      T[rr][c] = acc;
     }
+    __syncthreads();
+    for (int idx = tid; idx < nb * kSub; idx += blockDim.x) {
+      const int rr = o + kSub + idx / kSub, c = idx % kSub;
+      S[rr][o + c] = T[rr][c];
+    }
+    __syncthreads();
+    // trailing lower part: S[r][l] -= sum_m L[r][o+m] L[l][o+m], o+16 <= l <= r
+    for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
+      const int rr = o + kSub + idx / nb, l = o + kSub + idx % nb;
+      if (l <= rr) {
+        double acc = S[rr][l];
+#pragma unroll
+        for (int m = 0; m < kSub; ++m) acc = fma(-S[rr][o + m], S[l][o + m], acc);
+        S[rr][l] = acc;
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- inverse by doubling: blocks of 16 -> 32 -> 64.  For a pair of
+  // diagonal blocks of size b at offset q: X21 = -X22 (L21 X11).
+  for (int b = kSub; b < NB; b *= 2) {
+    const int npairs = NB / (2 * b);
+    // T = L21 X11 for every pair (b x b each)
+    for (int idx = tid; idx < npairs * b * b; idx += blockDim.x) {
+      const int pq = idx / (b * b), e = idx % (b * b), i = e / b, j = e % b;
+      const int q = pq * 2 * b;
+      double acc = 0.0;
+      for (int l = j; l < b; ++l) acc = fma(S[q + b + i][q + l], Xd[q + l][q + j], acc);
+      T[q + b + i][q + j] = acc;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < npairs * b * b; idx += blockDim.x) {
+      const int pq = idx / (b * b), e = idx % (b * b), i = e / b, j = e % b;
+      const int q = pq * 2 * b;
+      double acc = 0.0;
+      for (int l = 0; l <= i; ++l) acc = fma(Xd[q + b + i][q + b + l], T[q + b + l][q + j], acc);
+      Xd[q + b + i][q + j] = -acc;
+    }
+    __syncthreads();
+  }
+
+  if (blockIdx.x == 0) {
+    for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
+      const int i = idx / kb, j = idx % kb;
+      if (j <= i) A[(k + i) * d + k + j] = (float)S[i][j];
+      const float x = (float)Xd[i][j];
+      X[(k + i) * d + k + j] = x;            // lower (zeros above)
+      Y[(k + j) * d + k + i] = x;            // its transpose, upper
+    }
+    return;
+  }
+  // ---- L21 slice = A21 slice X11^T: thread (ty, tx) computes a 4 x 4 tile,
+  // L21[i][c] = sum_l R[i][l] X11[c][l]; X11 is staged transposed in T first
+  // so that the loop reads it along rows (free of bank conflicts).
+  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
+    const int c = idx / NB, l = idx % NB;
+    T[l][c] = Xd[c][l];
   }
   __syncthreads();
-  for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
-    const int i = idx / kb, j = idx % kb;
-    if (j <= i) A[(k + i) * d + k + j] = (float)S[i][j];
-    X[(k + i) * d + k + j] = (float)V[i][j];
+  const int ty = tid >> 4, tx = tid & 15, i0 = 4 * ty, l0 = 4 * tx;
+  double acc[4][4] = {};
+  for (int l = 0; l < NB; ++l) {
+    double rv[4], xv[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) rv[a] = R[i0 + a][l];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) xv[b] = T[l][l0 + b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fma(rv[a], xv[b], acc[a][b]);
   }
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if (i0 + a < rows && l0 + b < kb)
+        A[(r0 + i0 + a) * d + k + l0 + b] = (float)acc[a][b];
 }
 
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
@@ -140,9 +301,10 @@ __global__ void reverse_to_upper_kernel(const float* __restrict__ X, int64_t d,
 
 struct PrepLayout {
   PrepHeader* hdr;
-  float* A;
-  float* X;
-  float* T;
+  float* A;   // J H_d J, then its Cholesky factor L (lower)
+  float* X;   // L^-1 (lower)
+  float* Y;   // L^-T (upper)
+  float* T;   // scratch of the inverse doubling
 };
 
 PrepLayout prep_layout(void* ws, int64_t d) {
@@ -153,6 +315,8 @@ PrepLayout prep_layout(void* ws, int64_t d) {
   L.A = reinterpret_cast<float*>(p + off);
   off += align256(sizeof(float) * d * d);
   L.X = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * d * d);
+  L.Y = reinterpret_cast<float*>(p + off);
   off += align256(sizeof(float) * d * d);
   L.T = reinterpret_cast<float*>(p + off);
   return L;
@@ -166,7 +330,7 @@ int grid_for(int64_t n, int threads) {
 }  // namespace
 
 size_t prepare_ws_bytes(int64_t d) {
-  return kWsHeader + 2 * align256(sizeof(float) * d * d) +
+  return kWsHeader + 3 * align256(sizeof(float) * d * d) +
          align256(sizeof(float) * (size_t)((d * d + 3) / 4 + d * NB));
 }
 
@@ -181,55 +345,58 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
 
-  // Blocked right-looking Cholesky of A (lower).
-  const size_t diag_smem = 2 * sizeof(double) * NB * (NB + 1);
-  NVFP4_CUDA_TRY(cudaFuncSetAttribute(chol_diag_block_kernel,
+  NVFP4_CUDA_TRY(cudaMemsetAsync(L.Y, 0, sizeof(float) * d * d, st));
+  int* status = &L.hdr->status;
+
+  // Blocked right-looking Cholesky of A (lower): per 64-column panel, one
+  // fused panel kernel (diagonal factor + inverse + panel solve), then the
+  // trailing update A22 -= L21 L21^T on the tensor cores.
+  NVFP4_CUDA_TRY(cudaFuncSetAttribute(chol_panel_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)diag_smem));
+                                      (int)kPanelSmem));
   for (int64_t k = 0; k < d; k += NB) {
     const int kb = (int)((d - k) < NB ? (d - k) : NB);
-    chol_diag_block_kernel<<<1, 256, diag_smem, st>>>(L.A, d, k, kb, L.X, L.hdr);
-    NVFP4_LAUNCH_CHECK();
-  count_launches(1);
     const int64_t m = d - k - kb;
+    const int grid = 1 + (int)((m + NB - 1) / NB);
+    chol_panel_kernel<<<grid, kPanelThreads, kPanelSmem, st>>>(L.A, d, k, kb, L.X, L.Y, L.hdr);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(1);
     if (m <= 0) break;
-    float* A21 = L.A + (k + kb) * d + k;
-    // L21 = A21 L11^-T, in place: each CTA owns whole rows of the panel.
-    nvfp4_status s = sgemm_simt((int)m, kb, kb, 1.f, A21, d, 0, L.X + k * d + k, d, 1, 0.f,
-                                A21, d, 0, st);
-    if (s != NVFP4_OK) return s;
-    // A22 -= L21 L21^T (lower tiles)
-    s = sgemm_simt((int)m, (int)m, kb, -1.f, A21, d, 0, A21, d, 1, 1.f,
-                   L.A + (k + kb) * d + (k + kb), d, 1, st);
+    const float* L21 = L.A + (k + kb) * d + k;
+    nvfp4_status s = gemm_nt_tc((int)m, (int)m, kb, -1.f, L21, d, 0, L21, d, 0, 1.f,
+                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 1, status,
+                                st);
     if (s != NVFP4_OK) return s;
   }
 
-  // X = L^-1 by recursive doubling: for adjacent diagonal blocks of size b,
-  // X21 = -X22 (L21 X11).  All pairs of one level are independent.
+  // X = L^-1 by recursive doubling over pairs of adjacent diagonal blocks of
+  // size b (all pairs of one level at once):  with L = [L11 0; L21 L22],
+  //   T^T = Y11 L21^T,  X21 = -X22 T,  Y12 = X21^T   (Y = X^T throughout),
+  // so every product is of the form P Q^T with K-contiguous operands.
   for (int64_t b = NB; b < d; b *= 2) {
-    const int64_t npairs_full = d / (2 * b);
+    const int64_t npairs = d / (2 * b);
     const int64_t stride = 2 * b * (d + 1);
-    if (npairs_full > 0) {
-      // T_p = L21 X11   (b x b each)
-      nvfp4_status s = sgemm_simt_batched((int)b, (int)b, (int)b, 1.f, L.A + b * d, d, stride,
-                                          0, L.X, d, stride, 0, 0.f, L.T, b, b * b, 0,
-                                          (int)npairs_full, st);
+    if (npairs > 0) {
+      nvfp4_status s = gemm_nt_tc((int)b, (int)b, (int)b, 1.f, L.Y, d, stride, L.A + b * d, d,
+                                  stride, 0.f, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0,
+                                  status, st);
       if (s != NVFP4_OK) return s;
-      // X21 = -X22 T_p
-      s = sgemm_simt_batched((int)b, (int)b, (int)b, -1.f, L.X + b * d + b, d, stride, 0,
-                             L.T, b, b * b, 0, 0.f, L.X + b * d, d, stride, 0,
-                             (int)npairs_full, st);
+      s = gemm_nt_tc((int)b, (int)b, (int)b, -1.f, L.X + b * (d + 1), d, stride, L.T, b, b * b,
+                     0.f, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, status,
+                     st);
       if (s != NVFP4_OK) return s;
     }
-    const int64_t r0 = npairs_full * 2 * b;         // start of a ragged pair
-    const int64_t rr = d - r0 - b;                  // rows in its right block
+    const int64_t r0 = npairs * 2 * b;   // a ragged pair: full left block, rr rows right
+    const int64_t rr = d - r0 - b;
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
-      nvfp4_status s = sgemm_simt((int)rr, (int)b, (int)b, 1.f, L.A + o + b * d, d, 0, L.X + o,
-                                  d, 0, 0.f, L.T, b, 0, st);
+      nvfp4_status s = gemm_nt_tc((int)b, (int)rr, (int)b, 1.f, L.Y + o, d, 0,
+                                  L.A + o + b * d, d, 0, 0.f, L.T, rr, 0, nullptr, 0, 0, 1, 0,
+                                  status, st);
       if (s != NVFP4_OK) return s;
-      s = sgemm_simt((int)rr, (int)b, (int)rr, -1.f, L.X + o + b * d + b, d, 0, L.T, b, 0, 0.f,
-                     L.X + o + b * d, d, 0, st);
+      // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
+      s = gemm_nt_tc((int)rr, (int)b, (int)rr, -1.f, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
+                     0.f, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, status, st);
       if (s != NVFP4_OK) return s;
     }
   }

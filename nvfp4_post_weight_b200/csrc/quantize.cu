@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "nvfp4_format.cuh"
+#include "sm100.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -133,14 +134,6 @@ constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a ba
 // Index of the upper tile (p, q), q >= p, in the packed tile array.
 __device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p) / 2 + q; }
 
-// x = hi + lo with hi rounded to tf32 (10 explicit mantissa bits, nearest,
-// ties to even) and lo = x - hi; the 3xTF32 update multiplies the pairs.
-__device__ __forceinline__ float tf32_rn(float x) {
-  uint32_t u = __float_as_uint(x);
-  u += 0xFFFu + ((u >> 13) & 1u);
-  return __uint_as_float(u & 0xFFFFE000u);
-}
-
 // Uh[j][k] + Ul[j][k] = U[c0 + k][j] for the batch rows k < 128 and the
 // columns j >= e right of the batch: the trailing update's B operand, stored
 // K-contiguous.  32x32 tiles transposed through shared memory.
@@ -161,7 +154,7 @@ __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restri
     const int64_t j = j0 + r;
     if (j < d_in) {
       const float u = t[tx][r];
-      const float h = tf32_rn(u);
+      const float h = sm100::tf32_rn(u);
       Uh[j * kLazyBatch + k0 + tx] = h;
       Ul[j * kLazyBatch + k0 + tx] = u - h;
     }
@@ -307,7 +300,7 @@ __global__ void __launch_bounds__(kReplayThreads)
     if (valid) {
       for (int c = hl; c < bw; c += 16) {
         const double x = row[c];
-        const float h = tf32_rn((float)x);
+        const float h = sm100::tf32_rn((float)x);
         Dh[r * kLazyBatch + c] = h;
         Dl[r * kLazyBatch + c] = (float)(x - (double)h);
       }

@@ -96,6 +96,12 @@ int num_sms() {
 bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                     const uint64_t dims[2], const uint64_t strides[1], const uint32_t box[2],
                     CUtensorMapSwizzle swizzle) {
+  return encode_tmap_nd(map, base, dtype, 2, dims, strides, box, swizzle);
+}
+
+bool encode_tmap_nd(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int rank,
+                    const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                    CUtensorMapSwizzle swizzle) {
   // The driver entry point is looked up at run time, so the library itself does
   // not link against libcuda.
   static PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
@@ -109,12 +115,16 @@ bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtyp
     }
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }();
-  if (!encode) return false;
-  cuuint64_t gd[2] = {dims[0], dims[1]};
-  cuuint64_t gs[1] = {strides[0]};
-  cuuint32_t bd[2] = {box[0], box[1]};
-  cuuint32_t es[2] = {1, 1};
-  return encode(map, dtype, 2, const_cast<void*>(base), gd, gs, bd, es,
+  if (!encode || rank < 1 || rank > 5) return false;
+  cuuint64_t gd[5], gs[5];
+  cuuint32_t bd[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bd[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) gs[i] = strides[i];
+  }
+  return encode(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bd, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -25,6 +25,19 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// x rounded to tf32 (10 explicit mantissa bits; nearest, ties to even), kept
+// in an fp32 container with the low 13 bits zero.  x = tf32_rn(x) + lo with lo
+// exact in fp32: the split the 3xTF32 products use.
+__host__ __device__ __forceinline__ float tf32_rn(float x) {
+#ifdef __CUDA_ARCH__
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
+#else
+  return x;
+#endif
+}
+
 // ---- mbarrier ---------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

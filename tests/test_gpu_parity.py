@@ -121,9 +121,39 @@ def test_hessian_zero_tokens_zeroes_h():
 
 
 # --------------------------------------------------------------------------
+# the factorisation's tensor-core GEMM (3xTF32) against fp64
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("M,N,K,lower", [(64, 64, 64, 0), (200, 72, 1000, 0), (384, 384, 96, 1),
+                                         (1024, 1024, 1024, 0), (130, 260, 36, 0)])
+def test_gemm_nt_tc_against_fp64(M, N, K, lower):
+    rng = np.random.default_rng(M + N + K)
+    P = rng.standard_normal((M, K)).astype(np.float32)
+    Q = (rng.standard_normal((N, K)) * rng.lognormal(0, 1, size=K)).astype(np.float32)
+    C0 = rng.standard_normal((M, N)).astype(np.float32)
+    Pd, Qd = torch.from_numpy(P).to(DEV), torch.from_numpy(Q).to(DEV)
+    Cd = torch.from_numpy(C0).to(DEV)
+    st = B.nvfp4_gemm_nt_f32(Pd, Qd, Cd, alpha=-0.75, beta=0.5, lower=bool(lower))
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ref = 0.5 * C0.astype(np.float64) - 0.75 * (P.astype(np.float64) @ Q.astype(np.float64).T)
+    got = Cd.cpu().numpy().astype(np.float64)
+    if lower:
+        mask = np.zeros((M, N), bool)
+        for i in range(0, M, 128):
+            mask[i:i + 128, :i + 128] = True
+        assert np.array_equal(got[~mask], C0.astype(np.float64)[~mask])
+        got, ref = got[mask], ref[mask]
+    # fp32-level: each entry within a few ulps of the magnitude of its terms
+    scale = 0.75 * (np.abs(P).astype(np.float64) @ np.abs(Q).astype(np.float64).T)
+    if lower:
+        scale = scale[mask]
+    assert np.all(np.abs(got - ref) <= 4e-6 * (scale + np.abs(ref)) + 1e-30)
+
+
+# --------------------------------------------------------------------------
 # a2-a4 prepare
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("d", [16, 208, 256, 1040])
+@pytest.mark.parametrize("d", [16, 208, 256, 1040, 2000])
 def test_prepare_factor(d):
     rng = np.random.default_rng(d)
     n = 2 * d
