@@ -204,20 +204,24 @@ __global__ void __launch_bounds__(kReplayThreads)
   double* invd = Ut + kUTiles * 256;                         // 128
   double* rows = invd + kLazyBatch;                          // kRowsPerCta x 128
   const int nblk = bw / kBlock;
-  for (int idx = threadIdx.x; idx < kUTiles * 256; idx += blockDim.x) {
-    const int t = idx >> 8, e = idx & 255;
-    // recover (p, q) of tile t
-    int p = 0;
-    while (p + 1 < kNb && utile(p + 1, p + 1) <= t) ++p;
-    const int q = p + (t - utile(p, p));
-    const int i = e >> 4, j = e & 15;
-    const int gi = 16 * p + i, gj = 16 * q + j;
-    double u = 0.0;
-    if (p < nblk && q < nblk && gj >= gi) u = (double)U[(int64_t)(c0 + gi) * d_in + c0 + gj];
-    Ut[idx] = u;
+  {
+    // Stage the batch's upper block-triangular part of U as 16 x 16 fp64
+    // tiles.  Thread t handles element e = t of every tile (kReplayThreads ==
+    // 256 == tile size) and issues all its loads before any store.
+    static_assert(kReplayThreads == 256, "one tile element per thread");
+    const int e = threadIdx.x, i = e >> 4, j = e & 15;
+    float u[kUTiles];
+#pragma unroll
+    for (int t = 0, p = 0, q = 0; t < kUTiles; ++t) {
+      const int gi = 16 * p + i, gj = 16 * q + j;
+      u[t] = (p < nblk && q < nblk && gj >= gi) ? U[(int64_t)(c0 + gi) * d_in + c0 + gj] : 0.f;
+      if (++q == kNb) q = ++p;   // tiles (p, q), q >= p, row-major
+    }
+#pragma unroll
+    for (int t = 0; t < kUTiles; ++t) Ut[t * 256 + e] = (double)u[t];
+    if (threadIdx.x < bw)
+      invd[threadIdx.x] = 1.0 / (double)U[(int64_t)(c0 + threadIdx.x) * d_in + c0 + threadIdx.x];
   }
-  for (int i = threadIdx.x; i < bw; i += blockDim.x)
-    invd[i] = 1.0 / (double)U[(int64_t)(c0 + i) * d_in + c0 + i];
   __syncthreads();
 
   const double sg = (double)*sg_ptr;
