@@ -122,15 +122,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def phase_work(d_out, d_in, n_tok):
     """Algorithmic work per phase of one step (flops or bytes)."""
-    upd = 0
+    upd_bytes = 0
     for c0 in range(0, d_in, 128):
         e = min(c0 + 128, d_in)
-        upd += 2 * d_out * (e - c0) * (d_in - e)
+        # fp64 W~[:, e:] read and written once per lazy batch
+        upd_bytes += 16 * d_out * (d_in - e)
+    nb = d_in // 16
     return {
         "hessian_flops": n_tok * d_in * (d_in + 1),          # symmetric half, 2 flops per MAC
-        "prepare_flops": 2 * d_in ** 3 // 3,
-        "update_flops": upd,
-        "replay_bytes": d_out * d_in * (8 + 8 + 0.5) + d_out * d_in / 16,
+        "prepare_flops": 2 * d_in ** 3 // 3,                  # Cholesky 1/3 d^3 + trtri 1/3 d^3
+        "update_bytes": upd_bytes,
+        # fp64 flops of the Schur Replay per weight: 16 candidates x (scale,
+        # residual, delta, score: 6 flops + 7.5 in-block update FMAs) plus the
+        # in-batch update (3.5 later blocks of 16 columns on average)
+        "replay_flops": d_out * nb * 16 * (16 * (6 + 15) + 2 * 16 * 3.5),
         "dequant_bytes": d_out * d_in * (0.5 + 2) + d_out * d_in / 16,
     }
 
@@ -228,27 +233,36 @@ def run_ours(args, rank, world, local_rank):
     ph_ms = {n: ms_ph[i] / args.steps for i, n in enumerate(names[:5])}
     ph_launch = {n: ln_ph[i] // args.steps for i, n in enumerate(names)}
     sm_ghz = peaks.get("sm_max_mhz", 1965.0) / 1e3
-    fp64_peak = N_SM * FP64_LANES_PER_SM * 2 * sm_ghz / 1e3    # TFLOP/s
-    fp32_peak = N_SM * FP32_LANES_PER_SM * 2 * sm_ghz / 1e3
-    bf16_peak = peaks["bf16_tflops"]
+    fp64_peak = N_SM * FP64_LANES_PER_SM * 2 * sm_ghz / 1e3    # TFLOP/s, derived
+    bf16_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])   # inside a long step
+    tf32x3_peak = bf16_peak * (1.1 / 2.25) / 3    # tf32 = nominal 1.1/2.25 of bf16; 3 MMAs
     hbm = peaks["hbm_gbs"]
     # per-phase roofline (what bounds each phase in this build)
     rl = {
-        "hessian": ("alu", wk["hessian_flops"] / (ph_ms["hessian"] * 1e9), fp32_peak, "TFLOP/s"),
-        "prepare": ("alu", wk["prepare_flops"] / (ph_ms["prepare"] * 1e9), fp32_peak, "TFLOP/s"),
-        "update": ("alu", wk["update_flops"] / (ph_ms["update"] * 1e9), fp64_peak, "TFLOP/s"),
-        "replay": ("hbm", wk["replay_bytes"] / (ph_ms["replay"] * 1e6), hbm, "GB/s"),
-        "dequant": ("hbm", wk["dequant_bytes"] / (ph_ms["dequant"] * 1e6), hbm, "GB/s"),
+        "hessian": ("tensor", wk["hessian_flops"] / (ph_ms["hessian"] * 1e9), bf16_peak,
+                    "TFLOP/s", "hessian_tc_kernel (tcgen05 kind::f16)"),
+        "prepare": ("tensor", wk["prepare_flops"] / (ph_ms["prepare"] * 1e9), tf32x3_peak,
+                    "TFLOP/s", "chol_panel_kernel + gemm_nt_tc_kernel (tcgen05 3xTF32)"),
+        "update": ("hbm", wk["update_bytes"] / (ph_ms["update"] * 1e6), hbm, "GB/s",
+                   "update_tc_kernel (tcgen05 3xTF32, fp64 W~ read-modify-write)"),
+        "replay": ("alu", wk["replay_flops"] / (ph_ms["replay"] * 1e9), fp64_peak, "TFLOP/s",
+                   "schur_replay_batch_kernel (fp64 CUDA cores)"),
+        "dequant": ("hbm", wk["dequant_bytes"] / (ph_ms["dequant"] * 1e6), hbm, "GB/s",
+                    "dequant_kernel"),
     }
     dom = max(rl, key=lambda n: ph_ms[n])
-    bound, ach, peak, unit = rl[dom]
+    bound, ach, peak, unit, kern = rl[dom]
+    peak_src = {"hessian": "measured bf16 sustained", "dequant": "measured HBM copy",
+                "update": "measured HBM copy",
+                "prepare": "measured bf16 sustained x 1.1/2.25 (tf32) / 3 (3xTF32)",
+                "replay": "derived: 148 SMs x 64 fp64 lanes x 2 x max SM clock"}
     solve_ms = ph_ms["prepare"] + ph_ms["replay"] + ph_ms["update"]
     weights = d_out * d_in
     out = {
         "metric": METRIC, "value": world * weights / (step_ms / 1e3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in; f32 H and U; f64 solve", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16 in; f32 H, U (3xTF32 GEMMs); f64 working copy and replay", "data": "synthetic",
         "config": {"workload": args.workload, "d_out": d_out, "d_in": d_in, "n_tok": n_tok,
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
                    "parallelism": f"{world} independent layer solves (one per GPU)"},
@@ -257,12 +271,12 @@ def run_ours(args, rank, world, local_rank):
         "hessian_tflops": {"algorithmic_syrk_half": wk["hessian_flops"] / (ph_ms["hessian"] * 1e9),
                            "conventional_2Nd2": 2 * n_tok * d_in * d_in / (ph_ms["hessian"] * 1e9)},
         "phase_ms": ph_ms, "phase_launches": ph_launch,
-        "phase_roofline": {n: {"bound": b, "achieved": a, "peak": p, "unit": u, "frac": a / p}
-                           for n, (b, a, p, u) in rl.items()},
-        "roofline": {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                     "frac": ach / peak, "traffic": None,
-                     "peak_source": peaks["source"] if unit == "GB/s" else
-                     "derived: 148 SMs x lanes x 2 x max SM clock"},
+        "phase_roofline": {n: {"bound": b, "achieved": a, "peak": p, "unit": u, "frac": a / p,
+                               "kernels": k_, "peak_source": peak_src[n]}
+                           for n, (b, a, p, u, k_) in rl.items()},
+        "roofline": {"phase": dom, "kernel": kern, "bound": bound, "achieved": ach, "peak": peak,
+                     "unit": unit, "frac": ach / peak, "traffic": None,
+                     "peak_source": f"{peak_src[dom]} ({peaks['source']})"},
         "e2e": {"value": world * weights / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": W.numel() * W.element_size() + X.numel() * X.element_size(),
                 "d2h_bytes_per_step": codes_h.numel() + scales_h.numel() + 4},

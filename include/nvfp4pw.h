@@ -226,6 +226,45 @@ nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t
                                nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Batched forms: `count` independent problems per call                      */
+/* ("Replay the Curvature", Abstract: a layer's solve is independent of the  */
+/* other layers' and, in a mixture-of-experts layer, every expert is its own */
+/* linear layer with its own Hessian).                                       */
+/* ------------------------------------------------------------------------ */
+/* Every array argument is a HOST array of length count holding the per-problem
+ * value of the argument of the same name in the single-problem call (device
+ * pointers, sizes, workspaces); the per-problem rules, layouts and status words
+ * are those of the single-problem call.  Optional per-problem pointers
+ * (dead, lambda_out, err_out) may be given as a NULL array.  The problems run
+ * concurrently on an internal pool of 8 streams per device that fork from and
+ * join back into `stream`: when the call returns, all of the work is ordered
+ * before anything later queued on `stream`.  The first failing problem's host
+ * status is returned (later problems are still issued).  count == 0 is a
+ * no-op; count < 0 or a NULL required array is NVFP4_ERR_INVALID_ARG. */
+nvfp4_status nvfp4_hessian_accumulate_batched(int count, float* const* H, const void* const* X,
+                                              nvfp4_dtype x_dtype, const int64_t* n_tok,
+                                              const int64_t* d, int beta,
+                                              nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_gptq_prepare_batched(int count, const float* const* H, const int64_t* d,
+                                        float damp, float* const* U, uint8_t* const* dead,
+                                        float* const* lambda_out, void* const* ws,
+                                        const size_t* ws_bytes, nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_gptq_schur_replay_quantize_batched(
+    int count, const void* const* W, nvfp4_dtype w_dtype, const int64_t* d_out,
+    const int64_t* d_in, const float* const* U, const nvfp4_solve_params* params,
+    const uint8_t* const* dead, uint8_t* const* codes, uint8_t* const* scales,
+    float* const* global_scale, double* const* err_out, void* const* ws,
+    const size_t* ws_bytes, nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_dequant_batched(int count, const uint8_t* const* codes,
+                                   const uint8_t* const* scales,
+                                   const float* const* global_scale, const int64_t* d_out,
+                                   const int64_t* d_in, void* const* out, nvfp4_dtype out_dtype,
+                                   nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Diagnostics: launch accounting and per-phase device timing                */
 /* (measurement support; the paper has no counterpart)                       */
 /* ------------------------------------------------------------------------ */

@@ -63,6 +63,12 @@ def lib():
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
                  vp], i32),
             "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
+            "nvfp4_hessian_accumulate_batched": ([i32, vp, vp, i32, vp, vp, i32, vp], i32),
+            "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, vp, vp], i32),
+            "nvfp4_gptq_schur_replay_quantize_batched": (
+                [i32, vp, i32, vp, vp, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
+                 vp, vp], i32),
+            "nvfp4_dequant_batched": ([i32, vp, vp, vp, vp, vp, vp, i32, vp], i32),
             "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
                                    vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
@@ -194,3 +200,67 @@ def nvfp4_gemm_nt_f32(P, Q, C, alpha=1.0, beta=0.0, lower=False, status=None, st
         M, N, K, float(alpha), _ptr(P), P.stride(0), _ptr(Q), Q.stride(0), float(beta), _ptr(C),
         C.stride(0), int(bool(lower)), _ptr(status), _stream(stream)))
     return status
+
+
+# ---------------------------------------------------------------------------
+# batched forms: lists of per-problem tensors -> host arrays of pointers/sizes
+# ---------------------------------------------------------------------------
+def _ptrs(ts):
+    """Host array of device pointers (NULL for None entries), kept alive by
+    the caller holding the returned object."""
+    arr = (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+    return arr
+
+
+def _i64s(vals):
+    return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])
+
+
+def _sizes(ws):
+    return (ctypes.c_size_t * len(ws))(*[w.numel() for w in ws])
+
+
+def _opt(ts):
+    return None if ts is None else _ptrs(ts)
+
+
+def nvfp4_hessian_accumulate_batched(Hs, Xs, beta=0, stream=None):
+    n = len(Hs)
+    if len({x.dtype for x in Xs}) > 1:
+        raise TypeError("all X must share one dtype")
+    _check("nvfp4_hessian_accumulate_batched", lib().nvfp4_hessian_accumulate_batched(
+        n, _ptrs(Hs), _ptrs(Xs), _dtype_code(Xs[0]) if n else 0,
+        _i64s([x.shape[0] for x in Xs]), _i64s([x.shape[1] for x in Xs]), int(beta),
+        _stream(stream)))
+
+
+def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, wss=None, stream=None):
+    n = len(Hs)
+    _check("nvfp4_gptq_prepare_batched", lib().nvfp4_gptq_prepare_batched(
+        n, _ptrs(Hs), _i64s([h.shape[0] for h in Hs]), float(damp), _ptrs(Us), _opt(deads),
+        _opt(lambdas), _ptrs(wss), _sizes(wss), _stream(stream)))
+
+
+def nvfp4_gptq_schur_replay_quantize_batched(Ws, Us, codes, scales, global_scales,
+                                             errs=None, deads=None, wss=None, params=None,
+                                             stream=None):
+    n = len(Ws)
+    if len({w.dtype for w in Ws}) > 1:
+        raise TypeError("all W must share one dtype")
+    p = params if params is not None else default_params()
+    _check("nvfp4_gptq_schur_replay_quantize_batched",
+           lib().nvfp4_gptq_schur_replay_quantize_batched(
+               n, _ptrs(Ws), _dtype_code(Ws[0]) if n else 0, _i64s([w.shape[0] for w in Ws]),
+               _i64s([w.shape[1] for w in Ws]), _ptrs(Us), ctypes.byref(p), _opt(deads),
+               _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _opt(errs), _ptrs(wss),
+               _sizes(wss), _stream(stream)))
+
+
+def nvfp4_dequant_batched(codes, scales, global_scales, outs, stream=None):
+    n = len(outs)
+    if len({o.dtype for o in outs}) > 1:
+        raise TypeError("all outputs must share one dtype")
+    _check("nvfp4_dequant_batched", lib().nvfp4_dequant_batched(
+        n, _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _i64s([o.shape[0] for o in outs]),
+        _i64s([o.shape[1] for o in outs]), _ptrs(outs), _dtype_code(outs[0]) if n else 0,
+        _stream(stream)))

@@ -24,7 +24,8 @@ struct PrepHeader {   // lives in the workspace header (first 256 bytes)
   int status;
   int pad;
   double diag_sum;
-  float lambda;
+  float lambda;       // fp32 copy for the caller
+  double lambda64;    // used for the damping
 };
 
 // Sum of the diagonal (dead entries counted as 1), dead flags, lambda.
@@ -48,8 +49,10 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int64_t d, float 
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (threadIdx.x == 0) {
       hdr->diag_sum = s;
-      const float lam = (float)((double)damp * (s / (double)d));
+      const double lam64 = (double)damp * (s / (double)d);
+      const float lam = (float)lam64;
       hdr->lambda = lam;
+      hdr->lambda64 = lam64;
       if (lambda_out) *lambda_out = lam;
     }
   }
@@ -58,27 +61,29 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int64_t d, float 
 // A[i][j] = H_d[d-1-i][d-1-j]; dead diagonal entries become 1 + lambda.
 // Also zero-fills X (the inverse is built from its block diagonal outward).
 __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
-                                    float* __restrict__ A, float* __restrict__ X,
+                                    double* __restrict__ A, double* __restrict__ X,
                                     PrepHeader* hdr) {
-  const float lam = hdr->lambda;
+  const double lam = hdr->lambda64;
   const int64_t total = d * d;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
     const int64_t i = idx / d, j = idx - i * d;
-    float h = H[(d - 1 - i) * d + (d - 1 - j)];
+    const float h = H[(d - 1 - i) * d + (d - 1 - j)];
     if (!isfinite(h)) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
-    if (i == j) h = (h == 0.f ? 1.f : h) + lam;
-    A[idx] = h;
-    X[idx] = 0.f;
+    double a = (double)h;
+    if (i == j) a = (h == 0.f ? 1.0 : a) + lam;
+    A[idx] = a;
+    X[idx] = 0.0;
   }
 }
 
 // One panel of the right-looking Cholesky: columns k .. k+kb-1 of A (lower,
 // already updated by the earlier panels).  Every CTA factors the 64 x 64
 // diagonal block A11 = L11 L11^T and inverts L11 in fp64 (redundantly: no CTA
-// waits for another); CTA 0 then writes L11 into A and X11 = L11^-1,
-// Y11 = X11^T into the diagonal blocks of X and Y, every other CTA solves its
-// own 64-row slice of the panel below, L21 = A21 X11^T, in place.
+// waits for another); CTA 0 then writes X11 = L11^-1 and Y11 = X11^T into the
+// diagonal blocks of X and Y (A11 stays as it is: the other CTAs of the launch
+// may still be reading it), every other CTA solves its own 64-row slice of the
+// panel below, L21 = A21 X11^T, in place.
 //
 // The 64 x 64 block is itself blocked by 16 (a per-column CTA barrier costs
 // far more than the arithmetic of a column):
@@ -162,8 +167,8 @@ __device__ __forceinline__ void factor_invert_16(double (*S)[kPitch], double (*X
 }
 
 __global__ void __launch_bounds__(kPanelThreads)
-    chol_panel_kernel(float* __restrict__ A, int64_t d, int64_t k, int kb,
-                      float* __restrict__ X, float* __restrict__ Y, PrepHeader* hdr) {
+    chol_panel_kernel(double* __restrict__ A, int64_t d, int64_t k, int kb,
+                      double* __restrict__ X, double* __restrict__ Y, PrepHeader* hdr) {
   extern __shared__ double dsm[];
   double(*S)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm);             // A11 -> L11
   double(*Xd)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + NB * kPitch);   // X11
@@ -176,19 +181,19 @@ __global__ void __launch_bounds__(kPanelThreads)
 
   {   // all global loads of a thread are issued before any is used
     constexpr int kPer = NB * NB / kPanelThreads;   // 16
-    float a11[kPer], a21[kPer];
+    double a11[kPer], a21[kPer];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
-      a11[q] = (i < kb && l <= i) ? A[(k + i) * d + k + l] : 0.f;
-      a21[q] = (i < rows && l < kb) ? A[(r0 + i) * d + k + l] : 0.f;
+      a11[q] = (i < kb && l <= i) ? A[(k + i) * d + k + l] : 0.0;
+      a21[q] = (i < rows && l < kb) ? A[(r0 + i) * d + k + l] : 0.0;
     }
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
-      S[i][l] = (i < kb && l < kb) ? (double)a11[q] : (i == l ? 1.0 : 0.0);
+      S[i][l] = (i < kb && l < kb) ? a11[q] : (i == l ? 1.0 : 0.0);
       Xd[i][l] = 0.0;
-      R[i][l] = (double)a21[q];
+      R[i][l] = a21[q];
     }
   }
   __syncthreads();
@@ -252,8 +257,9 @@ __global__ void __launch_bounds__(kPanelThreads)
   if (blockIdx.x == 0) {
     for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
       const int i = idx / kb, j = idx % kb;
-      if (j <= i) A[(k + i) * d + k + j] = (float)S[i][j];
-      const float x = (float)Xd[i][j];
+      // L11 itself is not written back: nothing reads the diagonal blocks of L
+      // later, and the other CTAs of this launch may still be reading A11.
+      const double x = Xd[i][j];
       X[(k + i) * d + k + j] = x;            // lower (zeros above)
       Y[(k + j) * d + k + i] = x;            // its transpose, upper
     }
@@ -285,26 +291,26 @@ __global__ void __launch_bounds__(kPanelThreads)
 #pragma unroll
     for (int b = 0; b < 4; ++b)
       if (i0 + a < rows && l0 + b < kb)
-        A[(r0 + i0 + a) * d + k + l0 + b] = (float)acc[a][b];
+        A[(r0 + i0 + a) * d + k + l0 + b] = acc[a][b];
 }
 
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
-__global__ void reverse_to_upper_kernel(const float* __restrict__ X, int64_t d,
+__global__ void reverse_to_upper_kernel(const double* __restrict__ X, int64_t d,
                                         float* __restrict__ U) {
   const int64_t total = d * d;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
     const int64_t i = idx / d, j = idx - i * d;
-    U[idx] = (j >= i) ? X[(d - 1 - i) * d + (d - 1 - j)] : 0.f;
+    U[idx] = (j >= i) ? (float)X[(d - 1 - i) * d + (d - 1 - j)] : 0.f;
   }
 }
 
 struct PrepLayout {
   PrepHeader* hdr;
-  float* A;   // J H_d J, then its Cholesky factor L (lower)
-  float* X;   // L^-1 (lower)
-  float* Y;   // L^-T (upper)
-  float* T;   // scratch of the inverse doubling
+  double* A;   // J H_d J, then its Cholesky factor L (lower)
+  double* X;   // L^-1 (lower)
+  double* Y;   // L^-T (upper)
+  double* T;   // scratch of the inverse doubling
 };
 
 PrepLayout prep_layout(void* ws, int64_t d) {
@@ -312,13 +318,13 @@ PrepLayout prep_layout(void* ws, int64_t d) {
   PrepLayout L;
   L.hdr = reinterpret_cast<PrepHeader*>(p);
   size_t off = kWsHeader;
-  L.A = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d * d);
-  L.X = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d * d);
-  L.Y = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d * d);
-  L.T = reinterpret_cast<float*>(p + off);
+  L.A = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * d * d);
+  L.X = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * d * d);
+  L.Y = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * d * d);
+  L.T = reinterpret_cast<double*>(p + off);
   return L;
 }
 
@@ -330,8 +336,8 @@ int grid_for(int64_t n, int threads) {
 }  // namespace
 
 size_t prepare_ws_bytes(int64_t d) {
-  return kWsHeader + 3 * align256(sizeof(float) * d * d) +
-         align256(sizeof(float) * (size_t)((d * d + 3) / 4 + d * NB));
+  return kWsHeader + 3 * align256(sizeof(double) * d * d) +
+         align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB));
 }
 
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uint8_t* dead,
@@ -345,8 +351,7 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
 
-  NVFP4_CUDA_TRY(cudaMemsetAsync(L.Y, 0, sizeof(float) * d * d, st));
-  int* status = &L.hdr->status;
+  NVFP4_CUDA_TRY(cudaMemsetAsync(L.Y, 0, sizeof(double) * d * d, st));
 
   // Blocked right-looking Cholesky of A (lower): per 64-column panel, one
   // fused panel kernel (diagonal factor + inverse + panel solve), then the
@@ -362,9 +367,9 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     NVFP4_LAUNCH_CHECK();
     count_launches(1);
     if (m <= 0) break;
-    const float* L21 = L.A + (k + kb) * d + k;
-    nvfp4_status s = gemm_nt_tc((int)m, (int)m, kb, -1.f, L21, d, 0, L21, d, 0, 1.f,
-                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 1, status,
+    const double* L21 = L.A + (k + kb) * d + k;
+    nvfp4_status s = dgemm_nt((int)m, (int)m, kb, -1.0, L21, d, 0, L21, d, 0, 1.0,
+                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 1,
                                 st);
     if (s != NVFP4_OK) return s;
   }
@@ -377,12 +382,11 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     const int64_t npairs = d / (2 * b);
     const int64_t stride = 2 * b * (d + 1);
     if (npairs > 0) {
-      nvfp4_status s = gemm_nt_tc((int)b, (int)b, (int)b, 1.f, L.Y, d, stride, L.A + b * d, d,
-                                  stride, 0.f, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0,
-                                  status, st);
+      nvfp4_status s = dgemm_nt((int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
+                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, st);
       if (s != NVFP4_OK) return s;
-      s = gemm_nt_tc((int)b, (int)b, (int)b, -1.f, L.X + b * (d + 1), d, stride, L.T, b, b * b,
-                     0.f, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, status,
+      s = dgemm_nt((int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
+                     0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0,
                      st);
       if (s != NVFP4_OK) return s;
     }
@@ -390,13 +394,12 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     const int64_t rr = d - r0 - b;
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
-      nvfp4_status s = gemm_nt_tc((int)b, (int)rr, (int)b, 1.f, L.Y + o, d, 0,
-                                  L.A + o + b * d, d, 0, 0.f, L.T, rr, 0, nullptr, 0, 0, 1, 0,
-                                  status, st);
+      nvfp4_status s = dgemm_nt((int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0,
+                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, st);
       if (s != NVFP4_OK) return s;
       // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
-      s = gemm_nt_tc((int)rr, (int)b, (int)rr, -1.f, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
-                     0.f, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, status, st);
+      s = dgemm_nt((int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
+                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, st);
       if (s != NVFP4_OK) return s;
     }
   }

@@ -59,6 +59,11 @@ def test_host_side_checks_need_no_device():
         ctypes.c_void_p(256), 0, 4096, 4096, ctypes.c_void_p(256), null, null,
         ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), null, null,
         null) == 3
+    # batched forms: count < 0 or missing arrays are rejected on the host
+    assert L.nvfp4_hessian_accumulate_batched(-1, null, null, 0, null, null, 0, null) == 1
+    assert L.nvfp4_gptq_prepare_batched(2, null, null, 0.01, null, null, null, null, null,
+                                        null) == 1
+    assert L.nvfp4_dequant_batched(0, null, null, null, null, null, null, 0, null) == 0
     assert L.nvfp4_status_string(5) == b"damped Hessian is not positive definite"
     assert L.nvfp4_prepare_workspace_size(-1) == 0
 
