@@ -88,12 +88,14 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
                         cudaStream_t st);
 
 // C = beta C + alpha P Q^T in fp64 on the CUDA cores (same operand conventions
-// as gemm_nt_tc; C2 = C^T needs beta == 0; lower: 64 x 64 tiles on or below
-// the diagonal only).
+// as gemm_nt_tc; C2 = C^T needs beta == 0; lower: only tiles on or below the
+// diagonal; ktri: 0 dense P, 1 P upper triangular, 2 P lower triangular -- the
+// zero part of K is skipped).
 nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_t ldp,
                       int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
                       double beta, double* C, int64_t ldc, int64_t strideC, double* C2,
-                      int64_t ldc2, int64_t strideC2, int batch, int lower, cudaStream_t st);
+                      int64_t ldc2, int64_t strideC2, int batch, int lower, int ktri,
+                      cudaStream_t st);
 
 // ---- kernel launchers implemented in the .cu files -------------------------
 bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,

@@ -8,96 +8,146 @@
 // decisions follow an exact solve: the damped Hessian of a layer calibrated on
 // few tokens is ill-conditioned (1e4 and more), and a factor carried in fp32
 // arithmetic moves block decisions that sit a few 1e-5 from a tie.  The
-// 5th-generation tensor cores have no fp64 kind, and B200's fp64 tensor and
-// CUDA-core rates are the same, so this is a register-tiled DFMA kernel:
-// 64 x 64 tiles, 256 threads with 4 x 4 outputs each, K in steps of 16
-// staged transposed in shared memory (double buffered through registers).
+// 5th-generation tcgen05 instructions have no fp64 kind; fp64 runs on the
+// warp-level mma.sync m8n8k4 (measured at ~36.7 TF/s on B200, its fp64 peak,
+// with 8 warps per SM, and 8x fewer instructions than fp64 FMAs):
+// 64 x 64 or 128 x 128 CTA tiles, 8 warps of 32 x 16 or 64 x 32, K in steps
+// of 16 staged in shared memory (double buffered through registers); a
+// triangular P skips its zero half of K.
 #include "common.cuh"
 
 namespace nvfp4 {
 namespace {
 
-constexpr int DM = 64, DN = 64, DK = 16;
-constexpr int kDThreads = 256;
+constexpr int DK = 16;
+constexpr int kDThreads = 256;   // 8 warps: 2 along M x 4 along N
 
+// D (8x8) += A (8x4, row) * B (4x8, col) in fp64 on the tensor cores.
+// Fragments: a = A[lane/4][lane%4], b = B[lane%4][lane/4],
+// d = D[lane/4][2*(lane%4) + {0,1}].
+__device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+// CTA tile (16 T) x (32 T) ... see below; T = 4: 64 x 64 (each warp 32 x 16),
+// T = 8: 128 x 128 (each warp 64 x 32).  ktri: 0 dense P; 1 P upper triangular
+// (P[m][k] = 0 for k < m), so a tile's K range starts at its first row; 2 P
+// lower triangular (P[m][k] = 0 for k > m), so it ends after its last row.
+template <int T>
 __global__ void __launch_bounds__(kDThreads)
     dgemm_nt_kernel(int M, int N, int K, double alpha, const double* __restrict__ P,
                     int64_t ldp, int64_t strideP, const double* __restrict__ Q, int64_t ldq,
                     int64_t strideQ, double beta, double* __restrict__ C, int64_t ldc,
                     int64_t strideC, double* __restrict__ C2, int64_t ldc2, int64_t strideC2,
-                    int lower) {
-  __shared__ double Ps[2][DK][DM + 2];
-  __shared__ double Qs[2][DK][DN + 2];
-  int tm = blockIdx.y, tn = blockIdx.x;
+                    int lower, int ktri) {
+  constexpr int TL = 16 * T;            // CTA tile side (64 or 128)
+  constexpr int WM = TL / 2, WN = TL / 4;   // warp tile
+  constexpr int MT = WM / 8, NT = WN / 8;   // 8x8 MMA tiles per warp
+  constexpr int PITCH = DK + 4;         // 20 doubles: fragment loads at the 2-wavefront minimum
+  constexpr int PER = TL * DK / kDThreads;  // values per thread per operand and K step
+  extern __shared__ double dsm[];
+  double(*Ps)[TL][PITCH] = reinterpret_cast<double(*)[TL][PITCH]>(dsm);
+  double(*Qs)[TL][PITCH] = reinterpret_cast<double(*)[TL][PITCH]>(dsm + 2 * TL * PITCH);
+  const int tm = blockIdx.y, tn = blockIdx.x;
   if (lower && tn > tm) return;
   const int b = blockIdx.z;
   P += b * strideP;
   Q += b * strideQ;
   C += b * strideC;
   if (C2) C2 += b * strideC2;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int m0 = tm * DM, n0 = tn * DN;
-  // loader mapping: 64 rows x 16 k per operand = 1024 values, 4 per thread
-  const int lr = tid >> 2, lk = (tid & 3) * 4;
-  double pr[4], qr[4];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = tm * TL, n0 = tn * TL;
+  const int wm0 = (warp & 1) * WM, wn0 = (warp >> 1) * WN;
+  int kbeg = 0, kend = K;
+  if (ktri == 1) kbeg = (m0 / DK) * DK;
+  if (ktri == 2) kend = (m0 + TL) < K ? (m0 + TL) : K;
+  // loader: row lr, PER consecutive k values from lk
+  constexpr int KG = DK / PER;
+  const int lr = tid / KG, lk = (tid % KG) * PER;
+  double pr[PER], qr[PER];
   auto load = [&](int k0) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    for (int t = 0; t < PER; ++t) {
       const int k = k0 + lk + t;
-      pr[t] = (m0 + lr < M && k < K) ? P[(int64_t)(m0 + lr) * ldp + k] : 0.0;
-      qr[t] = (n0 + lr < N && k < K) ? Q[(int64_t)(n0 + lr) * ldq + k] : 0.0;
+      pr[t] = (m0 + lr < M && k < kend) ? P[(int64_t)(m0 + lr) * ldp + k] : 0.0;
+      qr[t] = (n0 + lr < N && k < kend) ? Q[(int64_t)(n0 + lr) * ldq + k] : 0.0;
     }
   };
   auto stash = [&](int buf) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      Ps[buf][lk + t][lr] = pr[t];
-      Qs[buf][lk + t][lr] = qr[t];
+    for (int t = 0; t < PER; ++t) {
+      Ps[buf][lr][lk + t] = pr[t];
+      Qs[buf][lr][lk + t] = qr[t];
     }
   };
-  double acc[4][4];
+  double acc[MT][NT][2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < MT; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-  const int nk = (K + DK - 1) / DK;
+    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+  const int nk = kend > kbeg ? (kend - kbeg + DK - 1) / DK : 0;
   if (nk > 0) {
-    load(0);
+    load(kbeg);
     stash(0);
   }
   __syncthreads();
+  const int fr = lane >> 2, fc = lane & 3;
   for (int kt = 0; kt < nk; ++kt) {
     const int cur = kt & 1;
-    if (kt + 1 < nk) load((kt + 1) * DK);
+    if (kt + 1 < nk) load(kbeg + (kt + 1) * DK);
 #pragma unroll
-    for (int k = 0; k < DK; ++k) {
-      double a[4], c[4];
+    for (int k4 = 0; k4 < DK; k4 += 4) {
+      double af[MT], bf[NT];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = Ps[cur][k][ty + 16 * i];
+      for (int i = 0; i < MT; ++i) af[i] = Ps[cur][wm0 + 8 * i + fr][k4 + fc];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) c[j] = Qs[cur][k][tx + 16 * j];
+      for (int j = 0; j < NT; ++j) bf[j] = Qs[cur][wn0 + 8 * j + fr][k4 + fc];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < MT; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
+        for (int j = 0; j < NT; ++j) dmma(acc[i][j][0], acc[i][j][1], af[i], bf[j]);
     }
     if (kt + 1 < nk) stash(cur ^ 1);
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty + 16 * i;
+  for (int i = 0; i < MT; ++i) {
+    const int m = m0 + wm0 + 8 * i + fr;
     if (m >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx + 16 * j;
-      if (n >= N) continue;
-      double x = alpha * acc[i][j];
-      if (beta != 0.0) x = fma(beta, C[(int64_t)m * ldc + n], x);
-      C[(int64_t)m * ldc + n] = x;
-      if (C2) C2[(int64_t)n * ldc2 + m] = x;
-    }
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = n0 + wn0 + 8 * j + 2 * fc + h;
+        if (n >= N) continue;
+        double x = alpha * acc[i][j][h];
+        if (beta != 0.0) x = fma(beta, C[(int64_t)m * ldc + n], x);
+        C[(int64_t)m * ldc + n] = x;
+        if (C2) C2[(int64_t)n * ldc2 + m] = x;
+      }
   }
+}
+
+template <int T>
+nvfp4_status launch_dgemm(int M, int N, int K, double alpha, const double* P, int64_t ldp,
+                          int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
+                          double beta, double* C, int64_t ldc, int64_t strideC, double* C2,
+                          int64_t ldc2, int64_t strideC2, int batch, int lower, int ktri,
+                          cudaStream_t st) {
+  constexpr int TL = 16 * T;
+  const size_t smem = sizeof(double) * 4 * TL * (DK + 4);
+  const dim3 grid((unsigned)((N + TL - 1) / TL), (unsigned)((M + TL - 1) / TL), (unsigned)batch);
+  if (grid.y > 65535) return NVFP4_ERR_SHAPE;
+  NVFP4_CUDA_TRY(cudaFuncSetAttribute(dgemm_nt_kernel<T>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dgemm_nt_kernel<T><<<grid, kDThreads, smem, st>>>(M, N, K, alpha, P, ldp, strideP, Q, ldq,
+                                                    strideQ, beta, C, ldc, strideC, C2, ldc2,
+                                                    strideC2, lower, ktri);
+  NVFP4_LAUNCH_CHECK();
+  count_launches(1);
+  return NVFP4_OK;
 }
 
 }  // namespace
@@ -105,16 +155,18 @@ __global__ void __launch_bounds__(kDThreads)
 nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_t ldp,
                       int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
                       double beta, double* C, int64_t ldc, int64_t strideC, double* C2,
-                      int64_t ldc2, int64_t strideC2, int batch, int lower, cudaStream_t st) {
+                      int64_t ldc2, int64_t strideC2, int batch, int lower, int ktri,
+                      cudaStream_t st) {
   if (M <= 0 || N <= 0 || batch <= 0) return NVFP4_OK;
-  if ((C2 && beta != 0.0) || (lower && M != N) || batch > 65535) return NVFP4_ERR_INVALID_ARG;
-  const dim3 grid((unsigned)((N + DN - 1) / DN), (unsigned)((M + DM - 1) / DM), (unsigned)batch);
-  if (grid.y > 65535) return NVFP4_ERR_SHAPE;
-  dgemm_nt_kernel<<<grid, kDThreads, 0, st>>>(M, N, K, alpha, P, ldp, strideP, Q, ldq, strideQ,
-                                              beta, C, ldc, strideC, C2, ldc2, strideC2, lower);
-  NVFP4_LAUNCH_CHECK();
-  count_launches(1);
-  return NVFP4_OK;
+  if ((C2 && beta != 0.0) || (lower && M != N) || batch > 65535 || ktri < 0 || ktri > 2)
+    return NVFP4_ERR_INVALID_ARG;
+  // 128 x 128 tiles once there are enough of them to fill the GPU, else 64 x 64
+  const int64_t big_tiles = (int64_t)((M + 127) / 128) * ((N + 127) / 128) * batch;
+  if (big_tiles >= 2 * kNumSMs)
+    return launch_dgemm<8>(M, N, K, alpha, P, ldp, strideP, Q, ldq, strideQ, beta, C, ldc,
+                           strideC, C2, ldc2, strideC2, batch, lower, ktri, st);
+  return launch_dgemm<4>(M, N, K, alpha, P, ldp, strideP, Q, ldq, strideQ, beta, C, ldc,
+                         strideC, C2, ldc2, strideC2, batch, lower, ktri, st);
 }
 
 }  // namespace nvfp4

@@ -353,25 +353,39 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
 
   NVFP4_CUDA_TRY(cudaMemsetAsync(L.Y, 0, sizeof(double) * d * d, st));
 
-  // Blocked right-looking Cholesky of A (lower): per 64-column panel, one
-  // fused panel kernel (diagonal factor + inverse + panel solve), then the
-  // trailing update A22 -= L21 L21^T on the tensor cores.
+  // Blocked right-looking Cholesky of A (lower), two levels: 64-column panels
+  // (one fused panel kernel each: diagonal factor + inverse + panel solve)
+  // inside 256-column outer blocks.  A panel updates only the rest of its outer
+  // block right away; the trailing matrix beyond the block is updated once per
+  // block, A22 -= L21 L21^T with K = 256, which reads and writes it 4x less
+  // often than per-panel updates would.
+  constexpr int64_t OB = 4 * NB;
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(chol_panel_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kPanelSmem));
-  for (int64_t k = 0; k < d; k += NB) {
-    const int kb = (int)((d - k) < NB ? (d - k) : NB);
-    const int64_t m = d - k - kb;
-    const int grid = 1 + (int)((m + NB - 1) / NB);
-    chol_panel_kernel<<<grid, kPanelThreads, kPanelSmem, st>>>(L.A, d, k, kb, L.X, L.Y, L.hdr);
-    NVFP4_LAUNCH_CHECK();
-    count_launches(1);
-    if (m <= 0) break;
-    const double* L21 = L.A + (k + kb) * d + k;
-    nvfp4_status s = dgemm_nt((int)m, (int)m, kb, -1.0, L21, d, 0, L21, d, 0, 1.0,
-                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 1,
-                                st);
-    if (s != NVFP4_OK) return s;
+  for (int64_t k0 = 0; k0 < d; k0 += OB) {
+    const int64_t kend = (d - k0) < OB ? d : k0 + OB;
+    for (int64_t k = k0; k < kend; k += NB) {
+      const int kb = (int)((d - k) < NB ? (d - k) : NB);
+      const int64_t m = d - k - kb;
+      const int grid = 1 + (int)((m + NB - 1) / NB);
+      chol_panel_kernel<<<grid, kPanelThreads, kPanelSmem, st>>>(L.A, d, k, kb, L.X, L.Y, L.hdr);
+      NVFP4_LAUNCH_CHECK();
+      count_launches(1);
+      const int64_t nc = kend - (k + kb);   // columns of the outer block still to come
+      if (m <= 0 || nc <= 0) continue;
+      const double* L21 = L.A + (k + kb) * d + k;
+      nvfp4_status s = dgemm_nt((int)m, (int)nc, kb, -1.0, L21, d, 0, L21, d, 0, 1.0,
+                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 0, 0, st);
+      if (s != NVFP4_OK) return s;
+    }
+    const int64_t m2 = d - kend;
+    if (m2 > 0) {
+      const double* Lb = L.A + kend * d + k0;
+      nvfp4_status s = dgemm_nt((int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, 0, Lb, d, 0,
+                                1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0, st);
+      if (s != NVFP4_OK) return s;
+    }
   }
 
   // X = L^-1 by recursive doubling over pairs of adjacent diagonal blocks of
@@ -383,10 +397,10 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     const int64_t stride = 2 * b * (d + 1);
     if (npairs > 0) {
       nvfp4_status s = dgemm_nt((int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
-                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, st);
+                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1, st);
       if (s != NVFP4_OK) return s;
       s = dgemm_nt((int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
-                     0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0,
+                     0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, 2,
                      st);
       if (s != NVFP4_OK) return s;
     }
@@ -395,11 +409,11 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
       nvfp4_status s = dgemm_nt((int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0,
-                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, st);
+                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1, st);
       if (s != NVFP4_OK) return s;
       // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
       s = dgemm_nt((int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
-                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, st);
+                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2, st);
       if (s != NVFP4_OK) return s;
     }
   }
