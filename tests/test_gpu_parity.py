@@ -337,3 +337,42 @@ def test_solve_attn_4096_all_rows():
     L_gpu = O.layer_error(W64[rows], Q, H)
     L_ref = O.layer_error(W64[rows], ref["q"], H)
     assert abs(L_gpu - L_ref) <= 1e-4 * L_ref
+
+
+def test_solve_mlp_down_14336_given_hessian_row_sample():
+    """MLP down-projection-shaped layer (4096 x 14336, 8192 SiLU-gated bf16
+    tokens): the GPU Hessian against fp64 (1e-4 Frobenius), then the GPU
+    prepare + quantize of the whole layer from the oracle's fp32-rounded
+    Hessian (8192 tokens for 14336 channels: rank-deficient, so the solve is
+    checked given H), compared with the oracle on a seeded sample of 512 rows
+    (rows are independent given U)."""
+    W, X = synth.mlp_down_silu()
+    d_out, d_in = W.shape
+    Xn = X.double().numpy()
+    H = O.hessian(Xn)
+    Hg = torch.empty((d_in, d_in), dtype=torch.float32, device=DEV)
+    B.nvfp4_hessian_accumulate(Hg, X.to(DEV))
+    torch.cuda.synchronize()
+    assert rel_frob(Hg.cpu().numpy().astype(np.float64), H) < 1e-4
+    del Hg
+    H32 = H.astype(np.float32)
+    Hd32 = torch.from_numpy(H32).to(DEV)
+    U = torch.empty_like(Hd32)
+    wsp = B.workspace(B.nvfp4_prepare_workspace_size(d_in), DEV)
+    B.nvfp4_gptq_prepare(Hd32, 0.01, U, None, None, wsp)
+    codes, scales, sg_gpu, err = gpu_quantize(W, U)
+    assert B.nvfp4_workspace_status(wsp) == 0
+    Hdm, dead, lam = O.damp(H32.astype(np.float64))
+    Uo = O.inverse_cholesky_upper(Hdm)
+    W64 = W.double().numpy()
+    sg = O.global_scale(W64)
+    assert np.float32(sg_gpu) == sg
+    rows = np.sort(np.random.default_rng(102).choice(d_out, 512, replace=False))
+    ref = O.schur_replay_gptq(W64[rows], Uo, sg, return_diag=True)
+    c = classify(ref, Uo, sg, codes[rows], scales[rows], rows)
+    assert c["frac"] <= 1e-3, c
+    assert not c["bad_first"], c
+    Q = O.dequant(codes[rows], scales[rows], sg).astype(np.float64)
+    L_gpu = O.layer_error(W64[rows], Q, H)
+    L_ref = O.layer_error(W64[rows], ref["q"], H)
+    assert abs(L_gpu - L_ref) <= 1e-4 * L_ref
