@@ -140,6 +140,22 @@ def phase_work(d_out, d_in, n_tok):
     }
 
 
+def reduce_max(x, dist, device):
+    """x maximised over all ranks (the step time of the slowest GPU)."""
+    if not dist:
+        return float(x)
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, weights_per_rank, ms_per_step):
+    """Whole-job weights/s: every rank solves its own layer in the step."""
+    return world * weights_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from nvfp4_post_weight_b200 import binding as B
@@ -187,11 +203,8 @@ def run_ours(args, rank, world, local_rank):
     ln_ph = (ctypes.c_longlong * 6)()
     B.lib().nvfp4_profile_end(ms_ph, ln_ph, 6)
     launches = B.lib().nvfp4_launch_count() - n0
-    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    step_ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dist, dev)
     if dist:
-        t = torch.tensor([step_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        step_ms = float(t.item())
         tdist.barrier()
 
     # end to end through the C ABI from pinned host buffers: H2D of W and X,
@@ -219,11 +232,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
         ev2[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev2) / args.steps, dist, dev)
 
     if rank != 0:
         return None
@@ -258,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     solve_ms = ph_ms["prepare"] + ph_ms["replay"] + ph_ms["update"]
     weights = d_out * d_in
     out = {
-        "metric": METRIC, "value": world * weights / (step_ms / 1e3), "unit": UNIT,
+        "metric": METRIC, "value": job_throughput(world, weights, step_ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 in; f32 H; f64 factor (U stored f32); f64 working copy and replay; 3xTF32 update", "data": "synthetic",
@@ -276,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"phase": dom, "kernel": kern, "bound": bound, "achieved": ach, "peak": peak,
                      "unit": unit, "frac": ach / peak, "traffic": None,
                      "peak_source": f"{peak_src[dom]} ({peaks['source']})"},
-        "e2e": {"value": world * weights / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": job_throughput(world, weights, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": W.numel() * W.element_size() + X.numel() * X.element_size(),
                 "d2h_bytes_per_step": codes_h.numel() + scales_h.numel() + 4},
         "gpu_launches": launches,
