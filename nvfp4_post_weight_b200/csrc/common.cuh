@@ -108,10 +108,10 @@ int hessian_tc_take_status(cudaStream_t st);
 // (d_out x 128, fp32 each) and the split rows U = Uh + Ul of one batch,
 // transposed (d_in x 128, fp32 each, rows >= e used).
 struct UpdateMaps {
-  CUtensorMap Dh, Dl, Uh, Ul;
+  CUtensorMap Dh, Dl, Uh, Ul, W;   // W: the fp64 working copy (d_out x d_in)
 };
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
-                      const float* Ul, int64_t d_out, int64_t d_in);
+                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in);
 // W~[:, e:] -= (Dh + Dl)(Uh + Ul)[:, e:] (3xTF32, fp64 W~); a timed-out wait
 // sets NVFP4_ERR_TIMEOUT in *status.
 nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int64_t d_out,

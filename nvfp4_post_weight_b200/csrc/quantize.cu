@@ -374,7 +374,8 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kReplaySmem));
   UpdateMaps maps;
-  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, d_out, d_in)) return NVFP4_ERR_CUDA;
+  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in))
+    return NVFP4_ERR_CUDA;
   const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
   const int rgrid = (int)(row_groups < 2 * kNumSMs ? row_groups : 2 * kNumSMs);
   for (int64_t c0 = 0; c0 < d_in; c0 += kLazyBatch) {

@@ -17,10 +17,15 @@
 //
 // Persistent CTA per SM, warp-specialised:
 //   warp 0     TMA producer: the CTA's 128-row slice of Dh/Dl (all of K,
-//              128 KB, resident while the CTA walks its column tiles) and a
-//              4-stage ring of (Uh, Ul) chunks of 64 columns x 32 K values
+//              128 KB, resident while the CTA walks its column tiles), a
+//              2-stage ring of (Uh, Ul) chunks of 64 columns x 32 K values, and
+//              the W~ tile itself (128 rows x 64 fp64, as two 32-column halves
+//              in two 32 KB buffers, 128-byte swizzled)
 //   warp 1     MMA issuer, 12 MMAs (M=128, N=64, K=8) per K chunk
-//   warps 2-5  epilogue: TMEM -> registers, fp64 read-modify-write of W~
+//   warps 2-5  epilogue: per half tile, TMEM -> registers, W~ -= sum in the
+//              shared-memory buffer, then one thread writes the half back with
+//              a TMA store and frees the buffer once the store has read it.
+//   The W~ traffic (the roofline of this kernel) is all bulk asynchronous.
 // Work item = (128-row block, one of P interleaved column-tile sets).
 #include <cuda.h>
 
@@ -41,17 +46,21 @@ constexpr uint32_t kAChunk = UM * KC * 4;      // 16 KB (hi or lo)
 constexpr uint32_t kABytes = 2 * kNChunks * kAChunk;   // 128 KB
 constexpr uint32_t kBHalf = UN * KC * 4;       // 64 columns x 128 B = 8 KB (hi or lo)
 constexpr uint32_t kBStage = 2 * kBHalf;       // 16 KB
-constexpr int kBStages = 4;
+constexpr int kBStages = 2;
+constexpr int WBOX = 16;                       // fp64 per TMA box row (128 B)
+constexpr uint32_t kWBox = UM * WBOX * 8;      // 16 KB
+constexpr uint32_t kWHalf = 2 * kWBox;         // 32 columns = 32 KB
 constexpr int kThreads = 192;
 constexpr uint32_t kAccCols = 3 * UN;          // main0, main1, cross
 constexpr uint32_t kBufCols = 256;             // TMEM columns between the two buffers
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kSmem = kABytes + kBStages * kBStage + 1024 + 256;
+constexpr size_t kSmem = kABytes + kBStages * kBStage + 2 * kWHalf + 1024 + 256;
 
 struct Smem {
   uint64_t a_full, a_empty;
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t w_full[2], w_written[2], w_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -65,11 +74,30 @@ __device__ __forceinline__ bool aborted(Smem* sm) {
   return *reinterpret_cast<volatile int*>(&sm->abort) != 0;
 }
 
+// TMA tile store from shared memory (out-of-range parts are not written).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {   // sources of all committed stores read
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {    // all committed stores complete
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     update_tc_kernel(const __grid_constant__ CUtensorMap tmDh,
                      const __grid_constant__ CUtensorMap tmDl,
                      const __grid_constant__ CUtensorMap tmUh,
-                     const __grid_constant__ CUtensorMap tmUl, double* __restrict__ Wt,
+                     const __grid_constant__ CUtensorMap tmUl,
+                     const __grid_constant__ CUtensorMap tmW, double* __restrict__ Wt,
                      int64_t ldw, int d_out, int n, int e, int n_rb, int n_nt, int parts,
                      int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -77,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* A = base;                      // hi chunks 0..3, then lo chunks 0..3
   uint8_t* Bring = base + kABytes;
-  Smem* sm = reinterpret_cast<Smem*>(Bring + kBStages * kBStage);
+  uint8_t* Wbuf = Bring + kBStages * kBStage;   // two half-tile buffers
+  Smem* sm = reinterpret_cast<Smem*>(Wbuf + 2 * kWHalf);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = n_rb * parts;
 
@@ -91,6 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm->acc_full[a], 1);
       mbar_init(&sm->acc_empty[a], 128);
+      mbar_init(&sm->w_full[a], 1);
+      mbar_init(&sm->w_written[a], 128);
+      mbar_init(&sm->w_empty[a], 1);
     }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -108,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch(&tmDl);
     tma_prefetch(&tmUh);
     tma_prefetch(&tmUl);
-    int s = 0, it = 0, issued = 0;
+    tma_prefetch(&tmW);
+    int s = 0, it = 0, issued = 0, wt = 0;
     uint32_t ph = 0;
     bool ok = true;
     int a_armed = -1;   // last A load armed, to drain on abort
@@ -141,6 +174,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ph ^= 1;
           }
         }
+        if (!ok) break;
+        for (int h = 0; h < 2; ++h) {   // the W~ tile, as two 32-column halves
+          if (!mbar_wait(&sm->w_empty[h], (wt & 1) ^ 1)) {
+            give_up(sm, status);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm->w_full[h], kWHalf);
+          for (int q = 0; q < 2; ++q)
+            tma_load_2d(Wbuf + h * kWHalf + q * kWBox, &tmW, &sm->w_full[h],
+                        e + tn * UN + h * 32 + q * WBOX, rb * UM);
+        }
+        ++wt;
       }
     }
     if (aborted(sm)) {   // let issued copies land before the CTA exits
@@ -152,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_wait(&sm->b_full[s], ph);
       }
+      if (wt > 0)
+        for (int h = 0; h < 2; ++h) mbar_wait(&sm->w_full[h], (wt - 1) & 1);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -212,15 +260,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int r = q * 32 + lane;        // tile row = TMEM lane
+    const bool storer = threadIdx.x == 64;
     int lt = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < items && !__any_sync(0xffffffffu, aborted(sm));
          item += gridDim.x) {
       const int rb = item % n_rb, p = item / n_rb;
-      const int i = rb * UM + r;
-      double* wrow = Wt + (int64_t)i * ldw + e;
-      for (int tn = p; tn < n_nt; tn += parts, ++lt) {
+      for (int tn = p; ok && tn < n_nt; tn += parts, ++lt) {
         const int buf = lt & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&sm->acc_full[buf], (lt >> 1) & 1))) {
           give_up(sm, status);
@@ -229,34 +276,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + buf * kBufCols;
-#pragma unroll 1
-        for (int c = 0; c < UN / 32; ++c) {
+        for (int h = 0; h < 2; ++h) {
           float m0[32], m1[32], cr[32];
-          tmem_ld32(ta + c * 32, m0);
-          tmem_ld32(ta + UN + c * 32, m1);
-          tmem_ld32(ta + 2 * UN + c * 32, cr);
-          const int j0 = tn * UN + c * 32;
-          if (i < d_out) {
-            if (j0 + 32 <= n) {
-              double2* w = reinterpret_cast<double2*>(wrow + j0);
+          tmem_ld32(ta + h * 32, m0);
+          tmem_ld32(ta + UN + h * 32, m1);
+          tmem_ld32(ta + 2 * UN + h * 32, cr);
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm->w_full[h], lt & 1))) {
+            give_up(sm, status);
+            ok = false;
+            break;
+          }
+          // row r of the half: two 128-byte box rows, 16-byte chunk j stored at
+          // position j ^ (r % 8) (the 128-byte swizzle)
 #pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                double2 x = w[k];
-                x.x -= ((double)m0[2 * k] + (double)m1[2 * k]) + (double)cr[2 * k];
-                x.y -= ((double)m0[2 * k + 1] + (double)m1[2 * k + 1]) + (double)cr[2 * k + 1];
-                w[k] = x;
-              }
-            } else {
+          for (int qb = 0; qb < 2; ++qb) {
+            uint8_t* rowp = Wbuf + h * kWHalf + qb * kWBox + r * 128;
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (j0 + k < n) wrow[j0 + k] -= ((double)m0[k] + (double)m1[k]) + (double)cr[k];
+            for (int j = 0; j < 8; ++j) {
+              double2* w = reinterpret_cast<double2*>(rowp + ((j ^ (r & 7)) << 4));
+              const int c = qb * WBOX + 2 * j;
+              double2 x = *w;
+              x.x -= ((double)m0[c] + (double)m1[c]) + (double)cr[c];
+              x.y -= ((double)m0[c + 1] + (double)m1[c + 1]) + (double)cr[c + 1];
+              *w = x;
             }
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(&sm->w_written[h]);
+          if (storer) {
+            // all 128 rows written -> store the half back, free the buffer once
+            // the store has read it
+            if (!mbar_wait(&sm->w_written[h], lt & 1)) {
+              give_up(sm, status);
+            } else {
+              for (int qb = 0; qb < 2; ++qb)
+                tma_store_2d(&tmW, Wbuf + h * kWHalf + qb * kWBox,
+                             e + tn * UN + h * 32 + qb * WBOX, rb * UM);
+              bulk_commit();
+              bulk_wait_read();
+            }
+            mbar_arrive(&sm->w_empty[h]);
           }
         }
         tc_fence_before();
         mbar_arrive(&sm->acc_empty[buf]);
       }
     }
+    if (storer) bulk_wait_all();   // the last stores complete before the CTA exits
   }
   __syncthreads();
   if (warp == 1) {
@@ -268,7 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
-                      const float* Ul, int64_t d_out, int64_t d_in) {
+                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in) {
+  const uint64_t dw[2] = {(uint64_t)d_in, (uint64_t)d_out};
+  const uint64_t sw[1] = {(uint64_t)d_in * 8};
+  const uint32_t bw[2] = {(uint32_t)WBOX, (uint32_t)UM};
   const uint64_t da[2] = {(uint64_t)UK, (uint64_t)d_out};
   const uint64_t sa[1] = {(uint64_t)UK * 4};
   const uint32_t ba[2] = {(uint32_t)KC, (uint32_t)UM};
@@ -282,6 +351,8 @@ bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const flo
          encode_tmap_2d(&m->Uh, Uh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, db, sb, bb,
                         CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode_tmap_2d(&m->Ul, Ul, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, db, sb, bb,
+                        CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode_tmap_2d(&m->W, Wt, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, dw, sw, bw,
                         CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -299,7 +370,7 @@ nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int6
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(update_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   update_tc_kernel<<<items < sms ? items : sms, kThreads, kSmem, st>>>(
-      m.Dh, m.Dl, m.Uh, m.Ul, Wt, ldw, (int)d_out, n, (int)e, n_rb, n_nt, parts, status);
+      m.Dh, m.Dl, m.Uh, m.Ul, m.W, Wt, ldw, (int)d_out, n, (int)e, n_rb, n_nt, parts, status);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;
