@@ -44,6 +44,18 @@ scale.  The readings taken where it is silent are marked READING below:
               factor GPTQ updates with; no column reordering.
   READING R9  H = X^T X with no 1/N or factor 2 (codes are invariant to a
               scale of H because lambda scales with it).
+  READING R10 the rules Schur Replay is set against (Abstract, sentence on
+              why scale choice is hard: a block evaluated on its own can
+              misestimate its final error) are taken as two independent-block
+              rules run inside the same GPTQ sweep, same amax (R5) and same
+              window (R4), so that only the scale decision differs:
+                amax       k = k0, the scale that maps the block amax to 6;
+                block_mse  k = argmin over the window of sum_j (v_j - q_j)^2
+                           with every q_j = s * E2M1(v_j / s) taken on the
+                           block's values before any in-block update, no
+                           curvature weight; ties to the lower code.
+              The block's codes always come from the GPTQ sweep at the chosen
+              scale, as for Schur Replay.
 """
 from __future__ import annotations
 
@@ -61,6 +73,13 @@ BLOCK = 16            # weights per block scale
 N_CAND = 16           # candidate block scales (READING R4)
 CAND_LO = -8          # first candidate offset from k0 (READING R4)
 DAMP = 0.01           # READING R7
+
+# Block-scale rules (READING R6 for Schur Replay, R10 for the other two).
+RULE_SCHUR_REPLAY = 0
+RULE_AMAX = 1
+RULE_BLOCK_MSE = 2
+RULE_NAMES = {"schur_replay": RULE_SCHUR_REPLAY, "amax": RULE_AMAX,
+              "block_mse": RULE_BLOCK_MSE}
 
 
 def e4m3_value(code):
@@ -217,10 +236,32 @@ def replay_block(v, Ublk, s):
     return codes, q, delta, score
 
 
+def independent_block_error(v, s):
+    """Squared error of rounding each of a block's values on its own at scale
+    s, with no GPTQ update between the columns and no curvature weight
+    (READING R10).  v (..., 16), s (...) -> (...)."""
+    v = np.asarray(v, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)[..., None]
+    q = e2m1_value(e2m1_round(v / s)) * s
+    return np.sum((v - q) ** 2, axis=-1)
+
+
+def e4m3_rounding_margin(t):
+    """Relative distance of t >= 0 to the nearest E4M3 rounding boundary (the
+    midpoint of two adjacent codes): how far the amax rule's k0 is from
+    flipping.  Infinite for t == 0."""
+    t = np.asarray(t, dtype=np.float64)
+    mids = (E4M3_TABLE[:-1] + E4M3_TABLE[1:]) / 2.0
+    d = np.min(np.abs(t[..., None] - mids), axis=-1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return np.where(t > 0, d / t, np.inf)
+
+
 def schur_replay_gptq(W, U, s_g, dead=None, n_cand=N_CAND, cand_lo=CAND_LO,
-                      return_diag=False):
+                      return_diag=False, rule=RULE_SCHUR_REPLAY):
     """GPTQ over the columns of W (d_out x d_in) with every 16-column block's
-    E4M3 scale chosen by Schur Replay.
+    E4M3 scale chosen by Schur Replay (rule = RULE_SCHUR_REPLAY), or by one of
+    the independent-block rules of READING R10 (RULE_AMAX, RULE_BLOCK_MSE).
 
     Rows are independent given U.  For block b (columns c0..c0+15):
       a  = max |W~[r, block]| on the updated weights        (READING R5)
@@ -233,7 +274,13 @@ def schur_replay_gptq(W, U, s_g, dead=None, n_cand=N_CAND, cand_lo=CAND_LO,
     Returns dict: codes (d_out, d_in) int64 nibbles, scales (d_out, d_in/16)
     int64 E4M3 codes, q (fp64 dequantized values), delta (d_out, d_in),
     err_sum = sum delta^2, and with return_diag: cand (d_out, nb, n_cand),
-    scores (d_out, nb, n_cand), wblock (updated W~ block inputs)."""
+    scores (d_out, nb, n_cand) Schur Replay scores of every candidate (under
+    any rule), wblock (updated W~ block inputs), margin (d_out, nb): how
+    close the rule's decision is to flipping -- the relative gap of its two
+    best scores, or for the amax rule e4m3_rounding_margin(a / (6 s_g))."""
+    rule = RULE_NAMES.get(rule, rule)
+    if rule not in (RULE_SCHUR_REPLAY, RULE_AMAX, RULE_BLOCK_MSE):
+        raise ValueError(f"unknown scale rule {rule!r}")
     W = np.array(W, dtype=np.float64, copy=True)
     d_out, d_in = W.shape
     if d_in % BLOCK:
@@ -250,6 +297,7 @@ def schur_replay_gptq(W, U, s_g, dead=None, n_cand=N_CAND, cand_lo=CAND_LO,
         cand_all = np.zeros((d_out, nb, n_cand), dtype=np.int64)
         scores_all = np.zeros((d_out, nb, n_cand))
         win_all = np.zeros((d_out, nb, BLOCK))
+        margin_all = np.full((d_out, nb), np.inf)
     for b in range(nb):
         c0, c1 = b * BLOCK, (b + 1) * BLOCK
         v = W[:, c0:c1]
@@ -260,7 +308,15 @@ def schur_replay_gptq(W, U, s_g, dead=None, n_cand=N_CAND, cand_lo=CAND_LO,
         cand = candidate_codes(k0, n_cand, cand_lo)           # (d_out, n_cand)
         s = e4m3_value(cand) * s_g                            # exact in fp64
         c_codes, c_q, c_delta, c_score = replay_block(v[:, None, :], Ublk, s)
-        best = np.argmin(c_score, axis=1)                     # first = lowest code
+        if rule == RULE_AMAX:
+            best = k0 - cand[:, 0]                            # k0 is in the window
+            margin = e4m3_rounding_margin(amax / (E2M1_MAX * s_g))
+        else:
+            sel = c_score if rule == RULE_SCHUR_REPLAY else \
+                independent_block_error(v[:, None, :], s)
+            best = np.argmin(sel, axis=1)                     # first = lowest code
+            srt = np.sort(sel, axis=1)
+            margin = (srt[:, 1] - srt[:, 0]) / np.maximum(srt[:, 0], 1e-300)
         rows = np.arange(d_out)
         blk_codes = c_codes[rows, best]
         blk_q = c_q[rows, best]
@@ -278,13 +334,14 @@ def schur_replay_gptq(W, U, s_g, dead=None, n_cand=N_CAND, cand_lo=CAND_LO,
             cand_all[:, b] = cand
             scores_all[:, b] = np.where(live[:, None], c_score, 0.0)
             win_all[:, b] = v
+            margin_all[:, b] = np.where(live, margin, np.inf)
         if c1 < d_in:
             W[:, c1:] -= blk_delta @ U[c0:c1, c1:]
     out = dict(codes=codes, scales=scales, q=q, delta=delta,
                err_sum=float(np.sum(delta * delta)),
                row_err=np.sum(delta * delta, axis=1))
     if return_diag:
-        out.update(cand=cand_all, scores=scores_all, wblock=win_all)
+        out.update(cand=cand_all, scores=scores_all, wblock=win_all, margin=margin_all)
     return out
 
 
@@ -324,7 +381,7 @@ def layer_error(W, Q, H):
 
 
 def solve_layer(W, X=None, H=None, damp_frac=DAMP, n_cand=N_CAND,
-                cand_lo=CAND_LO, return_diag=False):
+                cand_lo=CAND_LO, return_diag=False, rule=RULE_SCHUR_REPLAY):
     """The whole per-layer solve: Hessian, damping, factor, global scale,
     Schur Replay GPTQ, dequant and layer error."""
     if H is None:
@@ -335,7 +392,7 @@ def solve_layer(W, X=None, H=None, damp_frac=DAMP, n_cand=N_CAND,
     Wz = W.copy()
     Wz[:, dead] = 0.0
     s_g = global_scale(Wz)
-    res = schur_replay_gptq(Wz, U, s_g, dead, n_cand, cand_lo, return_diag)
+    res = schur_replay_gptq(Wz, U, s_g, dead, n_cand, cand_lo, return_diag, rule)
     Q = dequant(res["codes"], res["scales"], s_g)
     res.update(H=H, H_d=H_d, U=U, dead=dead, lam=lam, s_g=s_g, Q=Q,
                W=Wz, layer_error=layer_error(Wz, res["q"], H))

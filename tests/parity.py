@@ -4,7 +4,9 @@ The acceptance rule for the discrete outputs (E2M1 codes, E4M3 scales):
   * small layers: bit-exact;
   * larger layers: at least 99.9% of the 16-weight blocks identical, and in
     every row the FIRST block that differs must sit at a near-tie of the
-    oracle -- its top-two candidate scores within 1e-5 relative, or one of its
+    oracle -- its scale decision within 1e-5 relative of flipping (the top two
+    candidate scores of a search rule; for the amax rule the block amax / 6 s_g
+    against the nearest E4M3 rounding midpoint), or one of its
     codes within 1e-5 (relative to the grid step) of an E2M1 rounding
     midpoint.  Once a row has taken a different discrete decision its later
     blocks start from different weights (GPTQ carries every column's error
@@ -82,7 +84,8 @@ def classify(ref: dict, U: np.ndarray, s_g: float, codes_gpu: np.ndarray,
     sg = float(np.float32(s_g))
     for r in np.nonzero(mism.any(axis=1))[0]:
         b = int(np.argmax(mism[r]))
-        margin = float(top2_margin(ref["scores"][r, b]))
+        margin = float(ref["margin"][r, b]) if "margin" in ref else \
+            float(top2_margin(ref["scores"][r, b]))
         if margin < NEAR_TIE:
             continue
         Ublk = U[16 * b:16 * b + 16, 16 * b:16 * b + 16]
