@@ -61,8 +61,31 @@ typedef enum { NVFP4_BF16 = 0, NVFP4_F32 = 1 } nvfp4_dtype;
 /* Opaque stream handle, layout-compatible with cudaStream_t / CUstream. */
 typedef struct CUstream_st* nvfp4_stream_t;
 
-/* Solve parameters.  Only the defaults below are supported by this build
- * (n_candidates = 16, cand_lo = -8, lazy_batch = 128); other values return
+/* Block-scale rule of the GPTQ sweep.
+ *
+ * NVFP4_RULE_SCHUR_REPLAY (default): every candidate scale of a block is
+ *   scored by replaying the in-block GPTQ updates it causes and summing
+ *   delta_j^2 = (v_j - q_j)^2 / U_jj^2, the block error left after
+ *   compensation by the still-unquantized columns; the lowest score wins
+ *   ("Replay the Curvature", Abstract, sentence introducing Schur Replay).
+ * The two rules below evaluate a block on its own, which can misestimate its
+ * final error once GPTQ updates the columns after each quantized one (the
+ * Abstract's sentence on why scale choice is hard in GPTQ); they exist for
+ * comparison (same sweep, same block amax and window, only the decision
+ * differs):
+ * NVFP4_RULE_AMAX: the centre code k0, which maps the block amax to 6.
+ * NVFP4_RULE_BLOCK_MSE: the window code minimising sum_j (v_j - q_j)^2 with
+ *   every v_j rounded on its own, before any in-block update; ties to the
+ *   lower code. */
+typedef enum {
+  NVFP4_RULE_SCHUR_REPLAY = 0,
+  NVFP4_RULE_AMAX = 1,
+  NVFP4_RULE_BLOCK_MSE = 2
+} nvfp4_scale_rule;
+
+/* Solve parameters.  n_candidates, cand_lo and lazy_batch support only the
+ * defaults below (n_candidates = 16, cand_lo = -8, lazy_batch = 128); other
+ * values, or a scale_rule outside nvfp4_scale_rule, return
  * NVFP4_ERR_UNSUPPORTED.  The candidate window is the n_candidates
  * consecutive E4M3 codes starting at k0 + cand_lo, shifted into 1..126,
  * where k0 = e4m3_rn(amax_block / (6 s_g)) (at least 1). */
@@ -70,7 +93,7 @@ typedef struct {
   int n_candidates; /* 16 */
   int cand_lo;      /* -8 */
   int lazy_batch;   /* 128: columns per batch of the trailing update */
-  int reserved;     /* 0 */
+  int scale_rule;   /* nvfp4_scale_rule, default NVFP4_RULE_SCHUR_REPLAY */
 } nvfp4_solve_params;
 
 /* Fills *p with the defaults above. */

@@ -31,7 +31,7 @@ class Nvfp4Error(RuntimeError):
 
 class SolveParams(ctypes.Structure):
     _fields_ = [("n_candidates", ctypes.c_int), ("cand_lo", ctypes.c_int),
-                ("lazy_batch", ctypes.c_int), ("reserved", ctypes.c_int)]
+                ("lazy_batch", ctypes.c_int), ("scale_rule", ctypes.c_int)]
 
 
 _lib = None
@@ -115,6 +115,18 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 def default_params() -> SolveParams:
     p = SolveParams()
     lib().nvfp4_default_params(ctypes.byref(p))
+    return p
+
+
+# nvfp4_scale_rule values
+SCALE_RULES = {"schur_replay": 0, "amax": 1, "block_mse": 2}
+
+
+def solve_params(scale_rule="schur_replay") -> SolveParams:
+    """The default parameters with the given block-scale rule (a name of
+    SCALE_RULES or its integer value)."""
+    p = default_params()
+    p.scale_rule = SCALE_RULES.get(scale_rule, scale_rule)
     return p
 
 

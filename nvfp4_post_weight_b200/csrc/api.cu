@@ -15,7 +15,7 @@ namespace {
 bool params_ok(const nvfp4_solve_params* p) {
   if (!p) return true;
   return p->n_candidates == kCand && p->cand_lo == -8 && p->lazy_batch == kLazyBatch &&
-         p->reserved == 0;
+         p->scale_rule >= NVFP4_RULE_SCHUR_REPLAY && p->scale_rule <= NVFP4_RULE_BLOCK_MSE;
 }
 
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
@@ -35,7 +35,7 @@ void nvfp4_default_params(nvfp4_solve_params* p) {
   p->n_candidates = kCand;
   p->cand_lo = -8;
   p->lazy_batch = kLazyBatch;
-  p->reserved = 0;
+  p->scale_rule = NVFP4_RULE_SCHUR_REPLAY;
 }
 
 const char* nvfp4_status_string(nvfp4_status s) {
@@ -114,7 +114,8 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
   if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
   if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(d_out, d_in))
     return NVFP4_ERR_WORKSPACE;
-  return launch_quantize(W, w_dtype, d_out, d_in, U, dead, codes, scales, global_scale,
+  const int rule = params ? params->scale_rule : NVFP4_RULE_SCHUR_REPLAY;
+  return launch_quantize(W, w_dtype, d_out, d_in, U, dead, rule, codes, scales, global_scale,
                          err_out, ws, as_cuda(stream));
 }
 

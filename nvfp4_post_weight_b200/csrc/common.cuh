@@ -122,7 +122,7 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,
                             uint8_t* dead, float* lambda_out, void* ws, cudaStream_t st);
 size_t prepare_ws_bytes(int64_t d);
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
-                             const float* U, const uint8_t* dead, uint8_t* codes,
+                             const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
                              cudaStream_t st);
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in);

@@ -190,9 +190,17 @@ __device__ __forceinline__ double replay(double (&v)[16], double s, double inv_s
   return score;
 }
 
+// Block-scale rules: Schur Replay, and the two independent-block rules it is
+// compared with ("Replay the Curvature", Abstract: a block evaluated on its own
+// misestimates its final error): the amax scale k0, and the window code whose
+// one-by-one rounding error of the block's values is smallest.  All three run
+// the same GPTQ sweep; only the scale decision differs.
+constexpr int kRuleSchurReplay = 0, kRuleAmax = 1, kRuleBlockMse = 2;
+
 // One lazy batch of Schur Replay.  Half-warp = one row; lane hl = candidate hl
 // of the current block.  The batch's upper block-triangular part of U lives in
 // shared memory as 16x16 fp64 tiles, the rows' batch values next to it.
+template <int kRule>
 __global__ void __launch_bounds__(kReplayThreads)
     schur_replay_batch_kernel(double* __restrict__ Wt, const float* __restrict__ U,
                               int64_t d_out, int64_t d_in, int c0, int bw,
@@ -256,22 +264,41 @@ __global__ void __launch_bounds__(kReplayThreads)
       const double* Ud = Ut + utile(b, b) * 256;
       const double* idb = invd + 16 * b;
 
+      // the rule's selection score: the replay score itself, or for the
+      // independent block-MSE rule the squared error of rounding the block's
+      // values one by one (no in-block update, no curvature weight)
+      double sel = 0.0;
+      if constexpr (kRule == kRuleBlockMse) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const double x = __dmul_rn(v[j], inv_s);
+          const double r = e2m1_round_mag(fabs(x));
+          const double res = __fma_rn(x < 0.0 ? r : -r, s, v[j]);
+          sel = __fma_rn(res, res, sel);
+        }
+      }
       double dl[16];
       uint64_t pk;
       const double score = replay(v, s, inv_s, Ud, idb, dl, pk);
+      if constexpr (kRule == kRuleSchurReplay) sel = score;
 
-      // argmin over the 16 candidates, ties to the lower code
-      double best = score;
-      int bl = hl;
+      // the chosen candidate: k0 for the amax rule, else the argmin of the
+      // selection score over the 16 candidates, ties to the lower code
+      int bl = k0 - lo;
+      if constexpr (kRule != kRuleAmax) {
+        double bs = sel;
+        bl = hl;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) {
-        const double os = __shfl_xor_sync(FULL, best, o, 16);
-        const int ol = __shfl_xor_sync(FULL, bl, o, 16);
-        if (os < best || (os == best && ol < bl)) {
-          best = os;
-          bl = ol;
+        for (int o = 8; o > 0; o >>= 1) {
+          const double os = __shfl_xor_sync(FULL, bs, o, 16);
+          const int ol = __shfl_xor_sync(FULL, bl, o, 16);
+          if (os < bs || (os == bs && ol < bl)) {
+            bs = os;
+            bl = ol;
+          }
         }
       }
+      const double best = __shfl_sync(FULL, score, bl, 16);   // the winner's sum delta^2
       const bool live = amax > 0.0;
       __syncwarp();
       if (hl == bl) {
@@ -346,7 +373,7 @@ size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
 }
 
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
-                             const float* U, const uint8_t* dead, uint8_t* codes,
+                             const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
                              cudaStream_t st) {
   QuantLayout L = quant_layout(ws, d_out, d_in);
@@ -370,8 +397,10 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
   NVFP4_LAUNCH_CHECK();
   count_launches(2);
 
-  NVFP4_CUDA_TRY(cudaFuncSetAttribute(schur_replay_batch_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto* replay_kernel = rule == kRuleAmax       ? schur_replay_batch_kernel<kRuleAmax>
+                       : rule == kRuleBlockMse ? schur_replay_batch_kernel<kRuleBlockMse>
+                                               : schur_replay_batch_kernel<kRuleSchurReplay>;
+  NVFP4_CUDA_TRY(cudaFuncSetAttribute(replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kReplaySmem));
   UpdateMaps maps;
   if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in))
@@ -382,7 +411,7 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
     const int bw = (int)((d_in - c0) < kLazyBatch ? (d_in - c0) : kLazyBatch);
     {
       ProfileScope ps(kPhaseReplay, st);
-      schur_replay_batch_kernel<<<rgrid, kReplayThreads, kReplaySmem, st>>>(
+      replay_kernel<<<rgrid, kReplayThreads, kReplaySmem, st>>>(
           L.Wt, U, d_out, d_in, (int)c0, bw, sg, codes, scales, L.Dh, L.Dl, L.rowerr);
       NVFP4_LAUNCH_CHECK();
       count_launches(1);

@@ -12,11 +12,14 @@ from . import binding as B
 
 class LayerSolver:
     """Hessian -> prepare -> Schur Replay quantize -> dequant -> layer error for
-    one (d_out, d_in) layer on one CUDA device."""
+    one (d_out, d_in) layer on one CUDA device.  scale_rule picks the block-scale
+    rule (binding.SCALE_RULES; Schur Replay by default, the independent-block
+    rules for comparison)."""
 
     def __init__(self, d_out: int, d_in: int, device="cuda", damp: float = 0.01,
-                 out_dtype=torch.bfloat16):
+                 out_dtype=torch.bfloat16, scale_rule="schur_replay"):
         self.d_out, self.d_in, self.damp = int(d_out), int(d_in), float(damp)
+        self.params = B.solve_params(scale_rule)
         dev = torch.device(device)
         self.device = dev
         d = self.d_in
@@ -42,7 +45,8 @@ class LayerSolver:
 
     def quantize(self, W, stream=None):
         B.nvfp4_gptq_schur_replay_quantize(W, self.U, self.codes, self.scales, self.s_g,
-                                           self.err, self.dead, self.ws_quant, None, stream)
+                                           self.err, self.dead, self.ws_quant, self.params,
+                                           stream)
 
     def dequant(self, stream=None):
         B.nvfp4_dequant(self.codes, self.scales, self.s_g, self.Q, stream)

@@ -54,6 +54,13 @@ def test_host_side_checks_need_no_device():
     # a workspace that is too small -> NVFP4_ERR_WORKSPACE
     assert L.nvfp4_gptq_prepare(ctypes.c_void_p(256), 32, 0.01, ctypes.c_void_p(256), null,
                                 null, ctypes.c_void_p(256), 16, null) == 3
+    # an unknown block-scale rule -> NVFP4_ERR_UNSUPPORTED
+    bad = B.solve_params(3)
+    assert L.nvfp4_gptq_schur_replay_quantize(
+        ctypes.c_void_p(256), 0, 4, 32, ctypes.c_void_p(256), ctypes.byref(bad), null,
+        ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), null,
+        ctypes.c_void_p(256), 1 << 20, null) == 8
+    assert B.solve_params("block_mse").scale_rule == 2 and B.default_params().scale_rule == 0
     # the allocation-free quantize refuses layers beyond its fixed scratch
     assert L.nvfp4_gptq_schur_replay_quantize_noalloc(
         ctypes.c_void_p(256), 0, 4096, 4096, ctypes.c_void_p(256), null, null,
