@@ -236,6 +236,17 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return None
+    # untimed: the same layer's error tr((W-Q) H (W-Q)^T) under the
+    # independent-block scale rules Schur Replay is compared with
+    by_rule = {"schur_replay": solver.layer_err.item()}
+    sr_params = solver.params
+    for rule in ("amax", "block_mse"):
+        solver.params = B.solve_params(rule)
+        solver.quantize(Wd)
+        solver.layer_error(Wd)
+        by_rule[rule] = solver.layer_err.item()
+    solver.params = sr_params
+    torch.cuda.synchronize()
     peaks = load_peaks()
     wk = phase_work(d_out, d_in, n_tok)
     names = ["hessian", "prepare", "replay", "update", "dequant", "other"]
@@ -289,6 +300,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": W.numel() * W.element_size() + X.numel() * X.element_size(),
                 "d2h_bytes_per_step": codes_h.numel() + scales_h.numel() + 4},
         "gpu_launches": launches,
+        "layer_error_by_scale_rule": by_rule,
         "clocks": clk.summary(),
     }
     return out

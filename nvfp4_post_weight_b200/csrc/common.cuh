@@ -135,4 +135,13 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
                                 cudaStream_t st);
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in);
 
+// D (8x8) += A (8x4) B (4x8) in fp64 on the tensor cores (warp-wide
+// mma.sync m8n8k4; tcgen05 has no fp64 kind).  Fragments per lane:
+// a = A[lane/4][lane%4], b = B[lane%4][lane/4], d = D[lane/4][2*(lane%4)+{0,1}].
+__device__ __forceinline__ void dmma_m8n8k4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
 }  // namespace nvfp4

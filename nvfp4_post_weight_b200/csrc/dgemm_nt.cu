@@ -22,15 +22,6 @@ namespace {
 constexpr int DK = 16;
 constexpr int kDThreads = 256;   // 8 warps: 2 along M x 4 along N
 
-// D (8x8) += A (8x4, row) * B (4x8, col) in fp64 on the tensor cores.
-// Fragments: a = A[lane/4][lane%4], b = B[lane%4][lane/4],
-// d = D[lane/4][2*(lane%4) + {0,1}].
-__device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(d0), "+d"(d1)
-               : "d"(a), "d"(b));
-}
-
 // CTA tile (16 T) x (32 T) ... see below; T = 4: 64 x 64 (each warp 32 x 16),
 // T = 8: 128 x 128 (each warp 64 x 32).  ktri: 0 dense P; 1 P upper triangular
 // (P[m][k] = 0 for k < m), so a tile's K range starts at its first row; 2 P
@@ -107,7 +98,7 @@ __global__ void __launch_bounds__(kDThreads)
 #pragma unroll
       for (int i = 0; i < MT; ++i)
 #pragma unroll
-        for (int j = 0; j < NT; ++j) dmma(acc[i][j][0], acc[i][j][1], af[i], bf[j]);
+        for (int j = 0; j < NT; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], af[i], bf[j]);
     }
     if (kt + 1 < nk) stash(cur ^ 1);
     __syncthreads();

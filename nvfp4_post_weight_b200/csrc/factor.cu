@@ -82,88 +82,173 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
 // diagonal block A11 = L11 L11^T and inverts L11 in fp64 (redundantly: no CTA
 // waits for another); CTA 0 then writes X11 = L11^-1 and Y11 = X11^T into the
 // diagonal blocks of X and Y (A11 stays as it is: the other CTAs of the launch
-// may still be reading it), every other CTA solves its own 64-row slice of the
+// may still be reading it), every other CTA solves its own 32-row slice of the
 // panel below, L21 = A21 X11^T, in place.
 //
-// The 64 x 64 block is itself blocked by 16 (a per-column CTA barrier costs
-// far more than the arithmetic of a column):
+// The 64 x 64 block is blocked by 16 (a per-column CTA barrier costs far more
+// than the arithmetic of a column):
 //   for each 16-column sub-panel K:
-//     one warp factors and inverts the 16 x 16 diagonal block in registers,
-//       exchanging values by shuffles (lane i holds row i);
-//     all threads solve the rows below it, L[r][K] = S[r][K] inv(L_KK)^T,
-//     and update the trailing lower part, S -= L[:,K] L[:,K]^T;
-//   the inverse of L is assembled from the four 16 x 16 inverses by two
-//   doubling steps, X21 = -X22 (L21 X11), as small products.
+//     one warp factors the 16 x 16 diagonal block in registers, exchanging
+//       values by shuffles (lane i holds row i) -- the only serial chain;
+//     one thread per row below solves L[r][K] L_KK^T = S[r][K] by forward
+//       substitution;
+//     the warps update the trailing lower part, S -= L[:,K] L[:,K]^T, as
+//       8 x 8 fp64 tensor-core tiles (mma.sync m8n8k4);
+//   four warps then invert the four 16 x 16 diagonal blocks at once, and two
+//   doubling steps, X21 = -X22 (L21 X11), assemble the inverse of L11; the
+//   doubling products and the slice solve are tensor-core tiles too.
 constexpr int kPanelThreads = 256;
-constexpr int kPitch = NB + 1;
+constexpr int kPitch = NB + 4;   // 68: an 8 x 4 fragment (two half-warps) is conflict-free
 constexpr int kSub = 16;
+constexpr int kSlice = 32;       // rows of the panel below the diagonal block per CTA
 
-// 1/p for p > 0: the hardware's approximate fp64 reciprocal refined by two
-// Newton-Raphson steps (x <- x + x (1 - p x)), which square the relative
-// error each time.
-__device__ __forceinline__ double recip_nr(double p) {
+// 1/p for p > 0: the hardware's approximate fp64 reciprocal refined by one
+// Newton-Raphson step (x <- x + x (1 - p x)), which squares its relative
+// error (2^-23 -> 2^-46: far below what the fp32 factor U keeps).
+__device__ __forceinline__ double recip_nr1(double p) {
   double x;
   asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(x) : "d"(p));
-  x = fma(x, fma(-p, x, 1.0), x);
-  x = fma(x, fma(-p, x, 1.0), x);
-  return x;
+  return fma(x, fma(-p, x, 1.0), x);
 }
 
-constexpr size_t kPanelSmem = sizeof(double) * (4 * NB * kPitch);
+// sqrt(p) and 1/sqrt(p) for p > 0 by Newton-Raphson on the reciprocal square
+// root, y <- y + y (1/2 - (p/2) y^2), from the hardware approximation (two
+// steps), then one Newton correction of the square root s = p y,
+// s <- s + (y/2) (p - s^2).
+__device__ __forceinline__ void sqrt_rsqrt(double p, double& sq, double& isq) {
+  double y;
+  asm("rsqrt.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(p));
+  const double h = 0.5 * p;
+  y = fma(y, fma(-h * y, y, 0.5), y);
+  y = fma(y, fma(-h * y, y, 0.5), y);
+  const double s0 = p * y;
+  sq = fma(0.5 * y, fma(-s0, s0, p), s0);
+  isq = y;
+}
+
+constexpr size_t kPanelSmem = sizeof(double) * ((3 * NB + kSlice) * kPitch + NB);
 
 // One warp, lanes 0..15 meaningful: factor the 16 x 16 block at (o, o) of S
-// (lower part), write L_KK back into S and inv(L_KK) into the same block of
-// Xd (lower, zeros above).  A non-positive pivot is flagged and taken as 1.
-__device__ __forceinline__ void factor_invert_16(double (*S)[kPitch], double (*Xd)[kPitch],
-                                                 int o, PrepHeader* hdr) {
+// (lower part) and write L_KK back into S (zeros above) and 1/L_jj into invd.
+// A non-positive pivot is flagged and taken as 1.
+__device__ __forceinline__ void factor_16(double (*S)[kPitch], double* invd, int o,
+                                          PrepHeader* hdr) {
   const int lane = threadIdx.x & 31;
   const int i = lane & 15;
   const unsigned full = 0xffffffffu;
   double r[kSub];   // row i of the block
 #pragma unroll
   for (int l = 0; l < kSub; ++l) r[l] = (l <= i) ? S[o + i][o + l] : 0.0;
-  double sq[kSub];  // sqrt(pivot_j), the same in every lane
+  double pv[kSub];  // the pivots, the same in every lane
+  bool bad = false;
 #pragma unroll
   for (int j = 0; j < kSub; ++j) {
+    // branch-free: a (never taken) branch per pivot costs more than the pivot
     double p = __shfl_sync(full, r[j], j, 16);
-    const bool ok = p > 0.0;
-    if (!ok) {
-      if (lane == 0) flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
-      p = 1.0;
-    }
-    sq[j] = p;   // square root taken below, off the per-column chain
-    const double a = (i > j) ? r[j] * recip_nr(p) : 0.0;
+    bad |= !(p > 0.0);
+    p = p > 0.0 ? p : 1.0;
+    pv[j] = p;
+    const double a = (i > j) ? r[j] * recip_nr1(p) : 0.0;
 #pragma unroll
     for (int l = j + 1; l < kSub; ++l) {
       const double cl = __shfl_sync(full, r[j], l, 16);   // S[l][j]
       r[l] = fma(-a, cl, r[l]);
     }
   }
+  if (bad && lane == 0) flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
   // L[i][l] = r[l] / sqrt(p_l) (l < i), L[i][i] = sqrt(p_i)
-  double isq[kSub];
+  double sq[kSub], isq[kSub];
+#pragma unroll
+  for (int l = 0; l < kSub; ++l) sqrt_rsqrt(pv[l], sq[l], isq[l]);
+  if (lane < kSub) {
+    double isq_i = 0.0;   // isq[i] without a dynamic register index
+#pragma unroll
+    for (int l = 0; l < kSub; ++l) {
+      S[o + i][o + l] = l < i ? r[l] * isq[l] : (l == i ? sq[l] : 0.0);
+      isq_i = l == i ? isq[l] : isq_i;
+    }
+    invd[o + i] = isq_i;
+  }
+}
+
+// One warp, lanes 0..15 meaningful: column i of inv(L_KK) for the factored
+// block at (o, o) of S, by right-looking forward substitution (each x[m]
+// updates the later sums at once, so the serial chain is one fma per m),
+// written into the same block of Xd (lower, zeros above).
+__device__ __forceinline__ void invert_16(double (*S)[kPitch], double (*Xd)[kPitch],
+                                          const double* invd, int o) {
+  const int lane = threadIdx.x & 31;
+  const int i = lane & 15;
+  const unsigned full = 0xffffffffu;
+  double r[kSub], x[kSub], acc[kSub];
 #pragma unroll
   for (int l = 0; l < kSub; ++l) {
-    sq[l] = sqrt(sq[l]);
-    isq[l] = recip_nr(sq[l]);
+    r[l] = (l <= i) ? S[o + i][o + l] : 0.0;
+    acc[l] = 0.0;
   }
 #pragma unroll
-  for (int l = 0; l < kSub; ++l) r[l] = l < i ? r[l] * isq[l] : (l == i ? sq[i] : 0.0);
-  // column c = i of inv(L): x[m] = -(sum_{l<m} L[m][l] x[l]) / L[m][m] for m > c
-  double x[kSub];
-#pragma unroll
   for (int m = 0; m < kSub; ++m) {
-    double acc = 0.0;
+    const double id = invd[o + m];
+    x[m] = m < i ? 0.0 : (m == i ? id : -acc[m] * id);
 #pragma unroll
-    for (int l = 0; l < m; ++l) acc = fma(__shfl_sync(full, r[l], m, 16), x[l], acc);
-    x[m] = m < i ? 0.0 : (m == i ? isq[m] : -acc * isq[m]);
+    for (int n = m + 1; n < kSub; ++n)
+      acc[n] = fma(__shfl_sync(full, r[m], n, 16), x[m], acc[n]);   // L[n][m] x[m]
   }
   if (lane < kSub) {
 #pragma unroll
-    for (int l = 0; l < kSub; ++l) {
-      S[o + i][o + l] = l <= i ? r[l] : 0.0;
-      Xd[o + l][o + i] = x[l];   // column i of the inverse
-    }
+    for (int l = 0; l < kSub; ++l) Xd[o + l][o + i] = x[l];   // column i of the inverse
   }
+}
+
+// acc (8 x 8 tile, fragment layout of dmma_m8n8k4) += sgn * P[pm.., k] Q[qn.., k]^T
+// summed over k in [k0, k1) (steps of 4), P and Q row-major in shared memory.
+__device__ __forceinline__ void tile_pqt(double& d0, double& d1, double (*P)[kPitch], int pm,
+                                         double (*Q)[kPitch], int qn, int k0, int k1,
+                                         double sgn) {
+  const int lane = threadIdx.x & 31, fr = lane >> 2, fc = lane & 3;
+  for (int k = k0; k < k1; k += 4)
+    dmma_m8n8k4(d0, d1, sgn * P[pm + fr][k + fc], Q[qn + fr][k + fc]);
+}
+
+// acc += sgn * P[pm.., k] B[k, bn..] summed over k in [k0, k1), with B read
+// in place (row-major, N contiguous): no transposed copy needed.
+__device__ __forceinline__ void tile_pb(double& d0, double& d1, double (*P)[kPitch], int pm,
+                                        double (*Bm)[kPitch], int bn, int k0, int k1,
+                                        double sgn) {
+  const int lane = threadIdx.x & 31, fr = lane >> 2, fc = lane & 3;
+  for (int k = k0; k < k1; k += 4)
+    dmma_m8n8k4(d0, d1, sgn * P[pm + fr][k + fc], Bm[k + fc][bn + fr]);
+}
+
+// One level of the inverse doubling for every pair of adjacent b x b diagonal
+// blocks at offset q:  T = L21 X11,  X21 = -X22 T.  The triangular factors
+// are stored with zeros above their diagonals, so full-length sums are exact.
+// 8 x 8 output tiles spread over the 8 warps.
+template <int b>
+__device__ __forceinline__ void doubling_level(double (*S)[kPitch], double (*Xd)[kPitch],
+                                               double (*T)[kPitch]) {
+  constexpr int kPairs = NB / (2 * b);
+  constexpr int kTb = b / 8;                        // tiles per side of a block
+  constexpr int kTiles = kPairs * kTb * kTb;        // 8 (b = 16) or 16 (b = 32)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int fr = lane >> 2, fc2 = 2 * (lane & 3);
+  for (int t = warp; t < kTiles; t += kPanelThreads / 32) {
+    const int q = (t / (kTb * kTb)) * 2 * b, ti = (t / kTb) % kTb, tj = t % kTb;
+    double d0 = 0.0, d1 = 0.0;
+    tile_pb(d0, d1, S, q + b + 8 * ti, Xd, q + 8 * tj, q, q + b, 1.0);
+    T[q + b + 8 * ti + fr][q + 8 * tj + fc2] = d0;
+    T[q + b + 8 * ti + fr][q + 8 * tj + fc2 + 1] = d1;
+  }
+  __syncthreads();
+  for (int t = warp; t < kTiles; t += kPanelThreads / 32) {
+    const int q = (t / (kTb * kTb)) * 2 * b, ti = (t / kTb) % kTb, tj = t % kTb;
+    double d0 = 0.0, d1 = 0.0;
+    // P = X22 (rows and columns q+b ..), B = T (rows q+b .., columns q ..)
+    tile_pb(d0, d1, Xd, q + b + 8 * ti, T, q + 8 * tj, q + b, q + 2 * b, -1.0);
+    Xd[q + b + 8 * ti + fr][q + 8 * tj + fc2] = d0;
+    Xd[q + b + 8 * ti + fr][q + 8 * tj + fc2 + 1] = d1;
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kPanelThreads)
@@ -172,20 +257,27 @@ __global__ void __launch_bounds__(kPanelThreads)
   extern __shared__ double dsm[];
   double(*S)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm);             // A11 -> L11
   double(*Xd)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + NB * kPitch);   // X11
-  double(*R)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 2 * NB * kPitch);
-  double(*T)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 3 * NB * kPitch);  // scratch
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int64_t r0 = k + kb + (int64_t)(blockIdx.x - 1) * NB;   // slice rows (CTA >= 1)
+  double(*T)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 2 * NB * kPitch);  // scratch
+  double(*R)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + 3 * NB * kPitch);  // A21 slice
+  double* invd = dsm + (3 * NB + kSlice) * kPitch;                             // 1 / L_jj
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int fr = lane >> 2, fc2 = 2 * (lane & 3);
+  const int64_t r0 = k + kb + (int64_t)(blockIdx.x - 1) * kSlice;   // slice rows (CTA >= 1)
   const int64_t rem = d - r0;
-  const int rows = blockIdx.x == 0 ? 0 : (int)(rem < NB ? rem : NB);
+  const int rows = blockIdx.x == 0 ? 0 : (int)(rem < kSlice ? rem : kSlice);
 
   {   // all global loads of a thread are issued before any is used
-    constexpr int kPer = NB * NB / kPanelThreads;   // 16
-    double a11[kPer], a21[kPer];
+    constexpr int kPer = NB * NB / kPanelThreads;        // 16
+    constexpr int kPerS = kSlice * NB / kPanelThreads;   // 8
+    double a11[kPer], a21[kPerS];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
       a11[q] = (i < kb && l <= i) ? A[(k + i) * d + k + l] : 0.0;
+    }
+#pragma unroll
+    for (int q = 0; q < kPerS; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
       a21[q] = (i < rows && l < kb) ? A[(r0 + i) * d + k + l] : 0.0;
     }
 #pragma unroll
@@ -193,105 +285,98 @@ __global__ void __launch_bounds__(kPanelThreads)
       const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
       S[i][l] = (i < kb && l < kb) ? a11[q] : (i == l ? 1.0 : 0.0);
       Xd[i][l] = 0.0;
+    }
+#pragma unroll
+    for (int q = 0; q < kPerS; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx / NB, l = idx % NB;
       R[i][l] = a21[q];
     }
   }
   __syncthreads();
 
-  // ---- factor, 16 columns at a time
+  // ---- factor, 16 columns at a time (not unrolled: inlined copies of the
+  // warp factor overflow the instruction cache)
+#pragma unroll 1
   for (int K = 0; K < NB / kSub; ++K) {
     const int o = K * kSub;
-    if (warp == 0) factor_invert_16(S, Xd, o, hdr);
+    if (warp == 0) factor_16(S, invd, o, hdr);
     __syncthreads();
-    // rows below the sub-block: T[r][c] = sum_{l <= c} S[r][o+l] inv(L_KK)[c][l]
-    const int nb = NB - o - kSub;   // rows below (0, 16, 32 or 48)
-    for (int idx = tid; idx < nb * kSub; idx += blockDim.x) {
-      const int rr = o + kSub + idx / kSub, c = idx % kSub;
-      double acc = 0.0;
+    const int nb = NB - o - kSub;   // rows below the sub-block (48, 32, 16 or 0)
+    if (nb == 0) break;
+    // rows below: solve x L_KK^T = S[r][K] for the row's new L values, one
+    // thread per row, right-looking (one fma per step on the serial chain)
+    if (tid >= 32 && tid < 32 + nb) {
+      const int rr = o + kSub + tid - 32;
+      double x[kSub];
 #pragma unroll
-      for (int l = 0; l < kSub; ++l) acc = fma(S[rr][o + l], Xd[o + c][o + l], acc);
-      T[rr][c] = acc;
+      for (int c = 0; c < kSub; ++c) x[c] = S[rr][o + c];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) {
+        x[c] *= invd[o + c];
+#pragma unroll
+        for (int c2 = c + 1; c2 < kSub; ++c2) x[c2] = fma(-x[c], S[o + c2][o + c], x[c2]);
+      }
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) S[rr][o + c] = x[c];
     }
     __syncthreads();
-    for (int idx = tid; idx < nb * kSub; idx += blockDim.x) {
-      const int rr = o + kSub + idx / kSub, c = idx % kSub;
-      S[rr][o + c] = T[rr][c];
-    }
-    __syncthreads();
-    // trailing lower part: S[r][l] -= sum_m L[r][o+m] L[l][o+m], o+16 <= l <= r
-    for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
-      const int rr = o + kSub + idx / nb, l = o + kSub + idx % nb;
-      if (l <= rr) {
-        double acc = S[rr][l];
-#pragma unroll
-        for (int m = 0; m < kSub; ++m) acc = fma(-S[rr][o + m], S[l][o + m], acc);
-        S[rr][l] = acc;
+    // trailing lower part: S[r][l] -= sum_m L[r][o+m] L[l][o+m] for
+    // o+16 <= l <= r, as 8 x 8 tiles on or below the diagonal
+    {
+      const int nt = nb / 8, ntiles = nt * (nt + 1) / 2, b0 = o + kSub;
+      for (int t = warp; t < ntiles; t += kPanelThreads / 32) {
+        int ti = 0, tt = t;
+        while (tt > ti) tt -= ++ti;   // t -> (ti, tj), tj <= ti
+        const int tj = tt;
+        const int row = b0 + 8 * ti + fr, col = b0 + 8 * tj + fc2;
+        double d0 = S[row][col], d1 = S[row][col + 1];
+        tile_pqt(d0, d1, S, b0 + 8 * ti, S, b0 + 8 * tj, o, o + kSub, -1.0);
+        if (col <= row) S[row][col] = d0;
+        if (col + 1 <= row) S[row][col + 1] = d1;
       }
     }
     __syncthreads();
   }
 
-  // ---- inverse by doubling: blocks of 16 -> 32 -> 64.  For a pair of
-  // diagonal blocks of size b at offset q: X21 = -X22 (L21 X11).
-  for (int b = kSub; b < NB; b *= 2) {
-    const int npairs = NB / (2 * b);
-    // T = L21 X11 for every pair (b x b each)
-    for (int idx = tid; idx < npairs * b * b; idx += blockDim.x) {
-      const int pq = idx / (b * b), e = idx % (b * b), i = e / b, j = e % b;
-      const int q = pq * 2 * b;
-      double acc = 0.0;
-      for (int l = j; l < b; ++l) acc = fma(S[q + b + i][q + l], Xd[q + l][q + j], acc);
-      T[q + b + i][q + j] = acc;
-    }
-    __syncthreads();
-    for (int idx = tid; idx < npairs * b * b; idx += blockDim.x) {
-      const int pq = idx / (b * b), e = idx % (b * b), i = e / b, j = e % b;
-      const int q = pq * 2 * b;
-      double acc = 0.0;
-      for (int l = 0; l <= i; ++l) acc = fma(Xd[q + b + i][q + b + l], T[q + b + l][q + j], acc);
-      Xd[q + b + i][q + j] = -acc;
-    }
-    __syncthreads();
-  }
+  // ---- inverse: the four 16 x 16 diagonal inverses at once, then doubling
+  // 16 -> 32 -> 64
+  if (warp < NB / kSub) invert_16(S, Xd, invd, warp * kSub);
+  __syncthreads();
+  doubling_level<16>(S, Xd, T);
+  doubling_level<32>(S, Xd, T);
 
   if (blockIdx.x == 0) {
-    for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
+    // L11 itself is not written back: nothing reads the diagonal blocks of L
+    // later, and the other CTAs of this launch may still be reading A11.
+    for (int idx = tid; idx < kb * kb; idx += kPanelThreads) {
       const int i = idx / kb, j = idx % kb;
-      // L11 itself is not written back: nothing reads the diagonal blocks of L
-      // later, and the other CTAs of this launch may still be reading A11.
-      const double x = Xd[i][j];
-      X[(k + i) * d + k + j] = x;            // lower (zeros above)
-      Y[(k + j) * d + k + i] = x;            // its transpose, upper
+      X[(k + i) * d + k + j] = Xd[i][j];   // lower (zeros above), row by row
+    }
+    for (int idx = tid; idx < kb * kb; idx += kPanelThreads) {
+      const int j = idx / kb, i = idx % kb;
+      Y[(k + j) * d + k + i] = Xd[i][j];   // its transpose, upper, row by row
     }
     return;
   }
-  // ---- L21 slice = A21 slice X11^T: thread (ty, tx) computes a 4 x 4 tile,
-  // L21[i][c] = sum_l R[i][l] X11[c][l]; X11 is staged transposed in T first
-  // so that the loop reads it along rows (free of bank conflicts).
-  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
-    const int c = idx / NB, l = idx % NB;
-    T[l][c] = Xd[c][l];
+  // ---- L21 slice = A21 slice X11^T: 32 x 64 = 4 x 8 tiles, 4 per warp
+  {
+    const int ti = warp & 3, tj0 = (warp >> 2) * 4;
+    double acc[4][2] = {};
+    for (int kk = 0; kk < NB; kk += 4) {
+      const double a = R[8 * ti + fr][kk + (lane & 3)];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        dmma_m8n8k4(acc[j][0], acc[j][1], a, Xd[8 * (tj0 + j) + fr][kk + (lane & 3)]);
+    }
+    const int i = 8 * ti + fr;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = 8 * (tj0 + j) + fc2 + h;
+        if (i < rows && c < kb) A[(r0 + i) * d + k + c] = acc[j][h];
+      }
   }
-  __syncthreads();
-  const int ty = tid >> 4, tx = tid & 15, i0 = 4 * ty, l0 = 4 * tx;
-  double acc[4][4] = {};
-  for (int l = 0; l < NB; ++l) {
-    double rv[4], xv[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) rv[a] = R[i0 + a][l];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) xv[b] = T[l][l0 + b];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fma(rv[a], xv[b], acc[a][b]);
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      if (i0 + a < rows && l0 + b < kb)
-        A[(r0 + i0 + a) * d + k + l0 + b] = acc[a][b];
 }
 
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
@@ -368,7 +453,7 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     for (int64_t k = k0; k < kend; k += NB) {
       const int kb = (int)((d - k) < NB ? (d - k) : NB);
       const int64_t m = d - k - kb;
-      const int grid = 1 + (int)((m + NB - 1) / NB);
+      const int grid = 1 + (int)((m + kSlice - 1) / kSlice);
       chol_panel_kernel<<<grid, kPanelThreads, kPanelSmem, st>>>(L.A, d, k, kb, L.X, L.Y, L.hdr);
       NVFP4_LAUNCH_CHECK();
       count_launches(1);
