@@ -239,7 +239,10 @@ size_t nvfp4_layer_error_workspace_size(int64_t d_out, int64_t d_in);
 
 /* W, w_dtype : the original weights (dead columns contribute 0 because their
  *           H row is 0).  codes/scales/global_scale from the quantize call.
- * H       : d_in x d_in fp32, undamped.
+ * H       : d_in x d_in fp32, undamped, symmetric (the Hessian X^T X).  The
+ *           error is evaluated as <H, E^T E> with E = W - Q: the Gram matrix
+ *           E^T E is formed on its 128 x 128 tiles on or below the diagonal
+ *           (3xTF32 on the tensor cores), and only those tiles of H are read.
  * err_out : device fp64 scalar out.
  * ws      : at least nvfp4_layer_error_workspace_size() bytes. */
 nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t* codes,

@@ -87,15 +87,17 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
                         int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
                         cudaStream_t st);
 
-// C = beta C + alpha P Q^T in fp64 on the CUDA cores (same operand conventions
-// as gemm_nt_tc; C2 = C^T needs beta == 0; lower: only tiles on or below the
-// diagonal; ktri: 0 dense P, 1 P upper triangular, 2 P lower triangular -- the
-// zero part of K is skipped).
+// C = beta C + alpha P Q^T in fp64 on the tensor cores (mma.sync m8n8k4; same
+// operand conventions as gemm_nt_tc; C2 = C^T needs beta == 0; lower: only
+// tiles on or below the diagonal; ktri: 0 dense P, 1 P upper triangular, 2 P
+// lower triangular -- the zero part of K is skipped).  P and Q go through TMA:
+// 16-byte aligned, even leading dimensions and batch strides, K a multiple of
+// 16.  A wait that runs out records NVFP4_ERR_TIMEOUT in *status.
 nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_t ldp,
                       int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
                       double beta, double* C, int64_t ldc, int64_t strideC, double* C2,
                       int64_t ldc2, int64_t strideC2, int batch, int lower, int ktri,
-                      cudaStream_t st);
+                      int* status, cudaStream_t st);
 
 // ---- kernel launchers implemented in the .cu files -------------------------
 bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,

@@ -57,15 +57,22 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes,
   }
 }
 
-// E = W - Q in fp32 (W bf16 or fp32).
+// Et = (W - Q)^T in fp32 (W bf16 or fp32) for a 64 x 64 tile of W: one
+// thread per (row, 16-weight block) computes its 16 errors with a single
+// rounding each, the tile is transposed through shared memory, and Et's rows
+// (ldE >= d_out apart) are written whole.
 template <typename T>
-__global__ void error_matrix_kernel(const T* __restrict__ W, const uint8_t* __restrict__ codes,
-                                    const uint8_t* __restrict__ scales,
-                                    const float* __restrict__ sg_ptr, int64_t nblocks,
-                                    float* __restrict__ E) {
+__global__ void __launch_bounds__(256)
+    error_t_kernel(const T* __restrict__ W, const uint8_t* __restrict__ codes,
+                   const uint8_t* __restrict__ scales, const float* __restrict__ sg_ptr,
+                   int64_t d_out, int64_t d_in, float* __restrict__ Et, int64_t ldE) {
+  __shared__ float tile[64][65];
   const float sg = *sg_ptr;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks;
-       b += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int t = threadIdx.x, row = t >> 2, blk = t & 3;
+  const int64_t r = r0 + row, cb = c0 + 16 * blk;
+  if (r < d_out && cb < d_in) {
+    const int64_t b = r * (d_in / 16) + cb / 16;
     const uint2 c = reinterpret_cast<const uint2*>(codes)[b];
     const float sb = (float)e4m3_value(scales[b] & 0x7F);
     const uint64_t p = ((uint64_t)c.y << 32) | c.x;
@@ -73,23 +80,40 @@ __global__ void error_matrix_kernel(const T* __restrict__ W, const uint8_t* __re
     for (int j = 0; j < 16; ++j) {
       float w;
       if constexpr (sizeof(T) == 2)
-        w = __uint_as_float((uint32_t)W[16 * b + j] << 16);
+        w = __uint_as_float((uint32_t)W[r * d_in + cb + j] << 16);
       else
-        w = W[16 * b + j];
+        w = W[r * d_in + cb + j];
       // w - (e2m1 * e4m3) * s_g with a single rounding
-      E[16 * b + j] = fmaf(-e2m1_value((uint32_t)(p >> (4 * j)) & 0xF) * sb, sg, w);
+      tile[16 * blk + j][row] = fmaf(-e2m1_value((uint32_t)(p >> (4 * j)) & 0xF) * sb, sg, w);
     }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) tile[16 * blk + j][row] = 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int idx = t + 256 * q, j = idx >> 6, rr = idx & 63;
+    if (c0 + j < d_in && r0 + rr < d_out) Et[(c0 + j) * ldE + r0 + rr] = tile[j][rr];
   }
 }
 
-// sum_ij EH_ij * E_ij in fp64
-__global__ void dot_kernel(const float* __restrict__ A, const float* __restrict__ B, int64_t n,
-                           double* __restrict__ partial) {
+// sum_ij H_ij G_ij in fp64 with G = E^T E known on the 128 x 128 tiles on or
+// below the diagonal only (the tile size of gemm_nt_tc's lower mode): by the symmetry of G and H an off-diagonal tile
+// stands for its mirror image too (weight 2), a diagonal tile for itself.
+// Rows are shared out over the CTAs; tiles above the diagonal are not read.
+__global__ void sym_tile_dot_kernel(const float* __restrict__ H, const float* __restrict__ G,
+                                    int64_t d, double* __restrict__ partial) {
   __shared__ double part[32];
   double s = 0.0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    s += (double)A[i] * (double)B[i];
+  for (int64_t i = blockIdx.x; i < d; i += gridDim.x) {
+    const int64_t jdiag = (i / 128) * 128;
+    const int64_t jend = (jdiag + 128) < d ? (jdiag + 128) : d;
+    for (int64_t j = threadIdx.x; j < jend; j += blockDim.x) {
+      const double hg = (double)H[i * d + j] * (double)G[i * d + j];
+      s += j < jdiag ? 2.0 * hg : hg;
+    }
+  }
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
   __syncthreads();
@@ -131,40 +155,46 @@ nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const f
   return NVFP4_OK;
 }
 
+int64_t et_ld(int64_t d_out) { return (d_out + 31) / 32 * 32; }
+
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in) {
-  return kWsHeader + 2 * align256(sizeof(float) * d_out * d_in) +
-         align256(sizeof(double) * kDotBlocks);
+  return kWsHeader + align256(sizeof(float) * et_ld(d_out) * d_in) +
+         align256(sizeof(float) * d_in * d_in) + align256(sizeof(double) * kDotBlocks);
 }
 
+// tr(E H E^T) = <H, E^T E>: the Gram matrix G = E^T E is a symmetric
+// product, so only its tiles on or below the diagonal are formed (half the
+// flops of E H), on the tensor cores (3xTF32), then dotted with H.
 nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* codes,
                                 const uint8_t* scales, const float* sg, const float* H,
                                 int64_t d_out, int64_t d_in, double* err, void* ws,
                                 cudaStream_t st) {
   char* p = static_cast<char*>(ws) + kWsHeader;
-  float* E = reinterpret_cast<float*>(p);
-  float* EH = reinterpret_cast<float*>(p + align256(sizeof(float) * d_out * d_in));
-  double* part =
-      reinterpret_cast<double*>(p + 2 * align256(sizeof(float) * d_out * d_in));
-  const int64_t nb = d_out * (d_in / kBlock);
-  if (nb == 0) {
+  const int64_t ldE = et_ld(d_out);
+  float* Et = reinterpret_cast<float*>(p);
+  float* G = reinterpret_cast<float*>(p + align256(sizeof(float) * ldE * d_in));
+  double* part = reinterpret_cast<double*>(p + align256(sizeof(float) * ldE * d_in) +
+                                           align256(sizeof(float) * d_in * d_in));
+  if (d_out == 0 || d_in == 0) {
     NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
     return NVFP4_OK;
   }
+  const dim3 tgrid((unsigned)((d_in + 63) / 64), (unsigned)((d_out + 63) / 64));
   if (wt == NVFP4_BF16)
-    error_matrix_kernel<uint16_t><<<grid_for(nb, 256), 256, 0, st>>>(
-        static_cast<const uint16_t*>(W), codes, scales, sg, nb, E);
+    error_t_kernel<uint16_t><<<tgrid, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes,
+                                                    scales, sg, d_out, d_in, Et, ldE);
   else
-    error_matrix_kernel<float><<<grid_for(nb, 256), 256, 0, st>>>(
-        static_cast<const float*>(W), codes, scales, sg, nb, E);
+    error_t_kernel<float><<<tgrid, 256, 0, st>>>(static_cast<const float*>(W), codes, scales,
+                                                 sg, d_out, d_in, Et, ldE);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-  // EH = E H^T = E H (H symmetric) on the tensor cores
   int* status = static_cast<int*>(ws);
   NVFP4_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  nvfp4_status s = gemm_nt_tc((int)d_out, (int)d_in, (int)d_in, 1.f, E, d_in, 0, H, d_in, 0,
-                              0.f, EH, d_in, 0, nullptr, 0, 0, 1, 0, status, st);
+  // G = Et Et^T (d_in x d_in, K = d_out), lower tiles only
+  nvfp4_status s = gemm_nt_tc((int)d_in, (int)d_in, (int)d_out, 1.f, Et, ldE, 0, Et, ldE, 0,
+                              0.f, G, d_in, 0, nullptr, 0, 0, 1, 1, status, st);
   if (s != NVFP4_OK) return s;
-  dot_kernel<<<kDotBlocks, 256, 0, st>>>(E, EH, d_out * d_in, part);
+  sym_tile_dot_kernel<<<kDotBlocks, 256, 0, st>>>(H, G, d_in, part);
   NVFP4_LAUNCH_CHECK();
   sum_partials_kernel<<<1, 32, 0, st>>>(part, kDotBlocks, err);
   NVFP4_LAUNCH_CHECK();

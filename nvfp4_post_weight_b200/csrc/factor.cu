@@ -461,14 +461,14 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
       if (m <= 0 || nc <= 0) continue;
       const double* L21 = L.A + (k + kb) * d + k;
       nvfp4_status s = dgemm_nt((int)m, (int)nc, kb, -1.0, L21, d, 0, L21, d, 0, 1.0,
-                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 0, 0, st);
+                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 0, 0, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
     }
     const int64_t m2 = d - kend;
     if (m2 > 0) {
       const double* Lb = L.A + kend * d + k0;
       nvfp4_status s = dgemm_nt((int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, 0, Lb, d, 0,
-                                1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0, st);
+                                1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
     }
   }
@@ -482,11 +482,11 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     const int64_t stride = 2 * b * (d + 1);
     if (npairs > 0) {
       nvfp4_status s = dgemm_nt((int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
-                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1, st);
+                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
       s = dgemm_nt((int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
                      0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, 2,
-                     st);
+                     &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
     }
     const int64_t r0 = npairs * 2 * b;   // a ragged pair: full left block, rr rows right
@@ -494,11 +494,11 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
       nvfp4_status s = dgemm_nt((int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0,
-                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1, st);
+                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
       // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
       s = dgemm_nt((int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
-                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2, st);
+                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;
     }
   }
