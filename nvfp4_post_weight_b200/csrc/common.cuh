@@ -137,6 +137,33 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
                                 cudaStream_t st);
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in);
 
+// Programmatic dependent launch.  The kernels of a serial chain (panel ->
+// update -> panel, replay -> update -> replay) are launched with
+// launch_chained() and call pdl_wait() before their first global memory
+// access; it returns once the previous kernel of the stream has completed and
+// its writes are visible.  The launch itself and the set-up before the wait
+// (barrier init, tensor-map prefetch, TMEM allocation) overlap the previous
+// kernel's completion.  No kernel triggers its dependents early: measured on
+// the 4096-wide layer, CTAs of the next kernel parked beside a running panel
+// or GEMM slowed it more than the earlier start gained.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // D (8x8) += A (8x4) B (4x8) in fp64 on the tensor cores (warp-wide
 // mma.sync m8n8k4; tcgen05 has no fp64 kind).  Fragments per lane:
 // a = A[lane/4][lane%4], b = B[lane%4][lane/4], d = D[lane/4][2*(lane%4)+{0,1}].

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kThreads)
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -221,10 +222,9 @@ nvfp4_status launch_dgemm(int M, int N, int K, double alpha, const double* P, in
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(dgemm_nt_kernel<TL>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)G::kSmem));
-  dgemm_nt_kernel<TL><<<grid, kThreads, G::kSmem, st>>>(mp, mq, M, N, K, alpha, beta, C, ldc,
-                                                        strideC, C2, ldc2, strideC2, lower,
-                                                        ktri, status);
-  NVFP4_LAUNCH_CHECK();
+  NVFP4_CUDA_TRY(launch_chained(dgemm_nt_kernel<TL>, grid, dim3(kThreads), G::kSmem, st, mp, mq,
+                                M, N, K, alpha, beta, C, ldc, strideC, C2, ldc2, strideC2, lower,
+                                ktri, status));
   count_launches(1);
   return NVFP4_OK;
 }

@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kPanelThreads)
   const int64_t r0 = k + kb + (int64_t)(blockIdx.x - 1) * kSlice;   // slice rows (CTA >= 1)
   const int64_t rem = d - r0;
   const int rows = blockIdx.x == 0 ? 0 : (int)(rem < kSlice ? rem : kSlice);
+  pdl_wait();
 
   {   // all global loads of a thread are issued before any is used
     constexpr int kPer = NB * NB / kPanelThreads;        // 16
@@ -454,8 +455,8 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
       const int kb = (int)((d - k) < NB ? (d - k) : NB);
       const int64_t m = d - k - kb;
       const int grid = 1 + (int)((m + kSlice - 1) / kSlice);
-      chol_panel_kernel<<<grid, kPanelThreads, kPanelSmem, st>>>(L.A, d, k, kb, L.X, L.Y, L.hdr);
-      NVFP4_LAUNCH_CHECK();
+      NVFP4_CUDA_TRY(launch_chained(chol_panel_kernel, dim3(grid), dim3(kPanelThreads),
+                                    kPanelSmem, st, L.A, d, k, kb, L.X, L.Y, L.hdr));
       count_launches(1);
       const int64_t nc = kend - (k + kb);   // columns of the outer block still to come
       if (m <= 0 || nc <= 0) continue;

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restri
                                                            float* __restrict__ Uh,
                                                            float* __restrict__ Ul) {
   __shared__ float t[32][33];
+  pdl_wait();
   const int64_t j0 = e + (int64_t)blockIdx.x * 32;
   const int k0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(kReplayThreads)
   double* invd = Ut + kUTiles * 256;                         // 128
   double* rows = invd + kLazyBatch;                          // kRowsPerCta x 128
   const int nblk = bw / kBlock;
+  pdl_wait();
   {
     // Stage the batch's upper block-triangular part of U as 16 x 16 fp64
     // tiles.  Thread t handles element e = t of every tile (kReplayThreads ==
@@ -411,18 +413,19 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
     const int bw = (int)((d_in - c0) < kLazyBatch ? (d_in - c0) : kLazyBatch);
     {
       ProfileScope ps(kPhaseReplay, st);
-      replay_kernel<<<rgrid, kReplayThreads, kReplaySmem, st>>>(
-          L.Wt, U, d_out, d_in, (int)c0, bw, sg, codes, scales, L.Dh, L.Dl, L.rowerr);
-      NVFP4_LAUNCH_CHECK();
+      NVFP4_CUDA_TRY(launch_chained(replay_kernel, dim3(rgrid), dim3(kReplayThreads),
+                                    kReplaySmem, st, L.Wt, U, d_out, d_in, (int)c0, bw, sg,
+                                    codes, scales, L.Dh, L.Dl, L.rowerr));
       count_launches(1);
     }
     const int64_t e = c0 + bw;
     if (e < d_in) {
       ProfileScope ps(kPhaseUpdate, st);
       // W~[:, e:] -= Delta[:, :bw] U[c0:c0+bw, e:]   (bw = 128 here)
-      split_u_rows_kernel<<<dim3((unsigned)((d_in - e + 31) / 32), kLazyBatch / 32), 256, 0,
-                            st>>>(U, d_in, c0, e, L.Uh, L.Ul);
-      NVFP4_LAUNCH_CHECK();
+      NVFP4_CUDA_TRY(launch_chained(split_u_rows_kernel,
+                                    dim3((unsigned)((d_in - e + 31) / 32), kLazyBatch / 32),
+                                    dim3(256), 0, st, U, (int64_t)d_in, (int64_t)c0, e, L.Uh,
+                                    L.Ul));
       count_launches(1);
       nvfp4_status s = launch_update_tc(maps, L.Wt, d_in, d_out, d_in, e, &L.hdr->status, st);
       if (s != NVFP4_OK) return s;

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  pdl_wait();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -380,9 +381,9 @@ nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int6
   const int sms = num_sms();
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(update_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-  update_tc_kernel<<<n_tiles < sms ? n_tiles : sms, kThreads, kSmem, st>>>(
-      m.Dh, m.Dl, m.Uh, m.Ul, m.W, (int)e, n_rb, n_tiles, status);
-  NVFP4_LAUNCH_CHECK();
+  NVFP4_CUDA_TRY(launch_chained(update_tc_kernel, dim3(n_tiles < sms ? n_tiles : sms),
+                                dim3(kThreads), kSmem, st, m.Dh, m.Dl, m.Uh, m.Ul, m.W, (int)e,
+                                n_rb, n_tiles, status));
   count_launches(1);
   return NVFP4_OK;
 }
