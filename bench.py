@@ -190,7 +190,6 @@ def run_ours(args, rank, world, local_rank):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     n0 = B.lib().nvfp4_launch_count()
-    B.lib().nvfp4_profile_begin()
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
@@ -198,14 +197,23 @@ def run_ours(args, rank, world, local_rank):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    import ctypes
-    ms_ph = (ctypes.c_double * 6)()
-    ln_ph = (ctypes.c_longlong * 6)()
-    B.lib().nvfp4_profile_end(ms_ph, ln_ph, 6)
     launches = B.lib().nvfp4_launch_count() - n0
     step_ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dist, dev)
     if dist:
         tdist.barrier()
+
+    # phase breakdown: the same steps again with the library's per-phase
+    # events on (they sit between the kernels, so this pass is not the one
+    # whose time is reported as the step time)
+    import ctypes
+    B.lib().nvfp4_profile_begin()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    ms_ph = (ctypes.c_double * 6)()
+    ln_ph = (ctypes.c_longlong * 6)()
+    B.lib().nvfp4_profile_end(ms_ph, ln_ph, 6)
 
     # end to end through the C ABI from pinned host buffers: H2D of W and X,
     # the solve, D2H of codes, scales and the global scale

@@ -112,12 +112,17 @@ int hessian_tc_take_status(cudaStream_t st);
 struct UpdateMaps {
   CUtensorMap Dh, Dl, Uh, Ul, W;   // W: the fp64 working copy (d_out x d_in)
 };
+// Maps of the update operands: Dh/Dl (d_out x kcols) and Uh/Ul (d_in x kcols)
+// hold deltas and U rows K-contiguous, kcols K values per row.
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
-                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in);
-// W~[:, e:] -= (Dh + Dl)(Uh + Ul)[:, e:] (3xTF32, fp64 W~); a timed-out wait
-// sets NVFP4_ERR_TIMEOUT in *status.
-nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int64_t d_out,
-                              int64_t d_in, int64_t e, int* status, cudaStream_t st);
+                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in,
+                      int64_t kcols);
+// W~[:, e:e_end] -= sum over nkb 128-deep K blocks from K offset kofs of
+// (Dh + Dl)(Uh + Ul)^T (3xTF32, fp64 W~); keep_w keeps W~ in L2 (evict last)
+// instead of streaming it.  A timed-out wait sets NVFP4_ERR_TIMEOUT in *status.
+nvfp4_status launch_update_tc(const UpdateMaps& m, int64_t d_out, int64_t d_in, int64_t e,
+                              int64_t e_end, int kofs, int nkb, bool keep_w, int* status,
+                              cudaStream_t st);
 nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                             int64_t d, int beta, cudaStream_t st);
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,

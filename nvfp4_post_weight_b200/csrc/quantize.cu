@@ -40,13 +40,22 @@ struct QuantHeader {   // workspace header (first 256 bytes)
   unsigned amax_bits;  // max |W| as fp32 bits (non-negative floats order as uints)
 };
 
+// Columns per super-batch.  Inside a super-batch every lazy batch updates only
+// the super-batch's later columns (an fp64 W~ slab of d_out x 1024 that stays
+// in L2); the super-batch's deltas reach the columns beyond it in one update
+// with K = 1024, so the HBM-resident rest of W~ is read and written once per
+// super-batch instead of once per batch.  Narrow layers keep one batch per
+// super-batch (the plain lazy-batch scheme).
+int64_t super_width(int64_t d_in) { return d_in >= 2048 ? 8 * kLazyBatch : kLazyBatch; }
+
 struct QuantLayout {
   QuantHeader* hdr;
+  int64_t S;       // super-batch width (K values per row of the four below)
   double* Wt;      // d_out x d_in working copy
-  float* Dh;       // d_out x 128: the batch's deltas, tf32-rounded part
-  float* Dl;       // d_out x 128: remainder (delta - Dh)
-  float* Uh;       // d_in x 128: the batch's rows of U transposed, tf32 part
-  float* Ul;       // d_in x 128: remainder
+  float* Dh;       // d_out x S: the super-batch's deltas, tf32-rounded part
+  float* Dl;       // d_out x S: remainder (delta - Dh)
+  float* Uh;       // d_in x S: the super-batch's rows of U transposed, tf32 part
+  float* Ul;       // d_in x S: remainder
   double* rowerr;  // d_out
 };
 
@@ -54,17 +63,18 @@ QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in) {
   char* p = static_cast<char*>(ws);
   QuantLayout L;
   L.hdr = reinterpret_cast<QuantHeader*>(p);
+  L.S = super_width(d_in);
   size_t off = kWsHeader;
   L.Wt = reinterpret_cast<double*>(p + off);
   off += align256(sizeof(double) * d_out * d_in);
   L.Dh = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d_out * kLazyBatch);
+  off += align256(sizeof(float) * d_out * L.S);
   L.Dl = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d_out * kLazyBatch);
+  off += align256(sizeof(float) * d_out * L.S);
   L.Uh = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * kLazyBatch * d_in);
+  off += align256(sizeof(float) * L.S * d_in);
   L.Ul = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * kLazyBatch * d_in);
+  off += align256(sizeof(float) * L.S * d_in);
   L.rowerr = reinterpret_cast<double*>(p + off);
   return L;
 }
@@ -134,60 +144,66 @@ constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a ba
 // Index of the upper tile (p, q), q >= p, in the packed tile array.
 __device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p) / 2 + q; }
 
-// Uh[j][k] + Ul[j][k] = U[c0 + k][j] for the batch rows k < 128 and the
-// columns j >= e right of the batch: the trailing update's B operand, stored
-// K-contiguous.  32x32 tiles transposed through shared memory.
+// Uh[j][k] + Ul[j][k] = U[cs + k][j] for the super-batch's rows k < nk and
+// the columns j >= j0: the update's B operand, stored K-contiguous (S values
+// per row).  32 x 32 tiles transposed through shared memory.
 __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restrict__ U,
-                                                           int64_t d_in, int64_t c0, int64_t e,
+                                                           int64_t d_in, int64_t cs, int nk,
+                                                           int64_t j0, int64_t S,
                                                            float* __restrict__ Uh,
                                                            float* __restrict__ Ul) {
   __shared__ float t[32][33];
   pdl_wait();
-  const int64_t j0 = e + (int64_t)blockIdx.x * 32;
+  const int64_t jb = j0 + (int64_t)blockIdx.x * 32;
   const int k0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   for (int r = ty; r < 32; r += 8) {
-    const int64_t j = j0 + tx;
-    t[r][tx] = j < d_in ? U[(c0 + k0 + r) * d_in + j] : 0.f;
+    const int64_t j = jb + tx;
+    t[r][tx] = (j < d_in && k0 + r < nk) ? U[(cs + k0 + r) * d_in + j] : 0.f;
   }
   __syncthreads();
   for (int r = ty; r < 32; r += 8) {
-    const int64_t j = j0 + r;
-    if (j < d_in) {
+    const int64_t j = jb + r;
+    if (j < d_in && k0 + tx < nk) {
       const float u = t[tx][r];
       const float h = sm100::tf32_rn(u);
-      Uh[j * kLazyBatch + k0 + tx] = h;
-      Ul[j * kLazyBatch + k0 + tx] = u - h;
+      Uh[j * S + k0 + tx] = h;
+      Ul[j * S + k0 + tx] = u - h;
     }
   }
 }
 
 // One candidate's replay of the in-block GPTQ updates (fp64).  v holds the
 // block's 16 current values and is consumed.  Ud points at the block's
-// diagonal 16x16 tile (row-major), invd at its 1/U_jj.  Returns the score
-// sum delta_j^2; delta and the packed code nibbles are written out.
+// diagonal 16x16 tile (row-major, 16-byte aligned), invd at its 1/U_jj.
+// Returns the score sum delta_j^2; delta and the signed rounded magnitudes
+// q_j / s (exact in fp32) are written out -- the code nibbles are derived
+// once, from the winner's magnitudes, not by every candidate.
 __device__ __forceinline__ double replay(double (&v)[16], double s, double inv_s,
                                          const double* __restrict__ Ud,
                                          const double* __restrict__ invd, double (&dl)[16],
-                                         uint64_t& packed) {
+                                         float (&sq)[16]) {
   double score = 0.0;
-  uint64_t pk = 0;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const double x = __dmul_rn(v[j], inv_s);
     const double r = e2m1_round_mag(fabs(x));
-    const uint32_t idx = e2m1_index(r);
     const double sr = x < 0.0 ? -r : r;
-    const uint32_t nib = idx | ((x < 0.0 && idx) ? 8u : 0u);
-    pk |= (uint64_t)nib << (4 * j);
+    sq[j] = (float)sr;
     const double res = __fma_rn(-sr, s, v[j]);       // v_j - q_j, one rounding
     const double d = __dmul_rn(res, invd[j]);
     dl[j] = d;
     score = __fma_rn(d, d, score);
+    // the later columns of the block absorb d: row j of the tile, two
+    // values per 16-byte load
+    const double2* Urow = reinterpret_cast<const double2*>(Ud + j * 16);
 #pragma unroll
-    for (int i = j + 1; i < 16; ++i) v[i] = __fma_rn(-d, Ud[j * 16 + i], v[i]);
+    for (int p = (j + 1) / 2; p < 8; ++p) {
+      const double2 u = Urow[p];
+      if (2 * p > j) v[2 * p] = __fma_rn(-d, u.x, v[2 * p]);
+      v[2 * p + 1] = __fma_rn(-d, u.y, v[2 * p + 1]);
+    }
   }
-  packed = pk;
   return score;
 }
 
@@ -207,7 +223,8 @@ __global__ void __launch_bounds__(kReplayThreads)
                               int64_t d_out, int64_t d_in, int c0, int bw,
                               const float* __restrict__ sg_ptr, uint8_t* __restrict__ codes,
                               uint8_t* __restrict__ scales, float* __restrict__ Dh,
-                              float* __restrict__ Dl, double* __restrict__ rowerr) {
+                              float* __restrict__ Dl, int64_t ldD, int kofs,
+                              double* __restrict__ rowerr) {
   extern __shared__ double4 smem_d4[];
   double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
   double* invd = Ut + kUTiles * 256;                         // 128
@@ -240,6 +257,7 @@ __global__ void __launch_bounds__(kReplayThreads)
   const int warp = threadIdx.x >> 5;
   const int rloc = warp * 2 + half;
   double* row = rows + rloc * kLazyBatch;
+  float* mrow = reinterpret_cast<float*>(rows + kRowsPerCta * kLazyBatch) + rloc * 16;
   const unsigned FULL = 0xffffffffu;
 
   for (int64_t rb = (int64_t)blockIdx.x * kRowsPerCta; rb < d_out;
@@ -280,8 +298,8 @@ __global__ void __launch_bounds__(kReplayThreads)
         }
       }
       double dl[16];
-      uint64_t pk;
-      const double score = replay(v, s, inv_s, Ud, idb, dl, pk);
+      float sq[16];
+      const double score = replay(v, s, inv_s, Ud, idb, dl, sq);
       if constexpr (kRule == kRuleSchurReplay) sel = score;
 
       // the chosen candidate: k0 for the amax rule, else the argmin of the
@@ -304,22 +322,44 @@ __global__ void __launch_bounds__(kReplayThreads)
       const bool live = amax > 0.0;
       __syncwarp();
       if (hl == bl) {
-        // the winner publishes its deltas in place of the block's values
+        // the winner publishes its deltas in place of the block's values and
+        // its rounded magnitudes for the code nibbles
 #pragma unroll
-        for (int j = 0; j < 16; ++j) row[16 * b + j] = live ? dl[j] : 0.0;
-        if (valid) {
-          *reinterpret_cast<uint64_t*>(codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
-              live ? pk : 0ull;
-          scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
+        for (int j = 0; j < 16; ++j) {
+          row[16 * b + j] = live ? dl[j] : 0.0;
+          mrow[j] = sq[j];
         }
       }
       if (live) rowsum += best;
       __syncwarp();
+      {
+        // lane hl encodes column hl of the winner; the 16 nibbles are OR-ed
+        // into the block's 8 code bytes (low nibble = even column)
+        const float m = mrow[hl], am = fabsf(m);
+        const uint32_t idx =
+            (uint32_t)(am < 2.f ? 2.f * am : (am < 4.f ? am + 2.f : 0.5f * am + 4.f));
+        const uint32_t nib = live ? (idx | ((m < 0.f && idx) ? 8u : 0u)) : 0u;
+        uint32_t lo_w = hl < 8 ? nib << (4 * hl) : 0u, hi_w = hl < 8 ? 0u : nib << (4 * (hl - 8));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          lo_w |= __shfl_xor_sync(FULL, lo_w, o, 16);
+          hi_w |= __shfl_xor_sync(FULL, hi_w, o, 16);
+        }
+        if (valid && hl == 0) {
+          *reinterpret_cast<uint2*>(codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
+              make_uint2(lo_w, hi_w);
+          scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
+        }
+      }
       // later columns of the batch absorb the chosen block's deltas
       if (b + 1 < nblk) {
         double d[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) d[j] = row[16 * b + j];
+        for (int j = 0; j < 8; ++j) {
+          const double2 dd = reinterpret_cast<const double2*>(row + 16 * b)[j];
+          d[2 * j] = dd.x;
+          d[2 * j + 1] = dd.y;
+        }
         for (int q = b + 1; q < nblk; ++q) {
           const double* Uq = Ut + utile(b, q) * 256 + hl;
           double acc = row[16 * q + hl];
@@ -334,8 +374,8 @@ __global__ void __launch_bounds__(kReplayThreads)
       for (int c = hl; c < bw; c += 16) {
         const double x = row[c];
         const float h = sm100::tf32_rn((float)x);
-        Dh[r * kLazyBatch + c] = h;
-        Dl[r * kLazyBatch + c] = (float)(x - (double)h);
+        Dh[r * ldD + kofs + c] = h;
+        Dl[r * ldD + kofs + c] = (float)(x - (double)h);
       }
       if (hl == 0) rowerr[r] += rowsum;
     }
@@ -364,14 +404,16 @@ int grid_for(int64_t n, int threads) {
 }
 
 constexpr size_t kReplaySmem =
-    sizeof(double) * (kUTiles * 256 + kLazyBatch + kRowsPerCta * kLazyBatch);
+    sizeof(double) * (kUTiles * 256 + kLazyBatch + kRowsPerCta * kLazyBatch) +
+    sizeof(float) * kRowsPerCta * 16;
 
 }  // namespace
 
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
+  const int64_t S = super_width(d_in);
   return kWsHeader + align256(sizeof(double) * d_out * d_in) +
-         2 * align256(sizeof(float) * d_out * kLazyBatch) +
-         2 * align256(sizeof(float) * kLazyBatch * d_in) + align256(sizeof(double) * d_out);
+         2 * align256(sizeof(float) * d_out * S) + 2 * align256(sizeof(float) * S * d_in) +
+         align256(sizeof(double) * d_out);
 }
 
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
@@ -405,29 +447,47 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kReplaySmem));
   UpdateMaps maps;
-  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in))
+  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in, L.S))
     return NVFP4_ERR_CUDA;
   const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
   const int rgrid = (int)(row_groups < 2 * kNumSMs ? row_groups : 2 * kNumSMs);
-  for (int64_t c0 = 0; c0 < d_in; c0 += kLazyBatch) {
-    const int bw = (int)((d_in - c0) < kLazyBatch ? (d_in - c0) : kLazyBatch);
-    {
-      ProfileScope ps(kPhaseReplay, st);
-      NVFP4_CUDA_TRY(launch_chained(replay_kernel, dim3(rgrid), dim3(kReplayThreads),
-                                    kReplaySmem, st, L.Wt, U, d_out, d_in, (int)c0, bw, sg,
-                                    codes, scales, L.Dh, L.Dl, L.rowerr));
-      count_launches(1);
-    }
-    const int64_t e = c0 + bw;
-    if (e < d_in) {
+  for (int64_t cs = 0; cs < d_in; cs += L.S) {
+    const int64_t send = (d_in - cs) < L.S ? d_in : cs + L.S;
+    const int64_t j0 = cs + kLazyBatch;   // first column any update of this super-batch touches
+    if (j0 < d_in) {
       ProfileScope ps(kPhaseUpdate, st);
-      // W~[:, e:] -= Delta[:, :bw] U[c0:c0+bw, e:]   (bw = 128 here)
+      const int nk = (int)(send - cs);
       NVFP4_CUDA_TRY(launch_chained(split_u_rows_kernel,
-                                    dim3((unsigned)((d_in - e + 31) / 32), kLazyBatch / 32),
-                                    dim3(256), 0, st, U, (int64_t)d_in, (int64_t)c0, e, L.Uh,
+                                    dim3((unsigned)((d_in - j0 + 31) / 32), (unsigned)((nk + 31) / 32)),
+                                    dim3(256), 0, st, U, (int64_t)d_in, cs, nk, j0, L.S, L.Uh,
                                     L.Ul));
       count_launches(1);
-      nvfp4_status s = launch_update_tc(maps, L.Wt, d_in, d_out, d_in, e, &L.hdr->status, st);
+    }
+    for (int64_t c0 = cs; c0 < send; c0 += kLazyBatch) {
+      const int bw = (int)((d_in - c0) < kLazyBatch ? (d_in - c0) : kLazyBatch);
+      const int kofs = (int)(c0 - cs);
+      {
+        ProfileScope ps(kPhaseReplay, st);
+        NVFP4_CUDA_TRY(launch_chained(replay_kernel, dim3(rgrid), dim3(kReplayThreads),
+                                      kReplaySmem, st, L.Wt, U, d_out, d_in, (int)c0, bw, sg,
+                                      codes, scales, L.Dh, L.Dl, L.S, kofs, L.rowerr));
+        count_launches(1);
+      }
+      const int64_t e = c0 + bw;
+      if (e < send) {
+        // the batch's deltas into the rest of the super-batch (W~ slab kept in L2)
+        ProfileScope ps(kPhaseUpdate, st);
+        nvfp4_status s = launch_update_tc(maps, d_out, d_in, e, send, kofs, 1, true,
+                                          &L.hdr->status, st);
+        if (s != NVFP4_OK) return s;
+      }
+    }
+    if (send < d_in) {
+      // the whole super-batch's deltas into every later column, K = send - cs
+      ProfileScope ps(kPhaseUpdate, st);
+      nvfp4_status s = launch_update_tc(maps, d_out, d_in, send, d_in, 0,
+                                        (int)((send - cs) / kLazyBatch), false, &L.hdr->status,
+                                        st);
       if (s != NVFP4_OK) return s;
     }
   }

@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmUh,
                      const __grid_constant__ CUtensorMap tmUl,
                      const __grid_constant__ CUtensorMap tmW, int e, int n_rb, int n_tiles,
-                     int* status) {
+                     int kofs, int nkb, int keep_w, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch(&tmUh);
     tma_prefetch(&tmUl);
     tma_prefetch(&tmW);
-    const uint64_t stream_pol = policy_evict_first(), keep_pol = policy_evict_last();
+    const uint64_t keep_pol = policy_evict_last();
+    const uint64_t w_pol = keep_w ? keep_pol : policy_evict_first();
     int s = 0, issued = 0, hw = 0;   // hw: W~ halves issued
     uint32_t ph = 0;
     bool ok = true;
@@ -186,9 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sm->w_full[wb], kWHalf);
         for (int q = 0; q < 2; ++q)
           tma_load_2d_hint(Wbuf + wb * kWHalf + q * kWBox, &tmW, &sm->w_full[wb],
-                           e + tn * UN + h * 32 + q * WBOX, rb * UM, stream_pol);
+                           e + tn * UN + h * 32 + q * WBOX, rb * UM, w_pol);
       }
-      for (int kc = 0; ok && kc < kNChunks; ++kc) {
+      for (int kk = 0; ok && kk < nkb * kNChunks; ++kk) {
+        const int kx = kofs + kk * KC;   // K coordinate of this chunk
         if (!mbar_wait(&sm->empty[s], ph ^ 1)) {
           give_up(sm, status);
           ok = false;
@@ -196,10 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&sm->full[s], kStage);
         uint8_t* st = ring + s * kStage;
-        tma_load_2d_hint(st, &tmDh, &sm->full[s], kc * KC, rb * UM, keep_pol);
-        tma_load_2d_hint(st + kAPart, &tmDl, &sm->full[s], kc * KC, rb * UM, keep_pol);
-        tma_load_2d_hint(st + 2 * kAPart, &tmUh, &sm->full[s], kc * KC, e + tn * UN, keep_pol);
-        tma_load_2d_hint(st + 2 * kAPart + kBPart, &tmUl, &sm->full[s], kc * KC, e + tn * UN,
+        tma_load_2d_hint(st, &tmDh, &sm->full[s], kx, rb * UM, keep_pol);
+        tma_load_2d_hint(st + kAPart, &tmDl, &sm->full[s], kx, rb * UM, keep_pol);
+        tma_load_2d_hint(st + 2 * kAPart, &tmUh, &sm->full[s], kx, e + tn * UN, keep_pol);
+        tma_load_2d_hint(st + 2 * kAPart + kBPart, &tmUl, &sm->full[s], kx, e + tn * UN,
                          keep_pol);
         ++issued;
         if (++s == kStages) {
@@ -225,10 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s = 0, lt = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x, ++lt) {
+    // one accumulator round per 128-deep K block of a tile; lt counts rounds
+    for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x)
+     for (int kb = 0; ok && kb < nkb; ++kb, ++lt) {
       const int buf = lt & 1;
       if (!mbar_wait(&sm->acc_empty[buf], ((lt >> 1) & 1) ^ 1)) {
         give_up(sm, status);
+        ok = false;
         break;
       }
       tc_fence_after();
@@ -268,26 +273,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;        // tile row = TMEM lane
-    int lt = 0, hw = 0;
+    int lt = 0, ht = 0;   // lt: accumulator rounds, ht: tiles (W~ halves 2 ht, 2 ht + 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !__any_sync(0xffffffffu, aborted(sm));
-         t += gridDim.x, ++lt) {
-      const int rb = t % n_rb, tn = t / n_rb;
+         t += gridDim.x, ++ht)
+     for (int kb = 0; ok && kb < nkb; ++kb, ++lt) {
       const int buf = lt & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm->acc_full[buf], (lt >> 1) & 1))) {
         give_up(sm, status);
+        ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + buf * kBufCols;
-      for (int h = 0; h < 2; ++h, ++hw) {
-        const int wb = hw % kWBufs;
+      for (int h = 0; h < 2; ++h) {
+        const int hw = 2 * ht + h, wb = hw % kWBufs;
         const uint32_t wpar = (hw / kWBufs) & 1;
         float m0[32], m1[32], cr[32];
         tmem_ld32(ta + h * 32, m0);
         tmem_ld32(ta + UN + h * 32, m1);
         tmem_ld32(ta + 2 * UN + h * 32, cr);
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm->w_full[wb], wpar))) {
+        if (kb == 0 && !__all_sync(0xffffffffu, mbar_wait(&sm->w_full[wb], wpar))) {
           give_up(sm, status);
           ok = false;
           break;
@@ -305,15 +311,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             *w = x;
           }
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&sm->w_written[wb]);
+        if (kb == nkb - 1) {   // the tile's last K block: hand the half to the store
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(&sm->w_written[wb]);
+        }
       }
       tc_fence_before();
       mbar_arrive(&sm->acc_empty[buf]);
     }
   } else if (warp == 6 && lane == 0) {
     // ------------------------------------------------------------ store
-    const uint64_t stream_pol = policy_evict_first();
+    const uint64_t w_pol = keep_w ? policy_evict_last() : policy_evict_first();
     int hw = 0, prev = -1;
     for (int t = blockIdx.x; t < n_tiles && !aborted(sm); t += gridDim.x) {
       const int rb = t % n_rb, tn = t / n_rb;
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int qb = 0; qb < 2; ++qb)
           tma_store_2d(&tmW, Wbuf + wb * kWHalf + qb * kWBox, e + tn * UN + h * 32 + qb * WBOX,
-                       rb * UM, stream_pol);
+                       rb * UM, w_pol);
         bulk_commit();
         bulk_wait_read_all_but_one();   // the previous half's store has read its buffer
         if (prev >= 0) mbar_arrive(&sm->w_empty[prev]);
@@ -348,15 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
-                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in) {
+                      const float* Ul, const double* Wt, int64_t d_out, int64_t d_in,
+                      int64_t kcols) {
   const uint64_t dw[2] = {(uint64_t)d_in, (uint64_t)d_out};
   const uint64_t sw[1] = {(uint64_t)d_in * 8};
   const uint32_t bw[2] = {(uint32_t)WBOX, (uint32_t)UM};
-  const uint64_t da[2] = {(uint64_t)UK, (uint64_t)d_out};
-  const uint64_t sa[1] = {(uint64_t)UK * 4};
+  const uint64_t da[2] = {(uint64_t)kcols, (uint64_t)d_out};
+  const uint64_t sa[1] = {(uint64_t)kcols * 4};
   const uint32_t ba[2] = {(uint32_t)KC, (uint32_t)UM};
-  const uint64_t db[2] = {(uint64_t)UK, (uint64_t)d_in};
-  const uint64_t sb[1] = {(uint64_t)UK * 4};
+  const uint64_t db[2] = {(uint64_t)kcols, (uint64_t)d_in};
+  const uint64_t sb[1] = {(uint64_t)kcols * 4};
   const uint32_t bb[2] = {(uint32_t)KC, (uint32_t)UN};
   return encode_tmap_2d(&m->Dh, Dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, da, sa, ba,
                         CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -370,12 +379,14 @@ bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const flo
                         CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int64_t d_out,
-                              int64_t d_in, int64_t e, int* status, cudaStream_t st) {
-  (void)Wt;
-  (void)ldw;   // W~ is reached through m.W
-  const int n = (int)(d_in - e);
-  if (n <= 0 || d_out <= 0) return NVFP4_OK;
+nvfp4_status launch_update_tc(const UpdateMaps& m, int64_t d_out, int64_t d_in, int64_t e,
+                              int64_t e_end, int kofs, int nkb, bool keep_w, int* status,
+                              cudaStream_t st) {
+  const int n = (int)(e_end - e);
+  if (n <= 0 || d_out <= 0 || nkb <= 0) return NVFP4_OK;
+  // a tile may not reach past e_end unless e_end is the last column (the
+  // tensor map clips there): tiles are UN columns wide
+  if (e_end < d_in && n % UN != 0) return NVFP4_ERR_INVALID_ARG;
   const int n_rb = (int)((d_out + UM - 1) / UM);
   const int n_tiles = n_rb * ((n + UN - 1) / UN);
   const int sms = num_sms();
@@ -383,7 +394,7 @@ nvfp4_status launch_update_tc(const UpdateMaps& m, double* Wt, int64_t ldw, int6
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   NVFP4_CUDA_TRY(launch_chained(update_tc_kernel, dim3(n_tiles < sms ? n_tiles : sms),
                                 dim3(kThreads), kSmem, st, m.Dh, m.Dl, m.Uh, m.Ul, m.W, (int)e,
-                                n_rb, n_tiles, status));
+                                n_rb, n_tiles, kofs, nkb, keep_w ? 1 : 0, status));
   count_launches(1);
   return NVFP4_OK;
 }
