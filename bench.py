@@ -32,6 +32,8 @@ DEFAULT_WORKLOAD = "attn_massive_4096x4096"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 N_SM = 148
+N_PHASES = 8                # the library's profiling phases (nvfp4pw.h)
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor rates
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
 FP32_LANES_PER_SM = 128
 
@@ -122,16 +124,16 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def phase_work(d_out, d_in, n_tok):
     """Algorithmic work per phase of one step (flops or bytes)."""
-    upd_bytes = 0
+    upd_flops = 0
     for c0 in range(0, d_in, 128):
         e = min(c0 + 128, d_in)
-        # fp64 W~[:, e:] read and written once per lazy batch
-        upd_bytes += 16 * d_out * (d_in - e)
+        # W~[:, e:] -= Delta (d_out x 128) U[batch, e:]
+        upd_flops += 2 * d_out * (e - c0) * (d_in - e)
     nb = d_in // 16
     return {
         "hessian_flops": n_tok * d_in * (d_in + 1),          # symmetric half, 2 flops per MAC
         "prepare_flops": 2 * d_in ** 3 // 3,                  # Cholesky 1/3 d^3 + trtri 1/3 d^3
-        "update_bytes": upd_bytes,
+        "update_flops": upd_flops,
         # fp64 flops of the Schur Replay per weight: 16 candidates x (scale,
         # residual, delta, score: 6 flops + 7.5 in-block update FMAs) plus the
         # in-batch update (3.5 later blocks of 16 columns on average)
@@ -211,9 +213,11 @@ def run_ours(args, rank, world, local_rank):
         flush.fill_(i & 0xFF)
         step()
     torch.cuda.synchronize()
-    ms_ph = (ctypes.c_double * 6)()
-    ln_ph = (ctypes.c_longlong * 6)()
-    B.lib().nvfp4_profile_end(ms_ph, ln_ph, 6)
+    ms_ph = (ctypes.c_double * N_PHASES)()
+    ln_ph = (ctypes.c_longlong * N_PHASES)()
+    wk_ph = (ctypes.c_double * N_PHASES)()
+    B.lib().nvfp4_profile_end(ms_ph, ln_ph, N_PHASES)
+    B.lib().nvfp4_profile_work(wk_ph, N_PHASES)
 
     # end to end through the C ABI from pinned host buffers: H2D of W and X,
     # the solve, D2H of codes, scales and the global scale
@@ -257,32 +261,41 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     peaks = load_peaks()
     wk = phase_work(d_out, d_in, n_tok)
-    names = ["hessian", "prepare", "replay", "update", "dequant", "other"]
-    ph_ms = {n: ms_ph[i] / args.steps for i, n in enumerate(names[:5])}
+    names = ["hessian", "prepare", "replay", "update", "dequant", "other", "factor_gemm",
+             "panel"]
+    ph_ms = {n: ms_ph[i] / args.steps for i, n in enumerate(names) if n != "other"}
     ph_launch = {n: ln_ph[i] // args.steps for i, n in enumerate(names)}
     sm_ghz = peaks.get("sm_max_mhz", 1965.0) / 1e3
     fp64_peak = N_SM * FP64_LANES_PER_SM * 2 * sm_ghz / 1e3    # TFLOP/s, derived
     bf16_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])   # inside a long step
+    tf32_peak = bf16_peak * TF32_PER_BF16                        # nominal dense ratio
     hbm = peaks["hbm_gbs"]
-    # per-phase roofline (what bounds each phase in this build)
+    gemm_flops = wk_ph[6] / args.steps          # counted by the launcher from the shapes
+    panel_flops = wk_ph[7] / args.steps
+    # per-kernel roofline (what bounds each kernel group in this build); the
+    # prepare phase is the panel kernels plus the fp64 GEMMs
     rl = {
         "hessian": ("tensor", wk["hessian_flops"] / (ph_ms["hessian"] * 1e9), bf16_peak,
-                    "TFLOP/s", "hessian_tc_kernel (tcgen05 kind::f16)"),
-        "prepare": ("tensor", wk["prepare_flops"] / (ph_ms["prepare"] * 1e9), fp64_peak,
-                    "TFLOP/s", "chol_panel_kernel (fp64) + dgemm_nt_kernel (fp64 mma.sync)"),
-        "update": ("hbm", wk["update_bytes"] / (ph_ms["update"] * 1e6), hbm, "GB/s",
-                   "update_tc_kernel (tcgen05 3xTF32, fp64 W~ read-modify-write)"),
+                    "TFLOP/s", "hessian_tc_kernel (tcgen05 kind::f16)",
+                    "measured bf16 sustained"),
+        "factor_gemm": ("tensor", gemm_flops / (ph_ms["factor_gemm"] * 1e9), fp64_peak,
+                        "TFLOP/s", "dgemm_nt_kernel (fp64 mma.sync m8n8k4, TMA-fed)",
+                        "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock"),
+        "panel": ("latency", panel_flops / (ph_ms["panel"] * 1e9), fp64_peak, "TFLOP/s",
+                  "chol_panel_kernel (serial 64-pivot chain per panel)",
+                  "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock"),
+        "update": ("tensor", 3 * wk["update_flops"] / (ph_ms["update"] * 1e9), tf32_peak,
+                   "TFLOP/s", "update_tc_kernel (tcgen05 kind::tf32, 3 products per MAC)",
+                   "measured bf16 sustained x nominal tf32/bf16 ratio"),
         "replay": ("alu", wk["replay_flops"] / (ph_ms["replay"] * 1e9), fp64_peak, "TFLOP/s",
-                   "schur_replay_batch_kernel (fp64 CUDA cores)"),
+                   "schur_replay_batch_kernel (fp64 CUDA cores)",
+                   "derived: 148 SMs x 64 fp64 lanes x 2 x max SM clock"),
         "dequant": ("hbm", wk["dequant_bytes"] / (ph_ms["dequant"] * 1e6), hbm, "GB/s",
-                    "dequant_kernel"),
+                    "dequant_kernel", "measured HBM copy"),
     }
     dom = max(rl, key=lambda n: ph_ms[n])
-    bound, ach, peak, unit, kern = rl[dom]
-    peak_src = {"hessian": "measured bf16 sustained", "dequant": "measured HBM copy",
-                "update": "measured HBM copy",
-                "prepare": "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock",
-                "replay": "derived: 148 SMs x 64 fp64 lanes x 2 x max SM clock"}
+    bound, ach, peak, unit, kern, _ = rl[dom]
+    peak_src = {n: v[5] for n, v in rl.items()}
     solve_ms = ph_ms["prepare"] + ph_ms["replay"] + ph_ms["update"]
     weights = d_out * d_in
     out = {
@@ -299,8 +312,8 @@ def run_ours(args, rank, world, local_rank):
                            "conventional_2Nd2": 2 * n_tok * d_in * d_in / (ph_ms["hessian"] * 1e9)},
         "phase_ms": ph_ms, "phase_launches": ph_launch,
         "phase_roofline": {n: {"bound": b, "achieved": a, "peak": p, "unit": u, "frac": a / p,
-                               "kernels": k_, "peak_source": peak_src[n]}
-                           for n, (b, a, p, u, k_) in rl.items()},
+                               "kernels": k_, "peak_source": src}
+                           for n, (b, a, p, u, k_, src) in rl.items()},
         "roofline": {"phase": dom, "kernel": kern, "bound": bound, "achieved": ach, "peak": peak,
                      "unit": unit, "frac": ach / peak, "traffic": None,
                      "peak_source": f"{peak_src[dom]} ({peaks['source']})"},

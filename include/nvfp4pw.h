@@ -318,7 +318,9 @@ enum {
   NVFP4_PHASE_UPDATE = 3,  /* trailing-update GEMMs of the quantize call    */
   NVFP4_PHASE_DEQUANT = 4, /* nvfp4_dequant                                 */
   NVFP4_PHASE_OTHER = 5,   /* everything else (prologues, reductions)       */
-  NVFP4_NUM_PHASES = 6
+  NVFP4_PHASE_FACTOR_GEMM = 6, /* inside PREPARE: its fp64 GEMM launches     */
+  NVFP4_PHASE_PANEL = 7,   /* inside PREPARE: its Cholesky panel launches  */
+  NVFP4_NUM_PHASES = 8
 };
 
 /* Starts a profiling window: from now on every phase above records a CUDA
@@ -327,9 +329,19 @@ nvfp4_status nvfp4_profile_begin(void);
 
 /* Ends the window: waits for the recorded events and writes, for phases
  * 0..n_phases-1, the summed device time in ms (ms[]) and the number of kernel
- * launches (launches[]).  NVFP4_OTHER's time is not measured (0).  Returns
+ * launches (launches[]; a launch counts in the innermost phase open, so the
+ * PREPARE count excludes its FACTOR_GEMM and PANEL launches while its time
+ * includes them).  NVFP4_OTHER's time is not measured (0).  Returns
  * NVFP4_ERR_CUDA if an event could not be read. */
 nvfp4_status nvfp4_profile_end(double* ms, long long* launches, int n_phases);
+
+/* Algorithmic work the launches of each phase did inside the last profiling
+ * window, counted by the launchers from their shapes: for FACTOR_GEMM the
+ * flops a triangular-aware GEMM must do (2 M N K, halved where only a
+ * triangle of C is wanted or P is triangular), for PANEL the flops of the
+ * panel's Cholesky, inverse and slice solve.  Other phases report 0.  Call
+ * after nvfp4_profile_end. */
+nvfp4_status nvfp4_profile_work(double* work, int n_phases);
 
 #ifdef __cplusplus
 }

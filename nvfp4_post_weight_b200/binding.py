@@ -73,6 +73,10 @@ def lib():
                                    vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
             "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
+            "nvfp4_launch_count": ([], ctypes.c_longlong),
+            "nvfp4_profile_begin": ([], i32),
+            "nvfp4_profile_end": ([vp, vp, i32], i32),
+            "nvfp4_profile_work": ([vp, i32], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)

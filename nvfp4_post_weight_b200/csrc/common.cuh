@@ -34,8 +34,12 @@ enum Phase {
   kPhaseUpdate = 3,
   kPhaseDequant = 4,
   kPhaseOther = 5,
-  kNumPhases = 6
+  kPhaseFactorGemm = 6,   // sub-phases of kPhasePrepare
+  kPhasePanel = 7,
+  kNumPhases = 8
 };
+// While profiling is on, adds algorithmic work (flops) to the open phase.
+void add_phase_work(double work);
 // Adds n to the library's kernel-launch counter (and to the open phase's).
 void count_launches(int n);
 // While profiling is on, records a CUDA event pair around its lifetime on

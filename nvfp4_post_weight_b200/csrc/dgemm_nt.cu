@@ -244,6 +244,15 @@ nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_
   if (((ldp | ldq) & 1) != 0 || (batch > 1 && ((strideP | strideQ) & 1) != 0) || (K % DK) != 0 ||
       ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(Q)) & 15) != 0)
     return NVFP4_ERR_INVALID_ARG;
+  ProfileScope ps(kPhaseFactorGemm, st);
+  {
+    // useful flops: only C's lower triangle when lower; a triangular P has
+    // sum over rows of its nonzero K range (M <= K: M (M + 1) / 2 products per column)
+    double f = 2.0 * M * N * K;
+    if (lower) f = 2.0 * ((double)N * (N + 1) / 2) * K;
+    if (ktri != 0 && M <= K) f = 2.0 * N * ((double)M * (M + 1) / 2 + (double)M * (K - M) * (ktri == 1));
+    add_phase_work(f * batch);
+  }
   // 128 x 128 tiles once there are enough of them to fill the GPU, else 64 x 64
   const int64_t big_tiles = (int64_t)((M + 127) / 128) * ((N + 127) / 128) * batch;
   if (big_tiles >= kNumSMs)

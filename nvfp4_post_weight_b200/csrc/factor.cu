@@ -455,9 +455,14 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
       const int kb = (int)((d - k) < NB ? (d - k) : NB);
       const int64_t m = d - k - kb;
       const int grid = 1 + (int)((m + kSlice - 1) / kSlice);
-      NVFP4_CUDA_TRY(launch_chained(chol_panel_kernel, dim3(grid), dim3(kPanelThreads),
-                                    kPanelSmem, st, L.A, d, k, kb, L.X, L.Y, L.hdr));
-      count_launches(1);
+      {
+        ProfileScope ps(kPhasePanel, st);
+        // Cholesky and inverse of the kb x kb block, and the m x kb slice solve
+        add_phase_work(2.0 * kb * kb * kb / 3.0 + (double)m * kb * kb);
+        NVFP4_CUDA_TRY(launch_chained(chol_panel_kernel, dim3(grid), dim3(kPanelThreads),
+                                      kPanelSmem, st, L.A, d, k, kb, L.X, L.Y, L.hdr));
+        count_launches(1);
+      }
       const int64_t nc = kend - (k + kb);   // columns of the outer block still to come
       if (m <= 0 || nc <= 0) continue;
       const double* L21 = L.A + (k + kb) * d + k;

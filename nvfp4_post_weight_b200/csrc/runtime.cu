@@ -26,6 +26,7 @@ std::atomic<long long> g_launches{0};
 std::atomic<long long> g_phase_launches[kNumPhases];
 std::atomic<bool> g_profiling{false};
 std::vector<Record> g_records;
+double g_phase_work[kNumPhases];
 std::vector<cudaEvent_t> g_pool;
 thread_local int t_phase = -1;
 
@@ -49,6 +50,13 @@ void count_launches(int n) {
   g_launches.fetch_add(n, std::memory_order_relaxed);
   const int p = t_phase >= 0 ? t_phase : kPhaseOther;
   g_phase_launches[p].fetch_add(n, std::memory_order_relaxed);
+}
+
+void add_phase_work(double work) {
+  if (!g_profiling.load(std::memory_order_relaxed)) return;
+  const int p = t_phase >= 0 ? t_phase : kPhaseOther;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_phase_work[p] += work;
 }
 
 ProfileScope::ProfileScope(int phase, cudaStream_t s) : slot(-1), prev_phase(t_phase), st(s) {
@@ -144,7 +152,10 @@ nvfp4_status nvfp4_profile_begin(void) {
     g_pool.push_back(r.b);
   }
   g_records.clear();
-  for (int p = 0; p < kNumPhases; ++p) g_phase_launches[p].store(0);
+  for (int p = 0; p < kNumPhases; ++p) {
+    g_phase_launches[p].store(0);
+    g_phase_work[p] = 0.0;
+  }
   g_profiling.store(true);
   return NVFP4_OK;
 }
@@ -179,6 +190,13 @@ nvfp4_status nvfp4_profile_end(double* ms, long long* launches, int n_phases) {
   }
   g_records.clear();
   return st;
+}
+
+nvfp4_status nvfp4_profile_work(double* work, int n_phases) {
+  if (n_phases < 0 || (n_phases > 0 && !work)) return NVFP4_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int p = 0; p < n_phases; ++p) work[p] = p < kNumPhases ? g_phase_work[p] : 0.0;
+  return NVFP4_OK;
 }
 
 }  // extern "C"
