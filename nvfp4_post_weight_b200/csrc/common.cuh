@@ -84,12 +84,14 @@ bool encode_tmap_nd(CUtensorMap* map, const void* base, CUtensorMapDataType dtyp
 // C: M x N, all fp32 row-major with leading dimensions ld* (multiples of 4)
 // and, for batch > 1, element strides stride* between the batch's matrices.
 // C2 (optional): C^T is also written there.  lower: only the 128 x 128 tiles
-// on or below the diagonal (M == N).  A timed-out wait sets *status.
+// on or below the diagonal (M == N).  C64 (optional, then C is not written and
+// beta must be 0): an fp64 destination, C64 += alpha P Q^T, the fp32 product
+// added in fp64.  A timed-out wait sets *status.
 nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_t ldp,
                         int64_t strideP, const float* Q, int64_t ldq, int64_t strideQ,
                         float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
                         int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
-                        cudaStream_t st);
+                        cudaStream_t st, double* C64 = nullptr);
 
 // C = beta C + alpha P Q^T in fp64 on the tensor cores (mma.sync m8n8k4; same
 // operand conventions as gemm_nt_tc; C2 = C^T needs beta == 0; lower: only

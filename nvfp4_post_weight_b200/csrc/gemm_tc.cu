@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmQ, float* __restrict__ C,
                       int64_t ldc, int64_t strideC, float* __restrict__ C2, int64_t ldc2,
                       int64_t strideC2, int M, int N, int K, float alpha, float beta,
-                      TileSpace ts, int* status) {
+                      TileSpace ts, int* status, double* __restrict__ C64) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -291,7 +291,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 32; ++k) wb[lane * kEpiPitch + k] = sum[c * 32 + k];
         __syncwarp();
         const int col = tn * GN + h * kEpiCols + c * 32 + lane;
-        if (col < N) {
+        if (C64 && col < N) {
+          // fp64 destination: C64 += alpha (P Q^T), the fp32 result added in fp64
+          double* Cd = C64 + b * strideC;
+#pragma unroll
+          for (int r0 = 0; r0 < 32; r0 += 16) {
+            double old[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr)
+              old[rr] = (row0 + r0 + rr < M) ? Cd[(int64_t)(row0 + r0 + rr) * ldc + col] : 0.0;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr)
+              if (row0 + r0 + rr < M)
+                Cd[(int64_t)(row0 + r0 + rr) * ldc + col] =
+                    old[rr] + (double)(alpha * wb[(r0 + rr) * kEpiPitch + lane]);
+          }
+        } else if (col < N) {
 #pragma unroll
           for (int r0 = 0; r0 < 32; r0 += 16) {
             float old[16];
@@ -344,9 +359,10 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
                         int64_t strideP, const float* Q, int64_t ldq, int64_t strideQ,
                         float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
                         int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
-                        cudaStream_t st) {
+                        cudaStream_t st, double* C64) {
   if (M <= 0 || N <= 0 || batch <= 0) return NVFP4_OK;
   if (C2 && beta != 0.f) return NVFP4_ERR_INVALID_ARG;   // the transposed copy is alpha P Q^T
+  if (C64 && (C2 || beta != 0.f)) return NVFP4_ERR_INVALID_ARG;
   if (((ldp | ldq | strideP | strideQ) & 3) != 0 ||
       ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(Q)) & 15) != 0)
     return NVFP4_ERR_INVALID_ARG;   // TMA: 16-byte aligned rows
@@ -361,7 +377,7 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_nt_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   gemm_nt_tc_kernel<<<n_tiles < sms ? n_tiles : sms, kThreads, kSmem, st>>>(
-      mp, mq, C, ldc, strideC, C2, ldc2, strideC2, M, N, K, alpha, beta, ts, status);
+      mp, mq, C, ldc, strideC, C2, ldc2, strideC2, M, N, K, alpha, beta, ts, status, C64);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;
