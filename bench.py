@@ -33,6 +33,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 N_SM = 148
 N_PHASES = 8                # the library's profiling phases (nvfp4pw.h)
+E2E_CHUNK_TOK = 1024        # tokens per host-to-device chunk of the end-to-end step
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor rates
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
 FP32_LANES_PER_SM = 128
@@ -219,17 +220,17 @@ def run_ours(args, rank, world, local_rank):
     B.lib().nvfp4_profile_end(ms_ph, ln_ph, N_PHASES)
     B.lib().nvfp4_profile_work(wk_ph, N_PHASES)
 
-    # end to end through the C ABI from pinned host buffers: H2D of W and X,
-    # the solve, D2H of codes, scales and the global scale
+    # end to end through the C ABI from pinned host buffers: the tokens stream
+    # from host memory into the Hessian in 1024-token chunks, W is copied
+    # beside the prepare, then the solve; D2H of codes, scales and s_g
     Wh, Xh = W.pin_memory(), X.pin_memory()
+    W_e2e = torch.empty_like(Wd)
     codes_h = torch.empty(solver.codes.shape, dtype=torch.uint8).pin_memory()
     scales_h = torch.empty(solver.scales.shape, dtype=torch.uint8).pin_memory()
     sg_h = torch.empty(1, dtype=torch.float32).pin_memory()
 
     def e2e_step():
-        Wd.copy_(Wh, non_blocking=True)
-        Xd.copy_(Xh, non_blocking=True)
-        step()
+        solver.step_host(Wh, Xh, W_e2e, chunk_tok=E2E_CHUNK_TOK)
         codes_h.copy_(solver.codes, non_blocking=True)
         scales_h.copy_(solver.scales, non_blocking=True)
         sg_h.copy_(solver.s_g, non_blocking=True)

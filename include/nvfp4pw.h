@@ -128,6 +128,28 @@ nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dty
                                       int64_t n_tok, int64_t d, int beta,
                                       nvfp4_stream_t stream);
 
+/* The same accumulation with the tokens in HOST memory, streamed through the
+ * device chunk by chunk ("Replay the Curvature", Abstract, infrastructure
+ * sentence: calibration activations are tiered across device, host and disk;
+ * this is the device/host tier for the Hessian).
+ * X_host    : n_tok x d host array (bf16 or fp32), page-locked for the copies
+ *             to overlap the compute (pageable memory works, without overlap).
+ *             It is read asynchronously: keep it unchanged until `stream`
+ *             has passed this call.
+ * chunk_tok : tokens per chunk (>= 1); two device staging buffers of that
+ *             many tokens live in ws.
+ * ws        : device workspace of nvfp4_hessian_host_workspace_size() bytes,
+ *             256-byte aligned.
+ * The copy of chunk c + 1 runs on a library copy stream while the Hessian of
+ * chunk c runs on `stream`; H accumulates the chunks in fp32 (beta applies to
+ * the first chunk).  Host-side errors return at once: NVFP4_ERR_INVALID_ARG,
+ * NVFP4_ERR_SHAPE (d % 16), NVFP4_ERR_WORKSPACE. */
+size_t nvfp4_hessian_host_workspace_size(int64_t d, int64_t chunk_tok, nvfp4_dtype x_dtype);
+nvfp4_status nvfp4_hessian_accumulate_host(float* H, const void* X_host, nvfp4_dtype x_dtype,
+                                           int64_t n_tok, int64_t d, int beta,
+                                           int64_t chunk_tok, void* ws, size_t ws_bytes,
+                                           nvfp4_stream_t stream);
+
 /* Synchronizes `stream` and returns, then clears, the status word of the
  * Hessian calls on the current device: NVFP4_ERR_TIMEOUT if a tensor-core
  * Hessian kernel gave up on a bounded wait since the last query, NVFP4_OK

@@ -53,6 +53,9 @@ def lib():
             "nvfp4_default_params": ([ctypes.POINTER(SolveParams)], None),
             "nvfp4_hessian_accumulate": ([vp, vp, i32, i64, i64, i32, vp], i32),
             "nvfp4_hessian_status": ([vp], i32),
+            "nvfp4_hessian_host_workspace_size": ([i64, i64, i32], sz),
+            "nvfp4_hessian_accumulate_host": ([vp, vp, i32, i64, i64, i32, i64, vp, sz, vp],
+                                              i32),
             "nvfp4_prepare_workspace_size": ([i64], sz),
             "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
@@ -136,6 +139,24 @@ def solve_params(scale_rule="schur_replay") -> SolveParams:
 
 def nvfp4_workspace_status(ws, stream=None) -> int:
     return int(lib().nvfp4_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def nvfp4_hessian_host_workspace_size(d, chunk_tok, dtype=torch.bfloat16) -> int:
+    code = NVFP4_BF16 if dtype == torch.bfloat16 else NVFP4_F32
+    return int(lib().nvfp4_hessian_host_workspace_size(int(d), int(chunk_tok), code))
+
+
+def nvfp4_hessian_accumulate_host(H, X_host, chunk_tok, ws, beta=0, stream=None):
+    """H (device) (+)= X_host^T X_host with X_host a CPU tensor (pinned for
+    overlap), streamed in chunks of chunk_tok tokens through ws."""
+    if X_host.is_cuda:
+        raise ValueError("X_host must be a host (CPU) tensor")
+    if not X_host.is_contiguous():
+        raise ValueError("X_host must be contiguous")
+    n_tok, d = X_host.shape
+    _check("nvfp4_hessian_accumulate_host", lib().nvfp4_hessian_accumulate_host(
+        _ptr(H), ctypes.c_void_p(X_host.data_ptr()), _dtype_code(X_host), n_tok, d, int(beta),
+        int(chunk_tok), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def nvfp4_hessian_accumulate(H, X, beta=0, stream=None):

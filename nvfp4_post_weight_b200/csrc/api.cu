@@ -75,6 +75,29 @@ nvfp4_status nvfp4_hessian_accumulate(float* H, const void* X, nvfp4_dtype x_dty
   return launch_hessian_simt(H, X, x_dtype, n_tok, d, beta, as_cuda(stream));
 }
 
+size_t nvfp4_hessian_host_workspace_size(int64_t d, int64_t chunk_tok, nvfp4_dtype x_dtype) {
+  if (d < 0 || chunk_tok < 1 || (x_dtype != NVFP4_BF16 && x_dtype != NVFP4_F32)) return 0;
+  return hessian_host_ws_bytes(d, chunk_tok, x_dtype);
+}
+
+nvfp4_status nvfp4_hessian_accumulate_host(float* H, const void* X_host, nvfp4_dtype x_dtype,
+                                           int64_t n_tok, int64_t d, int beta,
+                                           int64_t chunk_tok, void* ws, size_t ws_bytes,
+                                           nvfp4_stream_t stream) {
+  if (!H || n_tok < 0 || d < 0 || (n_tok > 0 && !X_host) || chunk_tok < 1)
+    return NVFP4_ERR_INVALID_ARG;
+  if (x_dtype != NVFP4_BF16 && x_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (beta != 0 && beta != 1) return NVFP4_ERR_INVALID_ARG;
+  if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (d == 0) return NVFP4_OK;
+  if (n_tok > 0 && (!ws || !aligned256(ws) ||
+                    ws_bytes < hessian_host_ws_bytes(d, chunk_tok, x_dtype)))
+    return NVFP4_ERR_WORKSPACE;
+  ProfileScope ps(kPhaseHessian, as_cuda(stream));
+  return launch_hessian_host(H, X_host, x_dtype, n_tok, d, beta, chunk_tok, ws,
+                             as_cuda(stream));
+}
+
 nvfp4_status nvfp4_hessian_status(nvfp4_stream_t stream) {
   return static_cast<nvfp4_status>(hessian_tc_take_status(as_cuda(stream)));
 }

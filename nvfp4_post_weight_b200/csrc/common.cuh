@@ -108,6 +108,10 @@ nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_
 // ---- kernel launchers implemented in the .cu files -------------------------
 bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                           int64_t d);
+size_t hessian_host_ws_bytes(int64_t d, int64_t chunk_tok, nvfp4_dtype xt);
+nvfp4_status launch_hessian_host(float* H, const void* X_host, nvfp4_dtype xt, int64_t n_tok,
+                                 int64_t d, int beta, int64_t chunk_tok, void* ws,
+                                 cudaStream_t st);
 nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
                                cudaStream_t st);
 int hessian_tc_take_status(cudaStream_t st);

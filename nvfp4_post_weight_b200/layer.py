@@ -65,6 +65,37 @@ class LayerSolver:
         if with_error:
             self.layer_error(W, stream)
 
+    def hessian_host(self, X_host, chunk_tok=1024, beta=0, stream=None):
+        """H from host-resident tokens, streamed through the device in chunks
+        (the copy of the next chunk overlaps the Hessian of the current one)."""
+        key = (int(chunk_tok), X_host.dtype)
+        if getattr(self, "_ws_host_key", None) != key:
+            self.ws_host = B.workspace(
+                B.nvfp4_hessian_host_workspace_size(self.d_in, chunk_tok, X_host.dtype),
+                self.device)
+            self._ws_host_key = key
+        B.nvfp4_hessian_accumulate_host(self.H, X_host, chunk_tok, self.ws_host, beta, stream)
+
+    def step_host(self, W_host, X_host, W_dev, chunk_tok=1024, stream=None, with_error=True):
+        """One whole solve from host-resident inputs: the tokens stream into the
+        Hessian chunk by chunk, and W is copied into W_dev on a side stream while
+        the factor is prepared (quantize waits for it)."""
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if not hasattr(self, "_side"):
+            self._side = torch.cuda.Stream(self.device)
+            self._w_ready = torch.cuda.Event()
+        self._side.wait_stream(st)          # W_dev is free once earlier work on st is done
+        with torch.cuda.stream(self._side):
+            W_dev.copy_(W_host, non_blocking=True)
+            self._w_ready.record(self._side)
+        self.hessian_host(X_host, chunk_tok, 0, st)
+        self.prepare(st)
+        st.wait_event(self._w_ready)
+        self.quantize(W_dev, st)
+        self.dequant(st)
+        if with_error:
+            self.layer_error(W_dev, st)
+
     def status(self, stream=None):
         """Device status words of the prepare and quantize workspaces."""
         return (B.nvfp4_workspace_status(self.ws_prep, stream),

@@ -54,6 +54,15 @@ def test_host_side_checks_need_no_device():
     # a workspace that is too small -> NVFP4_ERR_WORKSPACE
     assert L.nvfp4_gptq_prepare(ctypes.c_void_p(256), 32, 0.01, ctypes.c_void_p(256), null,
                                 null, ctypes.c_void_p(256), 16, null) == 3
+    # host-streamed Hessian: bad chunk size, missing workspace, shape
+    assert L.nvfp4_hessian_accumulate_host(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 100,
+                                           256, 0, 0, ctypes.c_void_p(256), 1 << 30, null) == 1
+    assert L.nvfp4_hessian_accumulate_host(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 100,
+                                           256, 0, 64, null, 0, null) == 3
+    assert L.nvfp4_hessian_accumulate_host(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 100,
+                                           250, 0, 64, ctypes.c_void_p(256), 1 << 30, null) == 2
+    assert B.nvfp4_hessian_host_workspace_size(256, 1024) == 2 * 1024 * 256 * 2
+    assert L.nvfp4_hessian_host_workspace_size(256, 0, 0) == 0
     # an unknown block-scale rule -> NVFP4_ERR_UNSUPPORTED
     bad = B.solve_params(3)
     assert L.nvfp4_gptq_schur_replay_quantize(
