@@ -243,6 +243,35 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize_noalloc(
     nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Row shards: one layer's output rows split over calls (e.g. one per GPU)   */
+/* ------------------------------------------------------------------------ */
+/* "Replay the Curvature", Abstract, infrastructure sentence: independent
+ * output rows are distributed across tensor-parallel ranks.  Given U the rows
+ * of the solve are independent; only the global scale is shared.  So each
+ * shard computes its max |W| with nvfp4_weight_amax, the shards' values are
+ * reduced with MAX (a collective of the caller's, e.g. an NCCL all-reduce),
+ * and every shard quantizes its rows with nvfp4_gptq_schur_replay_quantize_rows
+ * from that layer amax: the codes and scales of the shards then equal the
+ * whole-layer call's rows bit for bit.
+ *
+ * nvfp4_weight_amax: max |W| of a d_out x d_in block (dead columns, if given,
+ * count as 0), written to the device fp32 scalar amax_out (0 for an empty
+ * block).  Non-finite weights are not reported here (the quantize call flags
+ * them). */
+nvfp4_status nvfp4_weight_amax(const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in,
+                               const uint8_t* dead, float* amax_out, nvfp4_stream_t stream);
+
+/* As nvfp4_gptq_schur_replay_quantize for the rows W (d_out x d_in, a block
+ * of rows of a larger layer), except that the global scale is computed from
+ * the device fp32 scalar `amax` (the layer's max |W|) with the same formula,
+ * s_g = fp32(amax / 2688) (1 when amax == 0), instead of from this block. */
+nvfp4_status nvfp4_gptq_schur_replay_quantize_rows(
+    const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in, const float* U,
+    const nvfp4_solve_params* params, const uint8_t* dead, const float* amax,
+    uint8_t* codes, uint8_t* scales, float* global_scale, double* err_out, void* ws,
+    size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* a9  dequantization: Q = e2m1(code) * e4m3(scale) * s_g                    */
 /* "Replay the Curvature", Abstract (NVFP4 format).                          */
 /* ------------------------------------------------------------------------ */

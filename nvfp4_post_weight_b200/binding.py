@@ -66,6 +66,10 @@ def lib():
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
                  vp], i32),
             "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
+            "nvfp4_weight_amax": ([vp, i32, i64, i64, vp, vp, vp], i32),
+            "nvfp4_gptq_schur_replay_quantize_rows": (
+                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, vp,
+                 sz, vp], i32),
             "nvfp4_hessian_accumulate_batched": ([i32, vp, vp, i32, vp, vp, i32, vp], i32),
             "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, vp, vp], i32),
             "nvfp4_gptq_schur_replay_quantize_batched": (
@@ -191,6 +195,22 @@ def nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, global_scale, err_out=
     p = params if params is not None else default_params()
     _check("nvfp4_gptq_schur_replay_quantize", lib().nvfp4_gptq_schur_replay_quantize(
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
+        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def nvfp4_weight_amax(W, amax_out, dead=None, stream=None):
+    d_out, d_in = W.shape
+    _check("nvfp4_weight_amax", lib().nvfp4_weight_amax(
+        _ptr(W), _dtype_code(W), d_out, d_in, _ptr(dead), _ptr(amax_out), _stream(stream)))
+
+
+def nvfp4_gptq_schur_replay_quantize_rows(W, U, amax, codes, scales, global_scale, err_out=None,
+                                          dead=None, ws=None, params=None, stream=None):
+    d_out, d_in = W.shape
+    p = params if params is not None else default_params()
+    _check("nvfp4_gptq_schur_replay_quantize_rows", lib().nvfp4_gptq_schur_replay_quantize_rows(
+        _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead), _ptr(amax),
         _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
 

@@ -142,6 +142,34 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
                          err_out, ws, as_cuda(stream));
 }
 
+nvfp4_status nvfp4_weight_amax(const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in,
+                               const uint8_t* dead, float* amax_out, nvfp4_stream_t stream) {
+  if (d_out < 0 || d_in < 0 || !amax_out || (d_out > 0 && d_in > 0 && !W))
+    return NVFP4_ERR_INVALID_ARG;
+  if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(amax_out, 4)) return NVFP4_ERR_INVALID_ARG;
+  return launch_weight_amax(W, w_dtype, d_out, d_in, dead, amax_out, as_cuda(stream));
+}
+
+nvfp4_status nvfp4_gptq_schur_replay_quantize_rows(
+    const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in, const float* U,
+    const nvfp4_solve_params* params, const uint8_t* dead, const float* amax,
+    uint8_t* codes, uint8_t* scales, float* global_scale, double* err_out, void* ws,
+    size_t ws_bytes, nvfp4_stream_t stream) {
+  if (!amax) return NVFP4_ERR_INVALID_ARG;
+  if (d_out < 0 || d_in < 0 || !global_scale) return NVFP4_ERR_INVALID_ARG;
+  if (d_out > 0 && d_in > 0 && (!W || !U || !codes || !scales)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 8)) return NVFP4_ERR_INVALID_ARG;
+  if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!params_ok(params)) return NVFP4_ERR_UNSUPPORTED;
+  if (d_in % 16 || d_in > kMaxDim || d_out > kMaxRows) return NVFP4_ERR_SHAPE;
+  if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(d_out, d_in))
+    return NVFP4_ERR_WORKSPACE;
+  const int rule = params ? params->scale_rule : NVFP4_RULE_SCHUR_REPLAY;
+  return launch_quantize(W, w_dtype, d_out, d_in, U, dead, rule, codes, scales, global_scale,
+                         err_out, ws, as_cuda(stream), amax);
+}
+
 nvfp4_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales,
                            const float* global_scale, int64_t d_out, int64_t d_in, void* out,
                            nvfp4_dtype out_dtype, nvfp4_stream_t stream) {

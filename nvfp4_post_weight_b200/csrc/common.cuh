@@ -141,7 +141,9 @@ size_t prepare_ws_bytes(int64_t d);
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
                              const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
-                             cudaStream_t st);
+                             cudaStream_t st, const float* amax_in = nullptr);
+nvfp4_status launch_weight_amax(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
+                                const uint8_t* dead, float* amax, cudaStream_t st);
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in);
 nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* sg,
                             int64_t d_out, int64_t d_in, void* out, nvfp4_dtype ot,

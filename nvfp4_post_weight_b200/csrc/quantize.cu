@@ -136,10 +136,34 @@ __global__ void wprep_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_i
   if ((threadIdx.x & 31) == 0) atomicMax(&hdr->amax_bits, __float_as_uint(m));
 }
 
-// s_g = amax / (6 * 448) correctly rounded to fp32, 1 when W == 0.
-__global__ void global_scale_kernel(QuantHeader* hdr, float* __restrict__ sg) {
-  const float amax = __uint_as_float(hdr->amax_bits);
+// s_g = amax / (6 * 448) correctly rounded to fp32, 1 when W == 0; amax is
+// this call's own max |W~| unless the caller gives the layer's (row shards).
+__global__ void global_scale_kernel(QuantHeader* hdr, const float* __restrict__ amax_in,
+                                    float* __restrict__ sg) {
+  const float amax = amax_in ? *amax_in : __uint_as_float(hdr->amax_bits);
   *sg = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// max |W| (dead columns as 0) into *amax_bits (fp32 bits; non-negative floats
+// order as unsigned integers), which the caller zeroed.
+template <typename T>
+__global__ void weight_amax_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_in,
+                                   const uint8_t* __restrict__ dead,
+                                   unsigned* __restrict__ amax_bits) {
+  const int64_t n = d_out * d_in;
+  float m = 0.f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float v;
+    if constexpr (sizeof(T) == 2)
+      v = __uint_as_float((uint32_t)W[i] << 16);
+    else
+      v = W[i];
+    if (dead && dead[i % d_in]) v = 0.f;
+    m = fmaxf(m, fabsf(v));
+  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
 }
 
 constexpr int kReplayThreads = 256;                 // 8 warps = 16 rows in flight
@@ -430,14 +454,31 @@ size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
          align256(sizeof(double) * d_out);
 }
 
+nvfp4_status launch_weight_amax(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
+                                const uint8_t* dead, float* amax, cudaStream_t st) {
+  NVFP4_CUDA_TRY(cudaMemsetAsync(amax, 0, sizeof(float), st));
+  if (d_out == 0 || d_in == 0) return NVFP4_OK;
+  const int g = grid_for(d_out * d_in, 256);
+  unsigned* bits = reinterpret_cast<unsigned*>(amax);
+  if (wt == NVFP4_BF16)
+    weight_amax_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), d_out,
+                                                    d_in, dead, bits);
+  else
+    weight_amax_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), d_out, d_in,
+                                                 dead, bits);
+  NVFP4_LAUNCH_CHECK();
+  count_launches(1);
+  return NVFP4_OK;
+}
+
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
                              const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
-                             cudaStream_t st) {
+                             cudaStream_t st, const float* amax_in) {
   QuantLayout L = quant_layout(ws, d_out, d_in);
   NVFP4_CUDA_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(QuantHeader), st));
   if (d_out == 0 || d_in == 0) {
-    global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, sg);
+    global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, amax_in, sg);
     NVFP4_LAUNCH_CHECK();
     count_launches(1);
     if (err) NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
@@ -451,7 +492,7 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
     wprep_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), d_out, d_in, dead,
                                            L.Wt, L.rowerr, L.hdr);
   NVFP4_LAUNCH_CHECK();
-  global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, sg);
+  global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, amax_in, sg);
   NVFP4_LAUNCH_CHECK();
   count_launches(2);
 
