@@ -284,6 +284,24 @@ nvfp4_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales,
                            void* out, nvfp4_dtype out_dtype, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Export to the block-scaled FP4 GEMM operand layout                         */
+/* ------------------------------------------------------------------------ */
+/* "Replay the Curvature", Abstract, infrastructure sentence: each layer is
+ * exported before its full-precision weights are retired.  The codes already
+ * have the K-major data layout of an FP4 GEMM operand (two E2M1 nibbles per
+ * byte, low nibble = even column); the E4M3 block scales are re-tiled here
+ * into the layout in which block-scaled tensor-core GEMMs read the scale
+ * operand of 16-element FP4 blocks: rows and scale columns padded (code 0) to
+ * multiples of 128 and 4, tiles of 128 rows x 4 scale columns stored as 512
+ * contiguous bytes in row-major tile order, and inside a tile the scale of row
+ * r, column c at byte (r % 32) * 16 + (r / 32) * 4 + c.  The global scale s_g
+ * is the GEMM's output scale.
+ * out: device buffer of nvfp4_export_scales_size(d_out, d_in) bytes. */
+size_t nvfp4_export_scales_size(int64_t d_out, int64_t d_in);
+nvfp4_status nvfp4_export_scales(const uint8_t* scales, int64_t d_out, int64_t d_in,
+                                 uint8_t* out, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* a10  layer error tr((W - Q) H (W - Q)^T) (measurement)                   */
 /* ------------------------------------------------------------------------ */
 size_t nvfp4_layer_error_workspace_size(int64_t d_out, int64_t d_in);

@@ -67,6 +67,8 @@ def lib():
                  vp], i32),
             "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
             "nvfp4_weight_amax": ([vp, i32, i64, i64, vp, vp, vp], i32),
+            "nvfp4_export_scales_size": ([i64, i64], sz),
+            "nvfp4_export_scales": ([vp, i64, i64, vp, vp], i32),
             "nvfp4_gptq_schur_replay_quantize_rows": (
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, vp,
                  sz, vp], i32),
@@ -197,6 +199,18 @@ def nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, global_scale, err_out=
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
         _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def nvfp4_export_scales_size(d_out, d_in) -> int:
+    return int(lib().nvfp4_export_scales_size(int(d_out), int(d_in)))
+
+
+def nvfp4_export_scales(scales, out, stream=None):
+    """scales: (d_out, d_in/16) uint8 device tensor -> out (flat uint8 device
+    tensor of nvfp4_export_scales_size bytes) in the 128 x 4 tiled layout."""
+    d_out, nb = scales.shape
+    _check("nvfp4_export_scales", lib().nvfp4_export_scales(
+        _ptr(scales), d_out, nb * 16, _ptr(out), _stream(stream)))
 
 
 def nvfp4_weight_amax(W, amax_out, dead=None, stream=None):

@@ -142,6 +142,19 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
                          err_out, ws, as_cuda(stream));
 }
 
+size_t nvfp4_export_scales_size(int64_t d_out, int64_t d_in) {
+  if (d_out < 0 || d_in < 0 || d_in % 16) return 0;
+  return scales_tiled_bytes(d_out, d_in);
+}
+
+nvfp4_status nvfp4_export_scales(const uint8_t* scales, int64_t d_out, int64_t d_in,
+                                 uint8_t* out, nvfp4_stream_t stream) {
+  if (d_out < 0 || d_in < 0) return NVFP4_ERR_INVALID_ARG;
+  if (d_in % 16) return NVFP4_ERR_SHAPE;
+  if (d_out > 0 && d_in > 0 && (!scales || !out)) return NVFP4_ERR_INVALID_ARG;
+  return launch_scales_tiled(scales, d_out, d_in, out, as_cuda(stream));
+}
+
 nvfp4_status nvfp4_weight_amax(const void* W, nvfp4_dtype w_dtype, int64_t d_out, int64_t d_in,
                                const uint8_t* dead, float* amax_out, nvfp4_stream_t stream) {
   if (d_out < 0 || d_in < 0 || !amax_out || (d_out > 0 && d_in > 0 && !W))

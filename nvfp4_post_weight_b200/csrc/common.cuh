@@ -142,6 +142,9 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
                              const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
                              cudaStream_t st, const float* amax_in = nullptr);
+size_t scales_tiled_bytes(int64_t rows, int64_t d_in);
+nvfp4_status launch_scales_tiled(const uint8_t* scales, int64_t rows, int64_t d_in,
+                                 uint8_t* out, cudaStream_t st);
 nvfp4_status launch_weight_amax(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
                                 const uint8_t* dead, float* amax, cudaStream_t st);
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in);

@@ -132,6 +132,23 @@ __global__ void sum_partials_kernel(const double* __restrict__ p, int n, double*
   }
 }
 
+// Export of the block scales into 128-row x 4-column tiles of 512 bytes (the
+// scale-operand layout of block-scaled tensor-core FP4 GEMMs): one thread per
+// output byte, so the writes are coalesced; padding rows and columns get code 0.
+__global__ void scales_tiled_kernel(const uint8_t* __restrict__ scales, int64_t rows,
+                                    int64_t nb, int64_t n_ct, int64_t total,
+                                    uint8_t* __restrict__ out) {
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < total;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tile = o >> 9;
+    const int in = (int)(o & 511);
+    const int a = in >> 4, b = (in >> 2) & 3, c = in & 3;   // byte 16 a + 4 b + c
+    const int64_t r = (tile / n_ct) * 128 + 32 * b + a;
+    const int64_t col = (tile % n_ct) * 4 + c;
+    out[o] = (r < rows && col < nb) ? scales[r * nb + col] : (uint8_t)0;
+  }
+}
+
 int grid_for(int64_t n, int threads) {
   int64_t b = (n + threads - 1) / threads;
   return (int)(b < 8 * kNumSMs ? (b < 1 ? 1 : b) : 8 * kNumSMs);
@@ -156,6 +173,23 @@ nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const f
 }
 
 int64_t et_ld(int64_t d_out) { return (d_out + 31) / 32 * 32; }
+
+size_t scales_tiled_bytes(int64_t rows, int64_t d_in) {
+  const int64_t nb = d_in / kBlock;
+  return (size_t)((rows + 127) / 128 * 128) * (size_t)((nb + 3) / 4 * 4);
+}
+
+nvfp4_status launch_scales_tiled(const uint8_t* scales, int64_t rows, int64_t d_in,
+                                 uint8_t* out, cudaStream_t st) {
+  const int64_t nb = d_in / kBlock;
+  const int64_t total = (int64_t)scales_tiled_bytes(rows, d_in);
+  if (total == 0) return NVFP4_OK;
+  scales_tiled_kernel<<<grid_for(total, 256), 256, 0, st>>>(scales, rows, nb, (nb + 3) / 4,
+                                                           total, out);
+  NVFP4_LAUNCH_CHECK();
+  count_launches(1);
+  return NVFP4_OK;
+}
 
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in) {
   return kWsHeader + align256(sizeof(float) * et_ld(d_out) * d_in) +

@@ -44,6 +44,14 @@ scale.  The readings taken where it is silent are marked READING below:
               factor GPTQ updates with; no column reordering.
   READING R9  H = X^T X with no 1/N or factor 2 (codes are invariant to a
               scale of H because lambda scales with it).
+  READING R14 export: the codes keep their row-major packed layout (two
+              E2M1 nibbles per byte, low nibble = even column), which is the
+              K-major data layout of an FP4 GEMM operand; the E4M3 block
+              scales are re-tiled into the 128-row x 4-column, 512-byte tiles
+              in which block-scaled tensor-core GEMMs read their scale operand
+              (the public cuBLAS/CUTLASS layout for 16-element-block FP4
+              operands); s_g becomes the GEMM's output scale.  The page only
+              says that layers are exported.
   READING R10 the rules Schur Replay is set against (Abstract, sentence on
               why scale choice is hard: a block evaluated on its own can
               misestimate its final error) are taken as two independent-block
@@ -361,6 +369,38 @@ def dequant(codes, scales, s_g, out_dtype=np.float32):
     if out_dtype == "bf16":
         return round_to_bf16(exact)
     raise ValueError(out_dtype)
+
+
+# --------------------------------------------------------------------------
+# Export layout (Abstract, infrastructure sentence: layers are exported before
+# their full-precision weights are retired)
+# --------------------------------------------------------------------------
+
+SF_TILE_ROWS, SF_TILE_COLS = 128, 4   # one 512-byte tile of block scales
+
+
+def scales_to_tiled(scales):
+    """The block scales (rows x nb E4M3 codes, nb = d_in / 16) in the tiled
+    layout that block-scaled tensor-core GEMMs read their scale operand in
+    (READING R14): rows and scale columns padded with zero codes to multiples
+    of 128 and 4; tile (R, C) of 128 rows x 4 scale columns is 512 contiguous
+    bytes, tiles in row-major order over (R, C); inside a tile, the scale of
+    row r and column c sits at byte (r % 32) * 16 + (r // 32) * 4 + c.
+    Returns a flat uint8 array."""
+    scales = np.asarray(scales, dtype=np.uint8)
+    rows, nb = scales.shape
+    rp = -(-rows // SF_TILE_ROWS) * SF_TILE_ROWS
+    cp = -(-nb // SF_TILE_COLS) * SF_TILE_COLS
+    padded = np.zeros((rp, cp), dtype=np.uint8)
+    padded[:rows, :nb] = scales
+    out = np.zeros(rp * cp, dtype=np.uint8)
+    n_ct = cp // SF_TILE_COLS
+    for r in range(rp):
+        for c in range(cp):
+            tile = (r // SF_TILE_ROWS) * n_ct + c // SF_TILE_COLS
+            rr, cc = r % SF_TILE_ROWS, c % SF_TILE_COLS
+            out[tile * 512 + (rr % 32) * 16 + (rr // 32) * 4 + cc] = padded[r, c]
+    return out
 
 
 def round_to_bf16(x):

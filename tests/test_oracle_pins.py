@@ -458,3 +458,40 @@ def test_amax_rule_margin_is_distance_to_e4m3_midpoint():
     assert m[2] == pytest.approx(0.03125 / 1.03125)
     assert m[3] == pytest.approx(16.0 / 448.0)       # 416 and 448: midpoint 432
     assert m[5] == np.inf
+
+
+# --------------------------------------------------------------------------
+# export layout of the block scales (128 x 4 tiles of 512 bytes)
+# --------------------------------------------------------------------------
+
+def _tiled_by_reshape(scales):
+    """The same tiling by reshapes: row r = 128 R + 32 b + a, column
+    c4 = 4 C + c goes to tile (R, C), byte 16 a + 4 b + c."""
+    rows, nb = scales.shape
+    rp, cp = -(-rows // 128) * 128, -(-nb // 4) * 4
+    p = np.zeros((rp, cp), dtype=np.uint8)
+    p[:rows, :nb] = scales
+    t = p.reshape(rp // 128, 4, 32, cp // 4, 4)        # (R, b, a, C, c)
+    return t.transpose(0, 3, 2, 1, 4).reshape(-1)       # (R, C, a, b, c)
+
+
+@pytest.mark.parametrize("rows,nb", [(1, 1), (7, 3), (128, 4), (200, 6), (300, 17)])
+def test_export_tiling_matches_reshape_route_and_inverts(rows, nb):
+    rng = np.random.default_rng(rows * 31 + nb)
+    sc = rng.integers(1, 127, size=(rows, nb)).astype(np.uint8)
+    t = O.scales_to_tiled(sc)
+    np.testing.assert_array_equal(t, _tiled_by_reshape(sc))
+    assert t.size == (-(-rows // 128) * 128) * (-(-nb // 4) * 4)
+    assert np.count_nonzero(t) == rows * nb                # padding is zero codes
+    assert sorted(t[t > 0].tolist()) == sorted(sc.reshape(-1).tolist())
+
+
+def test_export_tiling_hand_position():
+    sc = np.zeros((200, 6), dtype=np.uint8)
+    sc[33, 5] = 77                     # tile (0, 1); r % 32 = 1, r // 32 = 1, c % 4 = 1
+    t = O.scales_to_tiled(sc)
+    assert np.nonzero(t)[0].tolist() == [512 + 16 + 4 + 1]
+    sc = np.zeros((200, 6), dtype=np.uint8)
+    sc[130, 2] = 9                     # tile (1, 0) of a 2 x 2 grid = third tile
+    t = O.scales_to_tiled(sc)
+    assert np.nonzero(t)[0].tolist() == [2 * 512 + 2 * 16 + 0 * 4 + 2]
