@@ -99,6 +99,17 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
 // lower triangular -- the zero part of K is skipped).  P and Q go through TMA:
 // 16-byte aligned, even leading dimensions and batch strides, K a multiple of
 // 16.  A wait that runs out records NVFP4_ERR_TIMEOUT in *status.
+// The same product as dgemm_nt, fp64-accurate through int8 slices on tcgen05
+// (kind::i8): P and Q cut into 7 power-of-two-scaled 7-bit slices per row,
+// slice products exact in int32 TMEM, levels combined in fp64.  scratch holds
+// the slices: dgemm_i8_scratch_bytes(M, N, K, batch) bytes.  K < 65536, K a
+// multiple of 16.  A wait that runs out records NVFP4_ERR_TIMEOUT in *status.
+size_t dgemm_i8_scratch_bytes(int64_t M, int64_t N, int64_t K, int batch);
+nvfp4_status dgemm_i8(int M, int N, int K, double alpha, const double* P, int64_t ldp,
+                      int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
+                      double beta, double* C, int64_t ldc, int64_t strideC, double* C2,
+                      int64_t ldc2, int64_t strideC2, int batch, int lower, int ktri,
+                      void* scratch, size_t scratch_bytes, int* status, cudaStream_t st);
 nvfp4_status dgemm_nt(int M, int N, int K, double alpha, const double* P, int64_t ldp,
                       int64_t strideP, const double* Q, int64_t ldq, int64_t strideQ,
                       double beta, double* C, int64_t ldc, int64_t strideC, double* C2,

@@ -397,7 +397,14 @@ struct PrepLayout {
   double* X;   // L^-1 (lower)
   double* Y;   // L^-T (upper)
   double* T;   // scratch of the inverse doubling
+  void* S8;    // int8 slices of the tensor-core fp64 GEMMs
+  size_t s8_bytes;
 };
+
+// Slice scratch of the int8-slice GEMMs: the largest operand pair of a call
+// (trailing update: d x 256 twice; doubling level b: d/2b pairs of b x b,
+// twice) is below the bound for M = N = d, K = d/2.
+size_t slice_scratch_bytes(int64_t d) { return dgemm_i8_scratch_bytes(d, d, (d / 2 + 15) / 16 * 16 + 256, 1); }
 
 PrepLayout prep_layout(void* ws, int64_t d) {
   char* p = static_cast<char*>(ws);
@@ -411,6 +418,9 @@ PrepLayout prep_layout(void* ws, int64_t d) {
   L.Y = reinterpret_cast<double*>(p + off);
   off += align256(sizeof(double) * d * d);
   L.T = reinterpret_cast<double*>(p + off);
+  off += align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB));
+  L.S8 = p + off;
+  L.s8_bytes = slice_scratch_bytes(d);
   return L;
 }
 
@@ -423,7 +433,8 @@ int grid_for(int64_t n, int threads) {
 
 size_t prepare_ws_bytes(int64_t d) {
   return kWsHeader + 3 * align256(sizeof(double) * d * d) +
-         align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB));
+         align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB)) +
+         align256(slice_scratch_bytes(d));
 }
 
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uint8_t* dead,
@@ -446,6 +457,20 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   // block, A22 -= L21 L21^T with K = 256, which reads and writes it 4x less
   // often than per-panel updates would.
   constexpr int64_t OB = 4 * NB;
+  // the large products (trailing updates of at least 512 rows, doubling
+  // levels from 256) go to the int8-slice tensor-core engine, the small and
+  // narrow ones to mma.sync fp64, whose latency is lower
+  constexpr int64_t kBigGemm = 512;
+  auto gemm = [&](bool big, int M, int N, int K, double alpha, const double* P, int64_t ldp,
+                  int64_t sP, const double* Q, int64_t ldq, int64_t sQ, double beta, double* C,
+                  int64_t ldc, int64_t sC, double* C2, int64_t ldc2, int64_t sC2, int batch,
+                  int lower, int ktri) {
+    if (big && K < (1 << 16))
+      return dgemm_i8(M, N, K, alpha, P, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2,
+                      batch, lower, ktri, L.S8, L.s8_bytes, &L.hdr->status, st);
+    return dgemm_nt(M, N, K, alpha, P, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2, batch,
+                    lower, ktri, &L.hdr->status, st);
+  };
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(chol_panel_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kPanelSmem));
@@ -473,8 +498,8 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
     const int64_t m2 = d - kend;
     if (m2 > 0) {
       const double* Lb = L.A + kend * d + k0;
-      nvfp4_status s = dgemm_nt((int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, 0, Lb, d, 0,
-                                1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0, &L.hdr->status, st);
+      nvfp4_status s = gemm(m2 >= kBigGemm, (int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, 0,
+                            Lb, d, 0, 1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0);
       if (s != NVFP4_OK) return s;
     }
   }
@@ -486,25 +511,25 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   for (int64_t b = NB; b < d; b *= 2) {
     const int64_t npairs = d / (2 * b);
     const int64_t stride = 2 * b * (d + 1);
+    const bool big = b >= kBigGemm / 2;
     if (npairs > 0) {
-      nvfp4_status s = dgemm_nt((int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
-                                  stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1, &L.hdr->status, st);
+      nvfp4_status s = gemm(big, (int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
+                            stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1);
       if (s != NVFP4_OK) return s;
-      s = dgemm_nt((int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
-                     0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, 2,
-                     &L.hdr->status, st);
+      s = gemm(big, (int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
+               0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, 2);
       if (s != NVFP4_OK) return s;
     }
     const int64_t r0 = npairs * 2 * b;   // a ragged pair: full left block, rr rows right
     const int64_t rr = d - r0 - b;
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
-      nvfp4_status s = dgemm_nt((int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0,
-                                  L.A + o + b * d, d, 0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1, &L.hdr->status, st);
+      nvfp4_status s = gemm(big, (int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0, L.A + o + b * d, d,
+                            0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1);
       if (s != NVFP4_OK) return s;
       // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
-      s = dgemm_nt((int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
-                     0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2, &L.hdr->status, st);
+      s = gemm(big, (int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
+               0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2);
       if (s != NVFP4_OK) return s;
     }
   }
