@@ -19,13 +19,25 @@
 // the fp32 factor U keeps after the condition number of the damped Hessian
 // amplifies it.  The levels are combined in fp64 in the epilogue.
 //
-// Pipeline per 128 x 64 output tile, K in 64-byte chunks (SWIZZLE_64B, all S
-// slices of a chunk in one 3-D TMA load per operand):
-//   warp 0     TMA producer (2-stage ring of A and B slices)
-//   warp 1     MMA issuer: S (S + 1) / 2 slice pairs x 2 K-steps of 32 per chunk
-//   warps 2-5  epilogue: TMEM -> registers, levels summed in fp64, scaled by
-//              the row and column exponents, C written (beta, C2, alpha).
-// Every wait is bounded; a wait that runs out records NVFP4_ERR_TIMEOUT.
+// Persistent kernel, one CTA per SM, 128 x 64 output tiles:
+//   warp 0     TMA producer: a 3-stage ring, each stage 32 K-bytes of all S
+//              slices of A (128 rows) and B (64 rows), one 3-D load per
+//              operand (SWIZZLE_32B: one MMA's K per row)
+//   warp 1     MMA issuer.  The B slices of a stage lie one after another and
+//              so do the S level accumulators in TMEM (64 columns each), so
+//              A_t times the stacked B_0 .. B_{S-1-t} adds A_t B_u^T to level
+//              t + u for all u in one MMA of N = 64 (S - t) (cut at 256): 10
+//              MMAs per K step instead of S (S + 1) / 2 = 28 narrow ones
+//   warps 2-5  epilogue: levels summed in fp64 straight out of TMEM, TMEM
+//              handed back (the next tile's MMAs start), then the tile is
+//              scaled by the row and column exponents and written through a
+//              shared-memory staging tile (C coalesced by rows, C2 = C^T by
+//              columns) while the tensor cores work on the next tile.
+// Tiles are ordered so that the work per tile never grows along the order
+// (triangular P: longest K ranges first) and dealt to the CTAs in rounds,
+// every other round backwards.  Every wait is bounded; a wait that runs out
+// records NVFP4_ERR_TIMEOUT and the CTA drains its copies and MMAs and frees
+// TMEM before it returns.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -38,17 +50,19 @@ using namespace sm100;
 
 constexpr int S = 7;                     // slices per value
 constexpr int IM = 128, IN = 64;         // output tile
-constexpr int KC = 64;                   // K bytes (int8 values) per stage
-constexpr int kIStages = 2;
-constexpr uint32_t kASlice = IM * KC;    // 8 KB
-constexpr uint32_t kBSlice = IN * KC;    // 4 KB
-constexpr uint32_t kIStage = S * (kASlice + kBSlice);   // 84 KB
+constexpr int KC = 32;                   // K bytes (int8 values) per stage: one MMA's K
+constexpr int kIStages = 3;
+constexpr uint32_t kASlice = IM * KC;    // 4 KB
+constexpr uint32_t kBSlice = IN * KC;    // 2 KB
+constexpr uint32_t kIStage = S * (kASlice + kBSlice);   // 42 KB
 constexpr int kIThreads = 192;
 constexpr uint32_t kITmemCols = 512;     // S levels x IN columns = 448
-constexpr size_t kISmem = kIStages * kIStage + 1024 + 256;
+constexpr int kTilePitch = IN + 1;       // staged fp64 result tile, IM x kTilePitch
+constexpr size_t kITileBytes = sizeof(double) * IM * kTilePitch;
+constexpr size_t kISmem = kIStages * kIStage + kITileBytes + 1024 + 256;
 
 struct IBars {
-  uint64_t full[kIStages], empty[kIStages], done;
+  uint64_t full[kIStages], empty[kIStages], acc_full, acc_empty, done;
   uint32_t tmem;
   int abort;
 };
@@ -62,16 +76,30 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// K-major operand in the canonical 64-byte-swizzled layout: rows of 64 bytes,
-// 8-row groups 512 bytes apart.
-__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
+// K-major operand in the canonical 32-byte-swizzled layout: rows of 32 bytes
+// (one MMA's K), 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw32(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
   d |= (uint64_t)1 << 16;             // leading byte offset (unused when K fits a row)
-  d |= (uint64_t)(512 >> 4) << 32;    // stride byte offset: 8 rows x 64 B
+  d |= (uint64_t)(256 >> 4) << 32;    // stride byte offset: 8 rows x 32 B
   d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
-  d |= (uint64_t)4 << 61;             // SWIZZLE_64B
+  d |= (uint64_t)6 << 61;             // SWIZZLE_32B
   return d;
+}
+
+// AND of v over the 128 threads that take named barrier `id` (a barrier too).
+__device__ __forceinline__ bool bar_and_128(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -96,9 +124,13 @@ __device__ __forceinline__ void tmem_ld64_raw(uint32_t taddr, uint32_t (&r)[64])
       : "memory");
 }
 
-// D = s32, A and B signed 8-bit, both K-major, M = 128, N = 64.
-constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(IN >> 3) << 17) |
-                              ((uint32_t)(IM >> 4) << 24);
+// D = s32, A and B signed 8-bit, both K-major, M = 128, N = n (a multiple of
+// 16 up to kMaxN).
+constexpr int kMaxN = 256;
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(IM >> 4) << 24);
+}
 
 // Slices of one fp64 matrix (rows x K, leading dimension ld, batch entries
 // `stride` apart): slice t of row r (batch b) at out + t * plane +
@@ -161,8 +193,42 @@ __global__ void __launch_bounds__(256) slice_rows_kernel(const double* __restric
   }
 }
 
+// Output tiles of one launch.  A lower result (all K ranges equal) takes, per
+// batch entry, the tiles that reach the diagonal or below it (n0 <= m0 + 127:
+// row tm holds min(2 tm + 2, nt) of them and starts at tm (tm + 1)).  A full
+// result is ordered by tile row first, then batch entry and column, with the
+// rows of a triangular P in the order of falling K range (ktri 1: ascending,
+// ktri 2: descending), so that the work per tile never grows along the order.
 struct ITiles {
-  int mt, nt, lower, ktri;
+  int mt, nt, batch, lower, ktri;
+  __device__ int per() const {
+    if (!lower) return mt * nt;
+    return mt * (mt + 1) - (nt < 2 * mt ? 2 * mt - nt : 0);   // the last row may be short
+  }
+  __device__ int count() const { return per() * batch; }
+  __device__ void get(int t, int& tm, int& tn, int& b) const {
+    if (lower) {
+      const int p = per();
+      b = t / p;
+      t -= b * p;
+      int r = (int)((sqrtf(4.f * (float)t + 1.f) - 1.f) * 0.5f);
+      while ((r + 1) * (r + 2) <= t) ++r;
+      while (r * (r + 1) > t) --r;
+      tm = r;
+      tn = t - r * (r + 1);
+    } else {
+      const int row = nt * batch;
+      const int i = t / row;
+      t -= i * row;
+      b = t / nt;
+      tn = t - b * nt;
+      tm = ktri == 2 ? mt - 1 - i : i;
+    }
+  }
+  // The k-th tile of CTA c among g: rounds of g tiles, every other round
+  // walked backwards, so that a CTA given a heavy tile in one round gets a
+  // light one in the next.
+  __device__ static int pick(int k, int c, int g) { return k * g + ((k & 1) ? g - 1 - c : c); }
 };
 
 __global__ void __launch_bounds__(kIThreads, 1)
@@ -174,23 +240,26 @@ __global__ void __launch_bounds__(kIThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  IBars* sm = reinterpret_cast<IBars*>(ring + kIStages * kIStage);
+  double* tile = reinterpret_cast<double*>(ring + kIStages * kIStage);
+  IBars* sm = reinterpret_cast<IBars*>(ring + kIStages * kIStage + kITileBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tm = ts.ktri == 2 ? (int)gridDim.y - 1 - (int)blockIdx.y : (int)blockIdx.y;
-  const int tn = blockIdx.x, bz = blockIdx.z;
-  const int m0 = tm * IM, n0 = tn * IN;
-  if (ts.lower && n0 > m0 + IM - 1) return;   // wholly above the diagonal
-  int kbeg = 0, kend = K;
-  if (ts.ktri == 1) kbeg = (m0 / KC) * KC;
-  if (ts.ktri == 2) kend = (m0 + IM) < K ? (m0 + IM) : K;
-  const int kc0 = kbeg / KC;
-  const int nk = kend > kbeg ? (kend - kbeg + KC - 1) / KC : 0;
+  const int n_tiles = ts.count();
+  auto k_range = [&](int tm, int& kc0, int& nk) {
+    const int m0 = tm * IM;
+    int kbeg = 0, kend = K;
+    if (ts.ktri == 1) kbeg = (m0 / KC) * KC;
+    if (ts.ktri == 2) kend = (m0 + IM) < K ? (m0 + IM) : K;
+    kc0 = kbeg / KC;
+    nk = kend > kbeg ? (kend - kbeg + KC - 1) / KC : 0;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kIStages; ++s) {
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
     }
+    mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->acc_empty, 128);
     mbar_init(&sm->done, 1);
     sm->abort = 0;
     fence_mbar_init();
@@ -206,88 +275,124 @@ __global__ void __launch_bounds__(kIThreads, 1)
     // ------------------------------------------------------------ producer
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
-    int issued = 0;
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % kIStages;
-      if (i >= kIStages && !mbar_wait(&sm->empty[s], ((i / kIStages) - 1) & 1)) {
-        atomicExch(&sm->abort, 1);
-        atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
-        break;
+    int g = 0;   // stages issued over all tiles
+    bool ok = true;
+    for (int k = 0; ok && k * (int)gridDim.x < n_tiles; ++k) {
+      const int t = ITiles::pick(k, blockIdx.x, gridDim.x);
+      if (t >= n_tiles) continue;
+      int tm, tn, bz, kc0, nk;
+      ts.get(t, tm, tn, bz);
+      k_range(tm, kc0, nk);
+      for (int i = 0; i < nk; ++i, ++g) {
+        const int s = g % kIStages;
+        if ((g >= kIStages && !mbar_wait(&sm->empty[s], ((g / kIStages) - 1) & 1)) ||
+            *reinterpret_cast<volatile int*>(&sm->abort)) {
+          atomicExch(&sm->abort, 1);
+          atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        uint8_t* st = ring + s * kIStage;
+        mbar_arrive_expect_tx(&sm->full[s], kIStage);
+        tma_load_3d(st, &tmA, &sm->full[s], (kc0 + i) * KC, bz * M + tm * IM, 0);
+        tma_load_3d(st + S * kASlice, &tmB, &sm->full[s], (kc0 + i) * KC, bz * N + tn * IN, 0);
       }
-      uint8_t* st = ring + s * kIStage;
-      mbar_arrive_expect_tx(&sm->full[s], kIStage);
-      tma_load_3d(st, &tmA, &sm->full[s], (kc0 + i) * KC, bz * M + m0, 0);
-      tma_load_3d(st + S * kASlice, &tmB, &sm->full[s], (kc0 + i) * KC, bz * N + n0, 0);
-      ++issued;
     }
-    for (int i = issued - kIStages < 0 ? 0 : issued - kIStages; i < issued; ++i)
+    for (int i = g - kIStages < 0 ? 0 : g - kIStages; i < g; ++i)
       mbar_wait(&sm->full[i % kIStages], (i / kIStages) & 1);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
+    int g = 0, lt = 0;
     bool ok = true;
-    for (int i = 0; ok && i < nk; ++i) {
-      const int s = i % kIStages;
-      if (!mbar_wait(&sm->full[s], (i / kIStages) & 1)) {
+    for (int k = 0; ok && k * (int)gridDim.x < n_tiles; ++k) {
+      const int t = ITiles::pick(k, blockIdx.x, gridDim.x);
+      if (t >= n_tiles) continue;
+      int tm, tn, bz, kc0, nk;
+      ts.get(t, tm, tn, bz);
+      k_range(tm, kc0, nk);
+      // the epilogue has read the previous tile's accumulators out of TMEM
+      if (lt > 0 && !mbar_wait(&sm->acc_empty, (lt - 1) & 1)) {
         atomicExch(&sm->abort, 1);
         atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
-        ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t a0 = smem_u32(ring + s * kIStage), b0 = a0 + S * kASlice;
-#pragma unroll
-      for (int l = 0; l < S; ++l) {
-#pragma unroll
-        for (int t = 0; t <= l; ++t) {
-          const int u = l - t;
-#pragma unroll
-          for (int kk = 0; kk < KC / 32; ++kk)
-            mma_i8(tmem + l * IN, desc_sw64(a0 + t * kASlice + 32 * kk),
-                   desc_sw64(b0 + u * kBSlice + 32 * kk), kIdescI8,
-                   (i > 0 || t > 0 || kk > 0) ? 1u : 0u);
+      for (int i = 0; i < nk; ++i, ++g) {
+        const int s = g % kIStages;
+        if (!mbar_wait(&sm->full[s], (g / kIStages) & 1)) {
+          atomicExch(&sm->abort, 1);
+          atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(ring + s * kIStage), b0 = a0 + S * kASlice;
+        // A_t times the stacked B_0 .. B_{S-1-t} (N = IN (S - t), cut at
+        // 256) adds A_t B_u^T to level t + u for every u at once: the B
+        // slices lie one after another in the stage and so do the level
+        // accumulators in TMEM
+#pragma unroll
+        for (int t = 0; t < S; ++t)
+#pragma unroll
+          for (int c0 = 0; c0 < IN * (S - t); c0 += kMaxN)
+            mma_i8(tmem + IN * t + c0, desc_sw32(a0 + t * kASlice), desc_sw32(b0 + c0 * KC),
+                   idesc_i8(IN * (S - t) - c0 < kMaxN ? IN * (S - t) - c0 : kMaxN),
+                   (i > 0 || t > 0) ? 1u : 0u);
+        mma_commit(&sm->empty[s]);
       }
-      mma_commit(&sm->empty[s]);
+      mma_commit(&sm->acc_full);   // arrives when this tile's MMAs are done (also if nk == 0)
+      ++lt;
     }
+    // nothing of this thread's may still run on the tensor cores when TMEM is
+    // freed, also after a wait ran out
     mma_commit(&sm->done);
+    mbar_wait(&sm->done, 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    // (1) each thread sums the levels of its row in fp64 and stages the row,
-    // scaled by 2^(e_m - 14), in shared memory (the ring is free once the
-    // MMAs are done); (2) the four warps write C row by row and C2 column by
-    // column, both coalesced, with the column factors 2^(e_n).
-    constexpr int kPitch = IN + 1;
-    double* tile = reinterpret_cast<double*>(ring);   // IM x kPitch
+    // (1) the levels of each row are summed in fp64 straight out of TMEM,
+    // scaled by 2^(e_m - 14) and staged in shared memory, and TMEM is handed
+    // back to the MMA warp (the next tile's products start); (2) the four
+    // warps write C row by row and C2 column by column, both coalesced, with
+    // the column factors 2^(e_n).
     const int q = warp & 3;
     const int r = q * 32 + lane;   // tile row = TMEM lane
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm->done, 0)) &&
-                    !*reinterpret_cast<volatile int*>(&sm->abort);
-    if (!ok && lane == 0) atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
-    if (ok) {
+    int lt = 0;
+    for (int k = 0; k * (int)gridDim.x < n_tiles; ++k) {
+      const int t = ITiles::pick(k, blockIdx.x, gridDim.x);
+      if (t >= n_tiles) continue;
+      int tm, tn, bz, kc0, nk;
+      ts.get(t, tm, tn, bz);
+      k_range(tm, kc0, nk);
+      const int m0 = tm * IM, n0 = tn * IN;
+      const bool mine = __all_sync(0xffffffffu, mbar_wait(&sm->acc_full, lt & 1));
       tc_fence_after();
       double acc[IN];
 #pragma unroll
       for (int j = 0; j < IN; ++j) acc[j] = 0.0;
-      if (nk > 0) {
+      if (mine && nk > 0) {
         // levels from the smallest weight up: acc = sum_l 2^(-7 l) v_l
 #pragma unroll 1
         for (int l = S - 1; l >= 0; --l) {
-          const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + l * IN;
           uint32_t v[IN];
-          tmem_ld64_raw(ta, v);
+          tmem_ld64_raw(tmem + ((uint32_t)(q * 32) << 16) + l * IN, v);
 #pragma unroll
           for (int j = 0; j < IN; ++j)
             acc[j] = fma(acc[j], 0.0078125 /* 2^-7 */, (double)(int)v[j]);
         }
       }
-      // level 0 weighs 2^-14 relative to 2^(e_m + e_n)
+      tc_fence_before();
+      if (mine) mbar_arrive(&sm->acc_empty);
+      // one decision for the four warps; the barrier also keeps the staged
+      // tile from being overwritten before the previous tile's C writes
+      if (!bar_and_128(1, mine && !*reinterpret_cast<volatile int*>(&sm->abort))) {
+        if (threadIdx.x == 64) atomicCAS(status, 0, (int)NVFP4_ERR_TIMEOUT);
+        break;
+      }
       const int m = m0 + r;
-      const double fm = m < M ? scalbn(alpha, eA[bz * M + m] - 14) : 0.0;
+      const double fm = m < M ? scalbn(alpha, eA[bz * M + m] - 14) : 0.0;   // level 0 weighs 2^-14
 #pragma unroll
-      for (int j = 0; j < IN; ++j) tile[r * kPitch + j] = acc[j] * fm;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok) {
+      for (int j = 0; j < IN; ++j) tile[r * kTilePitch + j] = acc[j] * fm;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       double fn[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -299,23 +404,23 @@ __global__ void __launch_bounds__(kIThreads, 1)
       double old[IM / 4][2];
 #pragma unroll
       for (int i = 0; i < IM / 4; ++i) {
-        const int m = m0 + q + 4 * i;
+        const int mm = m0 + q + 4 * i;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int n = n0 + lane + 32 * h;
-          old[i][h] = (beta != 0.0 && m < M && n < N) ? Cb[(int64_t)m * ldc + n] : 0.0;
+          old[i][h] = (beta != 0.0 && mm < M && n < N) ? Cb[(int64_t)mm * ldc + n] : 0.0;
         }
       }
 #pragma unroll
       for (int i = 0; i < IM / 4; ++i) {
-        const int m = m0 + q + 4 * i;
+        const int mm = m0 + q + 4 * i;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int n = n0 + lane + 32 * h;
-          if (m < M && n < N) {
-            double xv = tile[(q + 4 * i) * kPitch + lane + 32 * h] * fn[h];
+          if (mm < M && n < N) {
+            double xv = tile[(q + 4 * i) * kTilePitch + lane + 32 * h] * fn[h];
             if (beta != 0.0) xv = fma(beta, old[i][h], xv);
-            Cb[(int64_t)m * ldc + n] = xv;
+            Cb[(int64_t)mm * ldc + n] = xv;
           }
         }
       }
@@ -327,11 +432,12 @@ __global__ void __launch_bounds__(kIThreads, 1)
           const double f = scalbn(1.0, eB[bz * N + n]);
 #pragma unroll
           for (int h = 0; h < IM / 32; ++h) {
-            const int m = m0 + lane + 32 * h;
-            if (m < M) C2b[(int64_t)n * ldc2 + m] = tile[(lane + 32 * h) * kPitch + j] * f;
+            const int mm = m0 + lane + 32 * h;
+            if (mm < M) C2b[(int64_t)n * ldc2 + mm] = tile[(lane + 32 * h) * kTilePitch + j] * f;
           }
         }
       }
+      ++lt;
     }
   }
   tc_fence_before();
@@ -342,14 +448,14 @@ __global__ void __launch_bounds__(kIThreads, 1)
   }
 }
 
-// 3-D map of the slices: (K bytes, batch * rows, S), box {64, box_rows, S}.
+// 3-D map of the slices: (K bytes, batch * rows, S), box {32, box_rows, S}.
 bool encode_slices(CUtensorMap* map, const int8_t* base, int64_t K, int64_t total_rows,
                    int64_t kp, int64_t plane, int box_rows) {
   const uint64_t dims[3] = {(uint64_t)K, (uint64_t)total_rows, (uint64_t)S};
   const uint64_t strides[2] = {(uint64_t)kp, (uint64_t)plane};
   const uint32_t box[3] = {(uint32_t)KC, (uint32_t)box_rows, (uint32_t)S};
   return encode_tmap_nd(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, dims, strides, box,
-                        CU_TENSOR_MAP_SWIZZLE_64B);
+                        CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 nvfp4_status slice(const double* X, int64_t rows, int64_t K, int64_t ld, int64_t stride,
@@ -411,9 +517,12 @@ nvfp4_status dgemm_i8(int M, int N, int K, double alpha, const double* P, int64_
   if (!encode_slices(&ma, A, K, (int64_t)batch * M, kp, planeA, IM) ||
       !encode_slices(&mb, Bsrc, K, (int64_t)batch * N, kp, same ? planeA : planeB, IN))
     return NVFP4_ERR_CUDA;
-  const ITiles ts{(M + IM - 1) / IM, (N + IN - 1) / IN, lower, ktri};
-  const dim3 grid((unsigned)ts.nt, (unsigned)ts.mt, (unsigned)batch);
-  if (grid.y > 65535) return NVFP4_ERR_SHAPE;
+  const ITiles ts{(M + IM - 1) / IM, (N + IN - 1) / IN, batch, lower, ktri};
+  const int64_t n_tiles =
+      (int64_t)(lower ? (int64_t)ts.mt * (ts.mt + 1) : (int64_t)ts.mt * ts.nt) * batch;
+  if (n_tiles > (1ll << 30)) return NVFP4_ERR_SHAPE;
+  const int sms = num_sms();
+  const dim3 grid((unsigned)(n_tiles < sms ? n_tiles : sms));
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(dgemm_i8_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kISmem));
   NVFP4_CUDA_TRY(launch_chained(dgemm_i8_kernel, grid, dim3(kIThreads), kISmem, st, ma, mb, eA,
