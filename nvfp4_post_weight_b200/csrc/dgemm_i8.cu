@@ -134,62 +134,104 @@ __host__ __device__ constexpr uint32_t idesc_i8(int n) {
 
 // Slices of one fp64 matrix (rows x K, leading dimension ld, batch entries
 // `stride` apart): slice t of row r (batch b) at out + t * plane +
-// (b * rows + r) * kp, exponent at e[b * rows + r].  One warp per row.
+// (b * rows + r) * kp, exponent at e[b * rows + r].  One CTA per row (blockIdx.x
+// = r, blockIdx.y = b), eight consecutive values per thread and chunk; the
+// first chunk stays in registers between the max pass and the digit pass.
+//
+// Each scaled value v = 2^(7 S) 2^-ex x (|v| < 2^48) is rounded once to an
+// integer, ties to even, by adding 1.5 * 2^52: the sum's 52-bit fraction is
+// then f = 2^51 + v, whose low 28 bits are those of v and whose bits from 28
+// up, less 2^23, are floor(v / 2^28).  The balanced base-128 digits are cut
+// from the bottom with 32-bit steps: four from the low 28 bits (whose carry,
+// 0 or 1, goes to the high part), two from the high part, and the rest is the
+// top digit.  Digit t in [-64, 63] for t > 0, the top one in [-64, 64].
+__device__ __forceinline__ void load8(const double* __restrict__ x, int64_t k, int64_t K,
+                                      double (&xv)[8]) {
+  if (k + 8 <= K && ((reinterpret_cast<uintptr_t>(x + k) & 15) == 0)) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const double2 p2 = reinterpret_cast<const double2*>(x + k)[q];
+      xv[2 * q] = p2.x;
+      xv[2 * q + 1] = p2.y;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xv[q] = k + q < K ? x[k + q] : 0.0;
+  }
+}
+
+__device__ __forceinline__ void digits8(const double (&xv)[8], double to_int, int8_t* o,
+                                        int64_t plane) {
+  static_assert(S == 7, "four low digits, two high ones and the top digit");
+  uint32_t w[S][2];
+#pragma unroll
+  for (int t = 0; t < S; ++t) w[t][0] = w[t][1] = 0u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const double tq = __dadd_rn(__dmul_rn(xv[q], to_int), 0x1.8p52);
+    const uint32_t lw = (uint32_t)__double2loint(tq), hw = (uint32_t)__double2hiint(tq);
+    int lo = (int)(lw & 0x0FFFFFFFu);
+    int hi = (int)(((hw & 0xFFFFFu) << 4) | (lw >> 28)) - (1 << 23);
+    const int sh = 8 * (q & 3);
+#pragma unroll
+    for (int t = S - 1; t >= S - 4; --t) {
+      const int a = ((lo + 64) & 127) - 64;
+      lo = (lo - a) >> 7;
+      w[t][q >> 2] |= ((uint32_t)a & 0xFFu) << sh;
+    }
+    hi += lo;
+#pragma unroll
+    for (int t = S - 5; t >= 1; --t) {
+      const int a = ((hi + 64) & 127) - 64;
+      hi = (hi - a) >> 7;
+      w[t][q >> 2] |= ((uint32_t)a & 0xFFu) << sh;
+    }
+    w[0][q >> 2] |= ((uint32_t)hi & 0xFFu) << sh;
+  }
+#pragma unroll
+  for (int t = 0; t < S; ++t) *reinterpret_cast<uint2*>(o + t * plane) = make_uint2(w[t][0], w[t][1]);
+}
+
 __global__ void __launch_bounds__(256) slice_rows_kernel(const double* __restrict__ X,
                                                          int64_t rows, int64_t K, int64_t ld,
                                                          int64_t stride, int64_t kp,
                                                          int64_t plane,
                                                          int8_t* __restrict__ out,
                                                          int* __restrict__ e) {
+  __shared__ double wmax[8];
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t r = blockIdx.x;
   const int b = blockIdx.y;
-  if (r >= rows) return;
+  const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31;
   const double* x = X + b * stride + r * ld;
+  const int64_t k0 = 8 * tid, step = 8 * (int64_t)T;
+  double xv[8];
+  load8(x, k0, K, xv);   // (zeros past K: kp and K are multiples of 16)
   double m = 0.0;
-  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(x[k]));
+#pragma unroll
+  for (int q = 0; q < 8; ++q) m = fmax(m, fabs(xv[q]));
+  for (int64_t k = k0 + step; k < kp; k += step) {
+    double yv[8];
+    load8(x, k, K, yv);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m = fmax(m, fabs(yv[q]));
+  }
   for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) wmax[tid >> 5] = m;
+  __syncthreads();
+  m = 0.0;
+  for (int w = 0; w < (T >> 5); ++w) m = fmax(m, wmax[w]);
   // 2^-ex m in [1/4, 1/2): the first slice rint(128 x) stays within [-64, 64]
   const int ex = m > 0.0 ? ilogb(m) + 2 : 0;
-  const double scale = scalbn(1.0, -ex);   // exact power of two
+  const double to_int = scalbn(1.0, 7 * S - ex);   // exact power of two
   const int64_t row = b * rows + r;
-  if (lane == 0) e[row] = ex;
+  if (tid == 0) e[row] = ex;
   int8_t* o = out + row * kp;
-  // eight consecutive values per lane and step (K and kp are multiples of 16).
-  // Each scaled value is rounded once to an integer multiple of 2^(-7 S)
-  // (|v| < 2^(7 S - 1)) and cut into balanced base-128 digits from the bottom:
-  // digit t in [-64, 63] for t > 0, the top digit in [-64, 64].
-  const double to_int = scalbn(scale, 7 * S);
-  for (int64_t k = 8 * lane; k < kp; k += 256) {
-    long long v[8];
-    if (k + 8 <= K && ((reinterpret_cast<uintptr_t>(x + k) & 15) == 0)) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const double2 p2 = reinterpret_cast<const double2*>(x + k)[q];
-        v[2 * q] = __double2ll_rn(p2.x * to_int);
-        v[2 * q + 1] = __double2ll_rn(p2.y * to_int);
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = k + q < K ? __double2ll_rn(x[k + q] * to_int) : 0ll;
-    }
-    uint32_t w[S][2];
-#pragma unroll
-    for (int t = 0; t < S; ++t) w[t][0] = w[t][1] = 0u;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      long long dgt = v[q];
-#pragma unroll
-      for (int t = S - 1; t >= 0; --t) {
-        const long long a = t > 0 ? ((dgt + 64) & 127) - 64 : dgt;
-        dgt = (dgt - a) >> 7;   // exact: dgt - a is a multiple of 128
-        w[t][q >> 2] |= ((uint32_t)(int)a & 0xFFu) << (8 * (q & 3));
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < S; ++t)
-      *reinterpret_cast<uint2*>(o + t * plane + k) = make_uint2(w[t][0], w[t][1]);
+  if (k0 < kp) digits8(xv, to_int, o + k0, plane);
+  for (int64_t k = k0 + step; k < kp; k += step) {
+    double yv[8];
+    load8(x, k, K, yv);
+    digits8(yv, to_int, o + k, plane);
   }
 }
 
@@ -460,9 +502,12 @@ bool encode_slices(CUtensorMap* map, const int8_t* base, int64_t K, int64_t tota
 
 nvfp4_status slice(const double* X, int64_t rows, int64_t K, int64_t ld, int64_t stride,
                    int batch, int8_t* out, int* e, int64_t kp, int64_t plane, cudaStream_t st) {
-  const dim3 grid((unsigned)((rows + 7) / 8), (unsigned)batch);
-  NVFP4_CUDA_TRY(launch_chained(slice_rows_kernel, grid, dim3(256), 0, st, X, rows, K, ld, stride,
-                                kp, plane, out, e));
+  // one CTA per row, one 8-value chunk per thread up to K = 2048
+  int threads = (int)((kp / 8 + 31) / 32 * 32);
+  threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
+  const dim3 grid((unsigned)rows, (unsigned)batch);
+  NVFP4_CUDA_TRY(launch_chained(slice_rows_kernel, grid, dim3(threads), 0, st, X, rows, K, ld,
+                                stride, kp, plane, out, e));
   count_launches(1);
   return NVFP4_OK;
 }

@@ -60,20 +60,40 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int64_t d, float 
 
 // A[i][j] = H_d[d-1-i][d-1-j]; dead diagonal entries become 1 + lambda.
 // Also zero-fills X (the inverse is built from its block diagonal outward).
+// Rows blockIdx.y, + gridDim.y, ...; four consecutive columns per thread (d
+// is a multiple of 16); H read as float4 when it is 16-byte aligned (vec).
 __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
                                     double* __restrict__ A, double* __restrict__ X,
-                                    PrepHeader* hdr) {
+                                    PrepHeader* hdr, int vec) {
   const double lam = hdr->lambda64;
-  const int64_t total = d * d;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t i = idx / d, j = idx - i * d;
-    const float h = H[(d - 1 - i) * d + (d - 1 - j)];
-    if (!isfinite(h)) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
-    double a = (double)h;
-    if (i == j) a = (h == 0.f ? 1.0 : a) + lam;
-    A[idx] = a;
-    X[idx] = 0.0;
+  const int64_t j = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (j >= d) return;
+  for (int64_t i = blockIdx.y; i < d; i += gridDim.y) {
+    // H row d-1-i, columns d-4-j .. d-1-j, i.e. hv[3..0] for A's columns j .. j+3
+    const float* hr = H + (d - 1 - i) * d + (d - 4 - j);
+    float hv[4];
+    if (vec) {
+      const float4 h4 = *reinterpret_cast<const float4*>(hr);
+      hv[0] = h4.w, hv[1] = h4.z, hv[2] = h4.y, hv[3] = h4.x;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) hv[q] = hr[3 - q];
+    }
+    double a[4];
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      bad |= !isfinite(hv[q]);
+      a[q] = (double)hv[q];
+      if (i == j + q) a[q] = (hv[q] == 0.f ? 1.0 : a[q]) + lam;
+    }
+    if (bad) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+    double2* Ar = reinterpret_cast<double2*>(A + i * d + j);   // workspace: aligned
+    double2* Xr = reinterpret_cast<double2*>(X + i * d + j);
+    Ar[0] = make_double2(a[0], a[1]);
+    Ar[1] = make_double2(a[2], a[3]);
+    Xr[0] = make_double2(0.0, 0.0);
+    Xr[1] = make_double2(0.0, 0.0);
   }
 }
 
@@ -380,14 +400,30 @@ __global__ void __launch_bounds__(kPanelThreads)
   }
 }
 
-// U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.
+// U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.  Rows
+// blockIdx.y, + gridDim.y, ...; four consecutive columns per thread, U
+// written as float4 when it is 16-byte aligned (vec).
 __global__ void reverse_to_upper_kernel(const double* __restrict__ X, int64_t d,
-                                        float* __restrict__ U) {
-  const int64_t total = d * d;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t i = idx / d, j = idx - i * d;
-    U[idx] = (j >= i) ? (float)X[(d - 1 - i) * d + (d - 1 - j)] : 0.f;
+                                        float* __restrict__ U, int vec) {
+  const int64_t j = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (j >= d) return;
+  for (int64_t i = blockIdx.y; i < d; i += gridDim.y) {
+    float u[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j + 3 >= i) {   // some of the four are on or above the diagonal
+      // X row d-1-i, columns d-4-j .. d-1-j (workspace: 16-byte aligned pairs)
+      const double2* xr = reinterpret_cast<const double2*>(X + (d - 1 - i) * d + (d - 4 - j));
+      const double2 p = xr[0], q2 = xr[1];
+      const double xv[4] = {q2.y, q2.x, p.y, p.x};   // columns j .. j+3 of the reversed row
+#pragma unroll
+      for (int q = 0; q < 4; ++q) u[q] = (j + q >= i) ? (float)xv[q] : 0.f;
+    }
+    float* ur = U + i * d + j;
+    if (vec) {
+      *reinterpret_cast<float4*>(ur) = make_float4(u[0], u[1], u[2], u[3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ur[q] = u[q];
+    }
   }
 }
 
@@ -444,7 +480,9 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   diag_stats_kernel<<<1, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-  reverse_damp_kernel<<<grid_for(d * d, 256), 256, 0, st>>>(H, d, L.A, L.X, L.hdr);
+  const dim3 rgrid((unsigned)((d / 4 + 255) / 256), (unsigned)(d < 65535 ? d : 65535));
+  reverse_damp_kernel<<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.hdr,
+                                             (reinterpret_cast<uintptr_t>(H) & 15) == 0);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
 
@@ -534,7 +572,8 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
       if (s != NVFP4_OK) return s;
     }
   }
-  reverse_to_upper_kernel<<<grid_for(d * d, 256), 256, 0, st>>>(L.X, d, U);
+  reverse_to_upper_kernel<<<rgrid, 256, 0, st>>>(L.X, d, U,
+                                                 (reinterpret_cast<uintptr_t>(U) & 15) == 0);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;

@@ -166,7 +166,9 @@ __global__ void weight_amax_kernel(const T* __restrict__ W, int64_t d_out, int64
   if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
 }
 
-constexpr int kReplayThreads = 256;                 // 8 warps = 16 rows in flight
+// 14 warps = 28 rows in flight, one CTA per SM: 4096 rows fill 147 SMs
+// evenly (16-row CTAs two to an SM would leave some SMs 32 rows, others 16)
+constexpr int kReplayThreads = 448;
 constexpr int kRowsPerCta = kReplayThreads / 16;
 constexpr int kNb = kLazyBatch / kBlock;            // blocks per batch (8)
 constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a batch (36)
@@ -213,20 +215,37 @@ __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restri
 // One candidate's replay of the in-block GPTQ updates (fp64).  v holds the
 // block's 16 current values and is consumed.  Ud points at the block's
 // diagonal 16x16 tile (row-major, 16-byte aligned), invd at its 1/U_jj.
-// Returns the score sum delta_j^2; delta and the signed rounded magnitudes
-// q_j / s (exact in fp32) are written out -- the code nibbles are derived
+// Returns the score sum delta_j^2; delta and the high words of the signed
+// rounded magnitudes q_j / s are written out -- the code nibbles are derived
 // once, from the winner's magnitudes, not by every candidate.
+//
+// The nearest E2M1 magnitude of |x| is taken by the add-and-subtract method
+// (nvfp4_format.cuh) with the spacing constant picked, the saturation at 6
+// and the sign applied on the high word of the double: every rounded value
+// below 2^20 is a multiple of 1/2 whose low word is zero, so these integer
+// steps give the same bits as the fp64 comparisons and selects they replace,
+// and only the additions and the GPTQ arithmetic use the fp64 pipe.
 __device__ __forceinline__ double replay(double (&v)[16], double s, double inv_s,
                                          const double* __restrict__ Ud,
                                          const double* __restrict__ invd, double (&dl)[16],
-                                         float (&sq)[16]) {
+                                         uint32_t (&sq)[16]) {
   double score = 0.0;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const double x = __dmul_rn(v[j], inv_s);
-    const double r = e2m1_round_mag(fabs(x));
-    const double sr = x < 0.0 ? -r : r;
-    sq[j] = (float)sr;
+    const uint32_t xh = (uint32_t)__double2hiint(x), xl = (uint32_t)__double2loint(x);
+    const uint32_t ah = xh & 0x7FFFFFFFu;
+    // 1.5 * 2^51, 2^52 or 2^53 for |x| below 2, below 4, from 4 up (spacing
+    // 1/2, 1, 2)
+    const int ex = (int)(ah >> 20) - 1023;
+    const uint32_t mh = 0x43280000u + ((uint32_t)min(max(ex, 0), 2) << 20);
+    const double M = __hiloint2double((int)mh, 0);
+    const double r = __dsub_rn(__dadd_rn(__hiloint2double((int)ah, (int)xl), M), M);
+    const bool neg = (xh >> 31) != 0 && (ah | xl) != 0;   // x < 0
+    const uint32_t rh =
+        min((uint32_t)__double2hiint(r), 0x40180000u /* 6.0 */) | (neg ? 0x80000000u : 0u);
+    sq[j] = rh;
+    const double sr = __hiloint2double((int)rh, 0);
     const double res = __fma_rn(-sr, s, v[j]);       // v_j - q_j, one rounding
     const double d = __dmul_rn(res, invd[j]);
     dl[j] = d;
@@ -242,6 +261,16 @@ __device__ __forceinline__ double replay(double (&v)[16], double s, double inv_s
     }
   }
   return score;
+}
+
+// E2M1 code nibble of a rounded signed magnitude given by its high word (the
+// form replay() writes): index 1 for 1/2, 2 (E - 1023) + 2 + m above it (E
+// the biased exponent, m the mantissa's top bit), sign bit 8 for a negative
+// nonzero value.
+__device__ __forceinline__ uint32_t e2m1_nibble_hi(uint32_t rh) {
+  const uint32_t mag = rh & 0x7FFFFFFFu, e = mag >> 20;
+  const uint32_t idx = mag == 0 ? 0u : (e == 1022u ? 1u : 2u * (e - 1023u) + 2u + ((mag >> 19) & 1u));
+  return idx | ((rh >> 31) && idx ? 8u : 0u);
 }
 
 // Block-scale rules: Schur Replay, and the two independent-block rules it is
@@ -265,26 +294,40 @@ __global__ void __launch_bounds__(kReplayThreads)
   extern __shared__ double4 smem_d4[];
   double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
   double* invd = Ut + kUTiles * 256;                         // 128
-  double* rows = invd + kLazyBatch;                          // kRowsPerCta x 128
+  double* s_tab = invd + kLazyBatch;                         // e4m3_value(k) * s_g
+  double* inv_tab = s_tab + 128;                             // 1 / s_tab[k]
+  double* rows = inv_tab + 128;                              // kRowsPerCta x 128
   const int nblk = bw / kBlock;
   pdl_wait();
   {
     // Stage the batch's upper block-triangular part of U as 16 x 16 fp64
-    // tiles.  Thread t handles element e = t of every tile (kReplayThreads ==
-    // 256 == tile size) and issues all its loads before any store.
-    static_assert(kReplayThreads == 256, "one tile element per thread");
-    const int e = threadIdx.x, i = e >> 4, j = e & 15;
-    float u[kUTiles];
+    // tiles: thread t < 256 handles element e = t of every tile and issues
+    // all its loads before any store.  The other threads fill the candidate
+    // scale table (e4m3_value(k) s_g and its reciprocal) and 1/U_jj.
+    static_assert(kReplayThreads >= 256 + 128, "tile elements, then the tables");
+    if (threadIdx.x < 256) {
+      const int e = threadIdx.x, i = e >> 4, j = e & 15;
+      float u[kUTiles];
 #pragma unroll
-    for (int t = 0, p = 0, q = 0; t < kUTiles; ++t) {
-      const int gi = 16 * p + i, gj = 16 * q + j;
-      u[t] = (p < nblk && q < nblk && gj >= gi) ? U[(int64_t)(c0 + gi) * d_in + c0 + gj] : 0.f;
-      if (++q == kNb) q = ++p;   // tiles (p, q), q >= p, row-major
+      for (int t = 0, p = 0, q = 0; t < kUTiles; ++t) {
+        const int gi = 16 * p + i, gj = 16 * q + j;
+        u[t] = (p < nblk && q < nblk && gj >= gi) ? U[(int64_t)(c0 + gi) * d_in + c0 + gj] : 0.f;
+        if (++q == kNb) q = ++p;   // tiles (p, q), q >= p, row-major
+      }
+#pragma unroll
+      for (int t = 0; t < kUTiles; ++t) Ut[t * 256 + e] = (double)u[t];
+    } else {
+      for (int c = threadIdx.x - 256; c < 128 + bw; c += kReplayThreads - 256) {
+        if (c < 128) {
+          const double sk = e4m3_value(c < 127 ? c : 126) * (double)*sg_ptr;
+          s_tab[c] = sk;
+          inv_tab[c] = 1.0 / sk;
+        } else {
+          const int jj = c - 128;
+          invd[jj] = 1.0 / (double)U[(int64_t)(c0 + jj) * d_in + c0 + jj];
+        }
+      }
     }
-#pragma unroll
-    for (int t = 0; t < kUTiles; ++t) Ut[t * 256 + e] = (double)u[t];
-    if (threadIdx.x < bw)
-      invd[threadIdx.x] = 1.0 / (double)U[(int64_t)(c0 + threadIdx.x) * d_in + c0 + threadIdx.x];
   }
   __syncthreads();
 
@@ -294,7 +337,7 @@ __global__ void __launch_bounds__(kReplayThreads)
   const int warp = threadIdx.x >> 5;
   const int rloc = warp * 2 + half;
   double* row = rows + rloc * kLazyBatch;
-  float* mrow = reinterpret_cast<float*>(rows + kRowsPerCta * kLazyBatch) + rloc * 16;
+  uint32_t* mrow = reinterpret_cast<uint32_t*>(rows + kRowsPerCta * kLazyBatch) + rloc * 16;
   const unsigned FULL = 0xffffffffu;
 
   for (int64_t rb = (int64_t)blockIdx.x * kRowsPerCta; rb < d_out;
@@ -316,8 +359,8 @@ __global__ void __launch_bounds__(kReplayThreads)
       }
       const int k0 = max(e4m3_code_rn(amax / six_sg), 1);
       const int lo = min(max(k0 - 8, 1), 127 - kCand);
-      const double s = e4m3_value(lo + hl) * sg;   // exact: 4 + 24 significant bits
-      const double inv_s = 1.0 / s;
+      const double s = s_tab[lo + hl];   // e4m3_value * s_g, exact: 4 + 24 significant bits
+      const double inv_s = inv_tab[lo + hl];
       const double* Ud = Ut + utile(b, b) * 256;
       const double* idb = invd + 16 * b;
 
@@ -335,7 +378,7 @@ __global__ void __launch_bounds__(kReplayThreads)
         }
       }
       double dl[16];
-      float sq[16];
+      uint32_t sq[16];
       const double score = replay(v, s, inv_s, Ud, idb, dl, sq);
       if constexpr (kRule == kRuleSchurReplay) sel = score;
 
@@ -372,10 +415,7 @@ __global__ void __launch_bounds__(kReplayThreads)
       {
         // lane hl encodes column hl of the winner; the 16 nibbles are OR-ed
         // into the block's 8 code bytes (low nibble = even column)
-        const float m = mrow[hl], am = fabsf(m);
-        const uint32_t idx =
-            (uint32_t)(am < 2.f ? 2.f * am : (am < 4.f ? am + 2.f : 0.5f * am + 4.f));
-        const uint32_t nib = live ? (idx | ((m < 0.f && idx) ? 8u : 0u)) : 0u;
+        const uint32_t nib = live ? e2m1_nibble_hi(mrow[hl]) : 0u;
         uint32_t lo_w = hl < 8 ? nib << (4 * hl) : 0u, hi_w = hl < 8 ? 0u : nib << (4 * (hl - 8));
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) {
@@ -442,8 +482,8 @@ int grid_for(int64_t n, int threads) {
 }
 
 constexpr size_t kReplaySmem =
-    sizeof(double) * (kUTiles * 256 + kLazyBatch + kRowsPerCta * kLazyBatch) +
-    sizeof(float) * kRowsPerCta * 16;
+    sizeof(double) * (kUTiles * 256 + kLazyBatch + 2 * 128 + kRowsPerCta * kLazyBatch) +
+    sizeof(uint32_t) * kRowsPerCta * 16;
 
 }  // namespace
 
@@ -505,7 +545,7 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
   if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in, L.S))
     return NVFP4_ERR_CUDA;
   const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
-  const int rgrid = (int)(row_groups < 2 * kNumSMs ? row_groups : 2 * kNumSMs);
+  const int rgrid = (int)(row_groups < kNumSMs ? row_groups : kNumSMs);
   for (int64_t cs = 0; cs < d_in; cs += L.S) {
     const int64_t send = (d_in - cs) < L.S ? d_in : cs + L.S;
     const int64_t j0 = cs + kLazyBatch;   // first column any update of this super-batch touches

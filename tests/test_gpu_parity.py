@@ -193,6 +193,29 @@ def test_prepare_dead_column():
     assert rel_frob(U.cpu().numpy(), O.inverse_cholesky_upper(Hd)) < 1e-4
 
 
+def test_prepare_unaligned_h_and_u_equal_aligned():
+    """H and U at 4-byte offsets (no 16-byte alignment): the element-wise
+    paths of the index-reversal kernels give the same factor bit for bit."""
+    d = 208
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((2 * d, d)) * rng.lognormal(0.0, 1.0, size=d)
+    H32 = (X.T @ X).astype(np.float32)
+    ws = B.workspace(B.nvfp4_prepare_workspace_size(d), DEV)
+    H = torch.from_numpy(H32).to(DEV)
+    U = torch.empty((d, d), dtype=torch.float32, device=DEV)
+    B.nvfp4_gptq_prepare(H, 0.01, U, None, None, ws)
+    Hbuf = torch.empty(d * d + 1, dtype=torch.float32, device=DEV)
+    Ubuf = torch.full((d * d + 1,), float("nan"), dtype=torch.float32, device=DEV)
+    Hu, Uu = Hbuf[1:].view(d, d), Ubuf[1:].view(d, d)
+    Hu.copy_(H)
+    assert Hu.data_ptr() % 16 != 0 and Uu.data_ptr() % 16 != 0
+    B.nvfp4_gptq_prepare(Hu, 0.01, Uu, None, None, ws)
+    torch.cuda.synchronize()
+    assert B.nvfp4_workspace_status(ws) == 0
+    assert torch.equal(Uu.cpu(), U.cpu())
+    assert torch.isnan(Ubuf[0]).item()
+
+
 def test_prepare_not_pd_sets_status():
     d = 32
     H = -torch.eye(d, dtype=torch.float32, device=DEV)
