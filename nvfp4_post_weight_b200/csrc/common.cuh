@@ -92,6 +92,14 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
                         float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
                         int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
                         cudaStream_t st, double* C64 = nullptr);
+// The same product with both operands given already split for 3xTF32:
+// Ph = tf32(P) and Pl = P - Ph (likewise Qh, Ql), same layout and strides.
+nvfp4_status gemm_nt_tc_split(int M, int N, int K, float alpha, const float* Ph,
+                              const float* Pl, int64_t ldp, int64_t strideP, const float* Qh,
+                              const float* Ql, int64_t ldq, int64_t strideQ, float beta,
+                              float* C, int64_t ldc, int64_t strideC, float* C2, int64_t ldc2,
+                              int64_t strideC2, int batch, int lower, int* status,
+                              cudaStream_t st, double* C64 = nullptr);
 
 // C = beta C + alpha P Q^T in fp64 on the tensor cores (mma.sync m8n8k4; same
 // operand conventions as gemm_nt_tc; C2 = C^T needs beta == 0; lower: only

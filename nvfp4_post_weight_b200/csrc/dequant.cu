@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "sm100.cuh"
 #include "nvfp4_format.cuh"
 
 namespace nvfp4 {
@@ -60,12 +61,14 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes,
 // Et = (W - Q)^T in fp32 (W bf16 or fp32) for a 64 x 64 tile of W: one
 // thread per (row, 16-weight block) computes its 16 errors with a single
 // rounding each, the tile is transposed through shared memory, and Et's rows
-// (ldE >= d_out apart) are written whole.
+// (ldE >= d_out apart) are written whole -- already split for the 3xTF32
+// Gram product: Eh = tf32(Et), El = Et - Eh (exact).
 template <typename T>
 __global__ void __launch_bounds__(256)
     error_t_kernel(const T* __restrict__ W, const uint8_t* __restrict__ codes,
                    const uint8_t* __restrict__ scales, const float* __restrict__ sg_ptr,
-                   int64_t d_out, int64_t d_in, float* __restrict__ Et, int64_t ldE) {
+                   int64_t d_out, int64_t d_in, float* __restrict__ Eh, float* __restrict__ El,
+                   int64_t ldE) {
   __shared__ float tile[64][65];
   const float sg = *sg_ptr;
   const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
@@ -94,7 +97,11 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const int idx = t + 256 * q, j = idx >> 6, rr = idx & 63;
-    if (c0 + j < d_in && r0 + rr < d_out) Et[(c0 + j) * ldE + r0 + rr] = tile[j][rr];
+    if (c0 + j < d_in && r0 + rr < d_out) {
+      const float v = tile[j][rr], h = sm100::tf32_rn(v);
+      Eh[(c0 + j) * ldE + r0 + rr] = h;
+      El[(c0 + j) * ldE + r0 + rr] = v - h;
+    }
   }
 }
 
@@ -192,7 +199,7 @@ nvfp4_status launch_scales_tiled(const uint8_t* scales, int64_t rows, int64_t d_
 }
 
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in) {
-  return kWsHeader + align256(sizeof(float) * et_ld(d_out) * d_in) +
+  return kWsHeader + 2 * align256(sizeof(float) * et_ld(d_out) * d_in) +
          align256(sizeof(float) * d_in * d_in) + align256(sizeof(double) * kDotBlocks);
 }
 
@@ -205,10 +212,12 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
                                 cudaStream_t st) {
   char* p = static_cast<char*>(ws) + kWsHeader;
   const int64_t ldE = et_ld(d_out);
-  float* Et = reinterpret_cast<float*>(p);
-  float* G = reinterpret_cast<float*>(p + align256(sizeof(float) * ldE * d_in));
-  double* part = reinterpret_cast<double*>(p + align256(sizeof(float) * ldE * d_in) +
-                                           align256(sizeof(float) * d_in * d_in));
+  const size_t et_bytes = align256(sizeof(float) * ldE * d_in);
+  float* Eh = reinterpret_cast<float*>(p);
+  float* El = reinterpret_cast<float*>(p + et_bytes);
+  float* G = reinterpret_cast<float*>(p + 2 * et_bytes);
+  double* part =
+      reinterpret_cast<double*>(p + 2 * et_bytes + align256(sizeof(float) * d_in * d_in));
   if (d_out == 0 || d_in == 0) {
     NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
     return NVFP4_OK;
@@ -216,17 +225,17 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
   const dim3 tgrid((unsigned)((d_in + 63) / 64), (unsigned)((d_out + 63) / 64));
   if (wt == NVFP4_BF16)
     error_t_kernel<uint16_t><<<tgrid, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes,
-                                                    scales, sg, d_out, d_in, Et, ldE);
+                                                    scales, sg, d_out, d_in, Eh, El, ldE);
   else
     error_t_kernel<float><<<tgrid, 256, 0, st>>>(static_cast<const float*>(W), codes, scales,
-                                                 sg, d_out, d_in, Et, ldE);
+                                                 sg, d_out, d_in, Eh, El, ldE);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   int* status = static_cast<int*>(ws);
   NVFP4_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
   // G = Et Et^T (d_in x d_in, K = d_out), lower tiles only
-  nvfp4_status s = gemm_nt_tc((int)d_in, (int)d_in, (int)d_out, 1.f, Et, ldE, 0, Et, ldE, 0,
-                              0.f, G, d_in, 0, nullptr, 0, 0, 1, 1, status, st);
+  nvfp4_status s = gemm_nt_tc_split((int)d_in, (int)d_in, (int)d_out, 1.f, Eh, El, ldE, 0, Eh,
+                                    El, ldE, 0, 0.f, G, d_in, 0, nullptr, 0, 0, 1, 1, status, st);
   if (s != NVFP4_OK) return s;
   sym_tile_dot_kernel<<<kDotBlocks, 256, 0, st>>>(H, G, d_in, part);
   NVFP4_LAUNCH_CHECK();

@@ -9,7 +9,12 @@
 //               128-byte swizzled (the canonical K-major layout)
 //   warps 2-5   split: each element x becomes hi = tf32(x) (rounded in place)
 //               and lo = x - hi (written to a twin buffer at the same offset,
-//               so the swizzle is kept); then fence.proxy.async
+//               so the swizzle is kept); then fence.proxy.async.  When the
+//               caller gives the operands already split (hi and lo arrays,
+//               gemm_nt_tc_split), the producer loads all four tiles and
+//               these warps stay idle: an operand that many tiles read is
+//               then split once instead of once per tile, and the shared
+//               memory traffic of the split is gone.
 //   warp 1      MMA issuer: per K step of 8, main += Ph Qh and
 //               cross += Ph Ql + Pl Qh (kind::tf32, M=128 N=128)
 //   warps 6-13  epilogue (two warps per TMEM lane quarter, 64 columns each):
@@ -92,7 +97,9 @@ struct TileSpace {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nt_tc_kernel(const __grid_constant__ CUtensorMap tmP,
-                      const __grid_constant__ CUtensorMap tmQ, float* __restrict__ C,
+                      const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmPl,
+                      const __grid_constant__ CUtensorMap tmQl, int presplit, float* __restrict__ C,
                       int64_t ldc, int64_t strideC, float* __restrict__ C2, int64_t ldc2,
                       int64_t strideC2, int M, int N, int K, float alpha, float beta,
                       TileSpace ts, int* status, double* __restrict__ C64) {
@@ -129,6 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     tma_prefetch(&tmP);
     tma_prefetch(&tmQ);
+    if (presplit) {
+      tma_prefetch(&tmPl);
+      tma_prefetch(&tmQl);
+    }
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -141,10 +152,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&sm->full[s], 2 * kTile);
+        mbar_arrive_expect_tx(&sm->full[s], (presplit ? 4 : 2) * kTile);
         uint8_t* st = ring + s * kStageBytes;
         tma_load_3d(st, &tmP, &sm->full[s], kb * GK, tm * GM, b);
         tma_load_3d(st + kTile, &tmQ, &sm->full[s], kb * GK, tn * GN, b);
+        if (presplit) {
+          tma_load_3d(st + 2 * kTile, &tmPl, &sm->full[s], kb * GK, tm * GM, b);
+          tma_load_3d(st + 3 * kTile, &tmQl, &sm->full[s], kb * GK, tn * GN, b);
+        }
         ++issued;
         if (++s == kStages) {
           s = 0;
@@ -161,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sm->full[s], ph);
       }
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp >= 2 && warp < 6 && !presplit) {
     // ------------------------------------------------------------ split
     const int tid = threadIdx.x - 64;   // 0..127
     int s = 0;
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t mainc = tmem + buf * kBufCols, cross = mainc + GN;
         const int kb1 = kb0 + kChunkSteps < nk ? kb0 + kChunkSteps : nk;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&sm->ready[s], ph)) {
+          if (!mbar_wait(presplit ? &sm->full[s] : &sm->ready[s], ph)) {
             give_up(sm, status);
             ok = false;
             break;
@@ -355,21 +370,34 @@ bool encode_tmap_3d(CUtensorMap* map, const float* base, int64_t cols, int64_t r
 
 }  // namespace
 
-nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_t ldp,
-                        int64_t strideP, const float* Q, int64_t ldq, int64_t strideQ,
-                        float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
-                        int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
-                        cudaStream_t st, double* C64) {
+namespace {
+
+nvfp4_status launch_gemm(int M, int N, int K, float alpha, const float* P, const float* Pl,
+                         int64_t ldp, int64_t strideP, const float* Q, const float* Ql,
+                         int64_t ldq, int64_t strideQ, float beta, float* C, int64_t ldc,
+                         int64_t strideC, float* C2, int64_t ldc2, int64_t strideC2, int batch,
+                         int lower, int* status, cudaStream_t st, double* C64) {
   if (M <= 0 || N <= 0 || batch <= 0) return NVFP4_OK;
   if (C2 && beta != 0.f) return NVFP4_ERR_INVALID_ARG;   // the transposed copy is alpha P Q^T
   if (C64 && (C2 || beta != 0.f)) return NVFP4_ERR_INVALID_ARG;
+  const int presplit = Pl != nullptr;
+  if (presplit != (Ql != nullptr)) return NVFP4_ERR_INVALID_ARG;
   if (((ldp | ldq | strideP | strideQ) & 3) != 0 ||
-      ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(Q)) & 15) != 0)
+      ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(Q) |
+        reinterpret_cast<uintptr_t>(Pl) | reinterpret_cast<uintptr_t>(Ql)) & 15) != 0)
     return NVFP4_ERR_INVALID_ARG;   // TMA: 16-byte aligned rows
-  CUtensorMap mp, mq;
+  CUtensorMap mp, mq, mpl, mql;
   if (!encode_tmap_3d(&mp, P, K, M, ldp, batch, strideP) ||
       !encode_tmap_3d(&mq, Q, K, N, ldq, batch, strideQ))
     return NVFP4_ERR_CUDA;
+  if (presplit) {
+    if (!encode_tmap_3d(&mpl, Pl, K, M, ldp, batch, strideP) ||
+        !encode_tmap_3d(&mql, Ql, K, N, ldq, batch, strideQ))
+      return NVFP4_ERR_CUDA;
+  } else {
+    mpl = mp;   // not read
+    mql = mq;
+  }
   TileSpace ts{(M + GM - 1) / GM, (N + GN - 1) / GN, batch, lower};
   const int per = lower ? ts.mt * (ts.mt + 1) / 2 : ts.mt * ts.nt;
   const int n_tiles = per * batch;
@@ -377,10 +405,33 @@ nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_nt_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   gemm_nt_tc_kernel<<<n_tiles < sms ? n_tiles : sms, kThreads, kSmem, st>>>(
-      mp, mq, C, ldc, strideC, C2, ldc2, strideC2, M, N, K, alpha, beta, ts, status, C64);
+      mp, mq, mpl, mql, presplit, C, ldc, strideC, C2, ldc2, strideC2, M, N, K, alpha, beta, ts,
+      status, C64);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;
+}
+
+}  // namespace
+
+nvfp4_status gemm_nt_tc(int M, int N, int K, float alpha, const float* P, int64_t ldp,
+                        int64_t strideP, const float* Q, int64_t ldq, int64_t strideQ,
+                        float beta, float* C, int64_t ldc, int64_t strideC, float* C2,
+                        int64_t ldc2, int64_t strideC2, int batch, int lower, int* status,
+                        cudaStream_t st, double* C64) {
+  return launch_gemm(M, N, K, alpha, P, nullptr, ldp, strideP, Q, nullptr, ldq, strideQ, beta, C,
+                     ldc, strideC, C2, ldc2, strideC2, batch, lower, status, st, C64);
+}
+
+nvfp4_status gemm_nt_tc_split(int M, int N, int K, float alpha, const float* Ph,
+                              const float* Pl, int64_t ldp, int64_t strideP, const float* Qh,
+                              const float* Ql, int64_t ldq, int64_t strideQ, float beta,
+                              float* C, int64_t ldc, int64_t strideC, float* C2, int64_t ldc2,
+                              int64_t strideC2, int batch, int lower, int* status,
+                              cudaStream_t st, double* C64) {
+  if (!Pl || !Ql) return NVFP4_ERR_INVALID_ARG;
+  return launch_gemm(M, N, K, alpha, Ph, Pl, ldp, strideP, Qh, Ql, ldq, strideQ, beta, C, ldc,
+                     strideC, C2, ldc2, strideC2, batch, lower, status, st, C64);
 }
 
 }  // namespace nvfp4

@@ -56,8 +56,6 @@ struct QuantLayout {
   float* Dl;       // d_out x S: remainder (delta - Dh)
   float* Uh;       // d_in x S: the super-batch's rows of U transposed, tf32 part
   float* Ul;       // d_in x S: remainder
-  float* D32;      // d_out x S: the deltas rounded to fp32 (super-batch update)
-  float* Ur;       // d_in x S: the rows of U transposed, fp32 (super-batch update)
   double* rowerr;  // d_out
 };
 
@@ -76,10 +74,6 @@ QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in) {
   L.Uh = reinterpret_cast<float*>(p + off);
   off += align256(sizeof(float) * L.S * d_in);
   L.Ul = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * L.S * d_in);
-  L.D32 = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d_out * L.S);
-  L.Ur = reinterpret_cast<float*>(p + off);
   off += align256(sizeof(float) * L.S * d_in);
   L.rowerr = reinterpret_cast<double*>(p + off);
   return L;
@@ -177,16 +171,15 @@ constexpr int kUTiles = kNb * (kNb + 1) / 2;        // upper 16x16 tiles of a ba
 __device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p) / 2 + q; }
 
 // The super-batch's rows k < nk of U, transposed (S values per row, K
-// contiguous: the updates' B operand), for the columns j >= j0: inside the
-// super-batch (j < send) split as Uh[j][k] + Ul[j][k] = U[cs + k][j] (tf32 part
-// and remainder) for the per-batch updates, beyond it as plain fp32 Ur[j][k]
-// for the super-batch update.  32 x 32 tiles transposed through shared memory.
+// contiguous: the updates' B operand), for the columns j >= j0, split as
+// Uh[j][k] + Ul[j][k] = U[cs + k][j] (tf32 part and remainder): the per-batch
+// updates read the super-batch's own columns, the super-batch update the
+// columns beyond it.  32 x 32 tiles transposed through shared memory.
 __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restrict__ U,
                                                            int64_t d_in, int64_t cs, int nk,
-                                                           int64_t j0, int64_t S, int64_t send,
+                                                           int64_t j0, int64_t S,
                                                            float* __restrict__ Uh,
-                                                           float* __restrict__ Ul,
-                                                           float* __restrict__ Ur) {
+                                                           float* __restrict__ Ul) {
   __shared__ float t[32][33];
   pdl_wait();
   const int64_t jb = j0 + (int64_t)blockIdx.x * 32;
@@ -201,13 +194,9 @@ __global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restri
     const int64_t j = jb + r;
     if (j < d_in && k0 + tx < nk) {
       const float u = t[tx][r];
-      if (j < send) {
-        const float h = sm100::tf32_rn(u);
-        Uh[j * S + k0 + tx] = h;
-        Ul[j * S + k0 + tx] = u - h;
-      } else {
-        Ur[j * S + k0 + tx] = u;
-      }
+      const float h = sm100::tf32_rn(u);
+      Uh[j * S + k0 + tx] = h;
+      Ul[j * S + k0 + tx] = u - h;
     }
   }
 }
@@ -289,7 +278,7 @@ __global__ void __launch_bounds__(kReplayThreads)
                               int64_t d_out, int64_t d_in, int c0, int bw,
                               const float* __restrict__ sg_ptr, uint8_t* __restrict__ codes,
                               uint8_t* __restrict__ scales, float* __restrict__ Dh,
-                              float* __restrict__ Dl, float* __restrict__ D32, int64_t ldD,
+                              float* __restrict__ Dl, int64_t ldD,
                               int kofs, double* __restrict__ rowerr) {
   extern __shared__ double4 smem_d4[];
   double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
@@ -453,7 +442,6 @@ __global__ void __launch_bounds__(kReplayThreads)
         const float h = sm100::tf32_rn((float)x);
         Dh[r * ldD + kofs + c] = h;
         Dl[r * ldD + kofs + c] = (float)(x - (double)h);
-        D32[r * ldD + kofs + c] = (float)x;
       }
       if (hl == 0) rowerr[r] += rowsum;
     }
@@ -490,7 +478,7 @@ constexpr size_t kReplaySmem =
 size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
   const int64_t S = super_width(d_in);
   return kWsHeader + align256(sizeof(double) * d_out * d_in) +
-         3 * align256(sizeof(float) * d_out * S) + 3 * align256(sizeof(float) * S * d_in) +
+         2 * align256(sizeof(float) * d_out * S) + 2 * align256(sizeof(float) * S * d_in) +
          align256(sizeof(double) * d_out);
 }
 
@@ -554,8 +542,8 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
       const int nk = (int)(send - cs);
       NVFP4_CUDA_TRY(launch_chained(split_u_rows_kernel,
                                     dim3((unsigned)((d_in - j0 + 31) / 32), (unsigned)((nk + 31) / 32)),
-                                    dim3(256), 0, st, U, (int64_t)d_in, cs, nk, j0, L.S, send,
-                                    L.Uh, L.Ul, L.Ur));
+                                    dim3(256), 0, st, U, (int64_t)d_in, cs, nk, j0, L.S,
+                                    L.Uh, L.Ul));
       count_launches(1);
     }
     for (int64_t c0 = cs; c0 < send; c0 += kLazyBatch) {
@@ -565,7 +553,7 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
         ProfileScope ps(kPhaseReplay, st);
         NVFP4_CUDA_TRY(launch_chained(replay_kernel, dim3(rgrid), dim3(kReplayThreads),
                                       kReplaySmem, st, L.Wt, U, d_out, d_in, (int)c0, bw, sg,
-                                      codes, scales, L.Dh, L.Dl, L.D32, L.S, kofs, L.rowerr));
+                                      codes, scales, L.Dh, L.Dl, L.S, kofs, L.rowerr));
         count_launches(1);
       }
       const int64_t e = c0 + bw;
@@ -579,13 +567,14 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
     }
     if (send < d_in) {
       // the whole super-batch's deltas into every later column, K = send - cs:
-      // the 3xTF32 GEMM engine (hi/lo split in shared memory, 128 x 128
+      // the 3xTF32 GEMM engine on the deltas' and U's hi/lo parts (128 x 128
       // tiles, 128-deep partials summed in fp32 registers), added to the fp64
       // working copy in its epilogue
       ProfileScope ps(kPhaseUpdate, st);
-      nvfp4_status s = gemm_nt_tc((int)d_out, (int)(d_in - send), (int)(send - cs), -1.f,
-                                  L.D32, L.S, 0, L.Ur + send * L.S, L.S, 0, 0.f, nullptr, d_in,
-                                  0, nullptr, 0, 0, 1, 0, &L.hdr->status, st, L.Wt + send);
+      nvfp4_status s = gemm_nt_tc_split(
+          (int)d_out, (int)(d_in - send), (int)(send - cs), -1.f, L.Dh, L.Dl, L.S, 0,
+          L.Uh + send * L.S, L.Ul + send * L.S, L.S, 0, 0.f, nullptr, d_in, 0, nullptr, 0, 0, 1,
+          0, &L.hdr->status, st, L.Wt + send);
       if (s != NVFP4_OK) return s;
     }
   }
