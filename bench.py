@@ -32,9 +32,18 @@ DEFAULT_WORKLOAD = "attn_massive_4096x4096"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 N_SM = 148
-N_PHASES = 8                # the library's profiling phases (nvfp4pw.h)
+N_PHASES = 9                # the library's profiling phases (nvfp4pw.h)
 E2E_CHUNK_TOK = 1024        # tokens per host-to-device chunk of the end-to-end step
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor rates
+INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
+# DRAM bytes (read + write) of one launch of a phase's kernel, from an ncu --set
+# full capture of the current kernel source (this script with --steps 1
+# --warmup 0 --no-cpu-baseline, the launch named); a phase without an entry
+# reports null, and an entry is dropped when its kernel changes
+NCU_TRAFFIC = {
+    "panel": {"bytes": 1.823e6, "launch": "chol_panel_kernel, panel 11 of 64 (3328 rows below)"},
+}
+I8_PAIRS = 28               # int8 slice products per fp64 MAC in the int8-slice GEMM (7 slices)
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
 FP32_LANES_PER_SM = 128
 
@@ -263,16 +272,18 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     wk = phase_work(d_out, d_in, n_tok)
     names = ["hessian", "prepare", "replay", "update", "dequant", "other", "factor_gemm",
-             "panel"]
+             "panel", "factor_i8"]
     ph_ms = {n: ms_ph[i] / args.steps for i, n in enumerate(names) if n != "other"}
     ph_launch = {n: ln_ph[i] // args.steps for i, n in enumerate(names)}
     sm_ghz = peaks.get("sm_max_mhz", 1965.0) / 1e3
     fp64_peak = N_SM * FP64_LANES_PER_SM * 2 * sm_ghz / 1e3    # TFLOP/s, derived
     bf16_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])   # inside a long step
     tf32_peak = bf16_peak * TF32_PER_BF16                        # nominal dense ratio
+    int8_peak = bf16_peak * INT8_PER_BF16                        # nominal dense ratio
     hbm = peaks["hbm_gbs"]
     gemm_flops = wk_ph[6] / args.steps          # counted by the launcher from the shapes
     panel_flops = wk_ph[7] / args.steps
+    i8_flops = wk_ph[8] / args.steps            # fp64-equivalent flops of the int8-slice GEMMs
     # per-kernel roofline (what bounds each kernel group in this build); the
     # prepare phase is the panel kernels plus the fp64 GEMMs
     rl = {
@@ -280,10 +291,17 @@ def run_ours(args, rank, world, local_rank):
                     "TFLOP/s", "hessian_tc_kernel (tcgen05 kind::f16)",
                     "measured bf16 sustained"),
         "factor_gemm": ("tensor", gemm_flops / (ph_ms["factor_gemm"] * 1e9), fp64_peak,
-                        "TFLOP/s", "dgemm_nt_kernel (fp64 mma.sync m8n8k4, TMA-fed)",
+                        "TFLOP/s", "dgemm_nt_kernel (fp64 mma.sync m8n8k4, TMA-fed; narrow "
+                        "in-block updates)",
                         "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock"),
-        "panel": ("latency", panel_flops / (ph_ms["panel"] * 1e9), fp64_peak, "TFLOP/s",
-                  "chol_panel_kernel (serial 64-pivot chain per panel)",
+        "factor_i8": ("tensor", I8_PAIRS * i8_flops / (ph_ms["factor_i8"] * 1e9), int8_peak,
+                      "TFLOP/s", "dgemm_i8_kernel + slice_rows_kernel (fp64-accurate GEMM on "
+                      "tcgen05 kind::i8; achieved counts the int8 ops: 28 slice products per "
+                      "fp64 MAC)",
+                      "measured bf16 sustained x nominal int8/bf16 ratio"),
+        "panel": ("alu", panel_flops / (ph_ms["panel"] * 1e9), fp64_peak, "TFLOP/s",
+                  "chol_panel_kernel (fp64; bound by its serial 64-pivot chain per panel, "
+                  "not by the fp64 rate)",
                   "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock"),
         "update": ("tensor", 3 * wk["update_flops"] / (ph_ms["update"] * 1e9), tf32_peak,
                    "TFLOP/s", "update_tc_kernel (tcgen05 kind::tf32, 3 products per MAC)",
@@ -303,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": job_throughput(world, weights, step_ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in; f32 H; f64 factor (U stored f32); f64 working copy and replay; 3xTF32 update", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16 in; f32 H; f64-accurate factor (int8-slice tensor cores + fp64 mma; U stored f32); f64 working copy and replay; 3xTF32 update", "data": "synthetic",
         "config": {"workload": args.workload, "d_out": d_out, "d_in": d_in, "n_tok": n_tok,
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
                    "parallelism": f"{world} independent layer solves (one per GPU)"},
@@ -316,7 +334,9 @@ def run_ours(args, rank, world, local_rank):
                                "kernels": k_, "peak_source": src}
                            for n, (b, a, p, u, k_, src) in rl.items()},
         "roofline": {"phase": dom, "kernel": kern, "bound": bound, "achieved": ach, "peak": peak,
-                     "unit": unit, "frac": ach / peak, "traffic": None,
+                     "unit": unit, "frac": ach / peak,
+                     "traffic": NCU_TRAFFIC.get(dom, {}).get("bytes"),
+                     "traffic_launch": NCU_TRAFFIC.get(dom, {}).get("launch"),
                      "peak_source": f"{peak_src[dom]} ({peaks['source']})"},
         "e2e": {"value": job_throughput(world, weights, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": W.numel() * W.element_size() + X.numel() * X.element_size(),

@@ -387,9 +387,11 @@ enum {
   NVFP4_PHASE_UPDATE = 3,  /* trailing-update GEMMs of the quantize call    */
   NVFP4_PHASE_DEQUANT = 4, /* nvfp4_dequant                                 */
   NVFP4_PHASE_OTHER = 5,   /* everything else (prologues, reductions)       */
-  NVFP4_PHASE_FACTOR_GEMM = 6, /* inside PREPARE: its fp64 GEMM launches     */
+  NVFP4_PHASE_FACTOR_GEMM = 6, /* inside PREPARE: its fp64 mma.sync GEMMs   */
   NVFP4_PHASE_PANEL = 7,   /* inside PREPARE: its Cholesky panel launches  */
-  NVFP4_NUM_PHASES = 8
+  NVFP4_PHASE_FACTOR_I8 = 8, /* inside PREPARE: its int8-slice GEMMs (with
+                                their slicing launches); work = fp64 flops */
+  NVFP4_NUM_PHASES = 9
 };
 
 /* Starts a profiling window: from now on every phase above records a CUDA

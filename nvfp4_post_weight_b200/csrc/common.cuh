@@ -36,7 +36,8 @@ enum Phase {
   kPhaseOther = 5,
   kPhaseFactorGemm = 6,   // sub-phases of kPhasePrepare
   kPhasePanel = 7,
-  kNumPhases = 8
+  kPhaseFactorI8 = 8,
+  kNumPhases = 9
 };
 // While profiling is on, adds algorithmic work (flops) to the open phase.
 void add_phase_work(double work);

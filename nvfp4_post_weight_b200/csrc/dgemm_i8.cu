@@ -531,7 +531,7 @@ nvfp4_status dgemm_i8(int M, int N, int K, double alpha, const double* P, int64_
       K >= (1 << 16) || (K % 16) != 0 || batch > 65535)
     return NVFP4_ERR_INVALID_ARG;
   if (scratch_bytes < dgemm_i8_scratch_bytes(M, N, K, batch)) return NVFP4_ERR_WORKSPACE;
-  ProfileScope ps(kPhaseFactorGemm, st);
+  ProfileScope ps(kPhaseFactorI8, st);
   {
     double f = 2.0 * M * N * K;
     if (lower) f = 2.0 * ((double)N * (N + 1) / 2) * K;
