@@ -194,27 +194,23 @@ __device__ __forceinline__ void factor_16(double (*S)[kPitch], double* invd, int
 // One warp, lanes 0..15 meaningful: column i of inv(L_KK) for the factored
 // block at (o, o) of S, by right-looking forward substitution (each x[m]
 // updates the later sums at once, so the serial chain is one fma per m),
-// written into the same block of Xd (lower, zeros above).
+// written into the same block of Xd (lower, zeros above).  L[n][m] is read
+// from shared memory (the same address in every lane: a broadcast), not
+// passed between lanes.
 __device__ __forceinline__ void invert_16(double (*S)[kPitch], double (*Xd)[kPitch],
                                           const double* invd, int o) {
-  const int lane = threadIdx.x & 31;
-  const int i = lane & 15;
-  const unsigned full = 0xffffffffu;
-  double r[kSub], x[kSub], acc[kSub];
+  const int i = threadIdx.x & 15;
+  double x[kSub], acc[kSub];
 #pragma unroll
-  for (int l = 0; l < kSub; ++l) {
-    r[l] = (l <= i) ? S[o + i][o + l] : 0.0;
-    acc[l] = 0.0;
-  }
+  for (int l = 0; l < kSub; ++l) acc[l] = 0.0;
 #pragma unroll
   for (int m = 0; m < kSub; ++m) {
     const double id = invd[o + m];
     x[m] = m < i ? 0.0 : (m == i ? id : -acc[m] * id);
 #pragma unroll
-    for (int n = m + 1; n < kSub; ++n)
-      acc[n] = fma(__shfl_sync(full, r[m], n, 16), x[m], acc[n]);   // L[n][m] x[m]
+    for (int n = m + 1; n < kSub; ++n) acc[n] = fma(S[o + n][o + m], x[m], acc[n]);
   }
-  if (lane < kSub) {
+  if ((threadIdx.x & 31) < kSub) {
 #pragma unroll
     for (int l = 0; l < kSub; ++l) Xd[o + l][o + i] = x[l];   // column i of the inverse
   }
@@ -369,13 +365,23 @@ __global__ void __launch_bounds__(kPanelThreads)
   if (blockIdx.x == 0) {
     // L11 itself is not written back: nothing reads the diagonal blocks of L
     // later, and the other CTAs of this launch may still be reading A11.
-    for (int idx = tid; idx < kb * kb; idx += kPanelThreads) {
-      const int i = idx / kb, j = idx % kb;
-      X[(k + i) * d + k + j] = Xd[i][j];   // lower (zeros above), row by row
+    // X11 (lower, zeros above) and its transpose into Y, row by row; all
+    // shared-memory reads of a thread before its stores, no division
+    constexpr int kPer = NB * NB / kPanelThreads;   // 16
+    double xv[kPer], yv[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx >> 6, j = idx & (NB - 1);
+      xv[q] = Xd[i][j];
+      yv[q] = Xd[j][i];   // Y[i][j] = X[j][i]
     }
-    for (int idx = tid; idx < kb * kb; idx += kPanelThreads) {
-      const int j = idx / kb, i = idx % kb;
-      Y[(k + j) * d + k + i] = Xd[i][j];   // its transpose, upper, row by row
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kPanelThreads, i = idx >> 6, j = idx & (NB - 1);
+      if (i < kb && j < kb) {
+        X[(k + i) * d + k + j] = xv[q];
+        Y[(k + i) * d + k + j] = yv[q];
+      }
     }
     return;
   }
