@@ -231,7 +231,8 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the C ABI from pinned host buffers: the tokens stream
     # from host memory into the Hessian in 1024-token chunks, W is copied
-    # beside the prepare, then the solve; D2H of codes, scales and s_g
+    # beside the prepare, then the solve; D2H of codes, scales and s_g beside
+    # dequant and the layer error, waited for before the step's end event
     Wh, Xh = W.pin_memory(), X.pin_memory()
     W_e2e = torch.empty_like(Wd)
     codes_h = torch.empty(solver.codes.shape, dtype=torch.uint8).pin_memory()
@@ -239,10 +240,8 @@ def run_ours(args, rank, world, local_rank):
     sg_h = torch.empty(1, dtype=torch.float32).pin_memory()
 
     def e2e_step():
-        solver.step_host(Wh, Xh, W_e2e, chunk_tok=E2E_CHUNK_TOK)
-        codes_h.copy_(solver.codes, non_blocking=True)
-        scales_h.copy_(solver.scales, non_blocking=True)
-        sg_h.copy_(solver.s_g, non_blocking=True)
+        solver.step_host(Wh, Xh, W_e2e, chunk_tok=E2E_CHUNK_TOK,
+                         out_host=(codes_h, scales_h, sg_h))
 
     e2e_step()
     torch.cuda.synchronize()

@@ -76,25 +76,46 @@ class LayerSolver:
             self._ws_host_key = key
         B.nvfp4_hessian_accumulate_host(self.H, X_host, chunk_tok, self.ws_host, beta, stream)
 
-    def step_host(self, W_host, X_host, W_dev, chunk_tok=1024, stream=None, with_error=True):
+    def step_host(self, W_host, X_host, W_dev, chunk_tok=1024, stream=None, with_error=True,
+                  out_host=None):
         """One whole solve from host-resident inputs: the tokens stream into the
-        Hessian chunk by chunk, and W is copied into W_dev on a side stream while
-        the factor is prepared (quantize waits for it)."""
+        Hessian chunk by chunk; W is copied into W_dev on a side stream once the
+        last token chunk is on the device (so the two copies do not share the
+        host link while the Hessian waits), beside the prepare; quantize waits
+        for it.  With out_host = (codes_h, scales_h, s_g_h) (pinned host
+        tensors) the codes, scales and global scale are read back on the side
+        stream as soon as quantize has written them, beside dequant and the
+        layer error; the caller's stream waits for that read-back at the end."""
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         if not hasattr(self, "_side"):
             self._side = torch.cuda.Stream(self.device)
+            self._x_done = torch.cuda.Event()
             self._w_ready = torch.cuda.Event()
-        self._side.wait_stream(st)          # W_dev is free once earlier work on st is done
+            self._q_done = torch.cuda.Event()
+            self._d2h_done = torch.cuda.Event()
+        self.hessian_host(X_host, chunk_tok, 0, st)
+        self._x_done.record(st)           # all tokens are on the device (and W_dev is free)
+        self._side.wait_event(self._x_done)
         with torch.cuda.stream(self._side):
             W_dev.copy_(W_host, non_blocking=True)
             self._w_ready.record(self._side)
-        self.hessian_host(X_host, chunk_tok, 0, st)
         self.prepare(st)
         st.wait_event(self._w_ready)
         self.quantize(W_dev, st)
+        if out_host is not None:
+            self._q_done.record(st)
+            self._side.wait_event(self._q_done)
+            with torch.cuda.stream(self._side):
+                codes_h, scales_h, sg_h = out_host
+                codes_h.copy_(self.codes, non_blocking=True)
+                scales_h.copy_(self.scales, non_blocking=True)
+                sg_h.copy_(self.s_g, non_blocking=True)
+                self._d2h_done.record(self._side)
         self.dequant(st)
         if with_error:
             self.layer_error(W_dev, st)
+        if out_host is not None:
+            st.wait_event(self._d2h_done)
 
     def status(self, stream=None):
         """Device status words of the prepare and quantize workspaces."""

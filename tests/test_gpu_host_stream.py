@@ -90,8 +90,15 @@ def test_solve_from_host_inputs_equals_device_solve():
     dev_solver.step(W.to(DEV), X.to(DEV))
     host_solver = LayerSolver(d_out, d_in, DEV, out_dtype=torch.bfloat16)
     W_dev = torch.empty((d_out, d_in), dtype=W.dtype, device=DEV)
-    host_solver.step_host(W.pin_memory(), X.pin_memory(), W_dev, chunk_tok=1024)
+    out_h = (torch.empty((d_out, d_in // 2), dtype=torch.uint8).pin_memory(),
+             torch.empty((d_out, d_in // 16), dtype=torch.uint8).pin_memory(),
+             torch.empty(1, dtype=torch.float32).pin_memory())
+    host_solver.step_host(W.pin_memory(), X.pin_memory(), W_dev, chunk_tok=1024, out_host=out_h)
     torch.cuda.synchronize()
+    # the read-back on the side stream holds the quantize's outputs
+    assert torch.equal(out_h[0], host_solver.codes.cpu())
+    assert torch.equal(out_h[1], host_solver.scales.cpu())
+    assert out_h[2].item() == host_solver.s_g.item()
     assert dev_solver.status() == (0, 0) and host_solver.status() == (0, 0)
     assert torch.equal(W_dev.cpu(), W)
     assert rel_frob(host_solver.H.cpu().numpy(), dev_solver.H.cpu().numpy()) < 1e-6
