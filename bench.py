@@ -43,7 +43,7 @@ INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
 NCU_TRAFFIC = {
     "panel": {"bytes": 1.823e6, "launch": "chol_panel_kernel, panel 11 of 64 (3328 rows below)"},
 }
-I8_PAIRS = 28               # int8 slice products per fp64 MAC in the int8-slice GEMM (7 slices)
+I8_PAIRS = 21               # int8 slice products per fp64 MAC in the int8-slice GEMM (6 slices)
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
 FP32_LANES_PER_SM = 128
 
@@ -295,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
                         "derived fp64: 148 SMs x 64 lanes x 2 x max SM clock"),
         "factor_i8": ("tensor", I8_PAIRS * i8_flops / (ph_ms["factor_i8"] * 1e9), int8_peak,
                       "TFLOP/s", "dgemm_i8_kernel + slice_rows_kernel (fp64-accurate GEMM on "
-                      "tcgen05 kind::i8; achieved counts the int8 ops: 28 slice products per "
+                      "tcgen05 kind::i8; achieved counts the int8 ops: 21 slice products per "
                       "fp64 MAC)",
                       "measured bf16 sustained x nominal int8/bf16 ratio"),
         "panel": ("alu", panel_flops / (ph_ms["panel"] * 1e9), fp64_peak, "TFLOP/s",
