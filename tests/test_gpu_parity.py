@@ -172,7 +172,10 @@ def test_prepare_factor(d):
     Ug = U.cpu().numpy().astype(np.float64)
     assert np.all(np.tril(Ug, -1) == 0.0)
     assert np.all(np.diag(Ug) > 0)
-    assert rel_frob(Ug, Uref) < 1e-4
+    # as close to the fp64 factor as fp32 storage allows: within 1.5x the
+    # error of rounding the oracle's own U to fp32 (measured 1.04x)
+    r32 = rel_frob(Uref.astype(np.float32).astype(np.float64), Uref)
+    assert rel_frob(Ug, Uref) <= 1.5 * r32
     assert abs(lam.item() - lam_ref) <= 1e-6 * lam_ref
     assert not dead.cpu().numpy().any()
 
