@@ -41,7 +41,7 @@ INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
 # --warmup 0 --no-cpu-baseline, the launch named); a phase without an entry
 # reports null, and an entry is dropped when its kernel changes
 NCU_TRAFFIC = {
-    "panel": {"bytes": 1.823e6, "launch": "chol_panel_kernel, panel 11 of 64 (3328 rows below)"},
+    "panel": {"bytes": 1.824e6, "launch": "chol_panel_kernel, panel 11 of 64 (3328 rows below)"},
 }
 I8_PAIRS = 21               # int8 slice products per fp64 MAC in the int8-slice GEMM (6 slices)
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
