@@ -106,19 +106,34 @@ __global__ void __launch_bounds__(256)
 }
 
 // sum_ij H_ij G_ij in fp64 with G = E^T E known on the 128 x 128 tiles on or
-// below the diagonal only (the tile size of gemm_nt_tc's lower mode): by the symmetry of G and H an off-diagonal tile
-// stands for its mirror image too (weight 2), a diagonal tile for itself.
-// Rows are shared out over the CTAs; tiles above the diagonal are not read.
+// below the diagonal only (the tile size of gemm_nt_tc's lower mode): by the
+// symmetry of G and H an off-diagonal tile stands for its mirror image too
+// (weight 2), a diagonal tile for itself.  Rows are shared out over the CTAs;
+// tiles above the diagonal are not read.  Four consecutive columns per thread
+// and step (d and the tile edges are multiples of 4), read as float4 when H
+// is 16-byte aligned (vec; G is workspace), so that several loads are in
+// flight per thread.
 __global__ void sym_tile_dot_kernel(const float* __restrict__ H, const float* __restrict__ G,
-                                    int64_t d, double* __restrict__ partial) {
+                                    int64_t d, double* __restrict__ partial, int vec) {
   __shared__ double part[32];
   double s = 0.0;
   for (int64_t i = blockIdx.x; i < d; i += gridDim.x) {
     const int64_t jdiag = (i / 128) * 128;
     const int64_t jend = (jdiag + 128) < d ? (jdiag + 128) : d;
-    for (int64_t j = threadIdx.x; j < jend; j += blockDim.x) {
-      const double hg = (double)H[i * d + j] * (double)G[i * d + j];
-      s += j < jdiag ? 2.0 * hg : hg;
+    const float* hr = H + i * d;
+    const float* gr = G + i * d;
+#pragma unroll 2
+    for (int64_t j = 4 * (int64_t)threadIdx.x; j < jend; j += 4 * (int64_t)blockDim.x) {
+      float4 h;
+      if (vec) {
+        h = *reinterpret_cast<const float4*>(hr + j);
+      } else {
+        h = make_float4(hr[j], hr[j + 1], hr[j + 2], hr[j + 3]);
+      }
+      const float4 g = *reinterpret_cast<const float4*>(gr + j);
+      const double t = (double)h.x * (double)g.x + (double)h.y * (double)g.y +
+                       (double)h.z * (double)g.z + (double)h.w * (double)g.w;
+      s += j < jdiag ? 2.0 * t : t;   // the four share a side: jdiag is a multiple of 4
     }
   }
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -131,12 +146,12 @@ __global__ void sym_tile_dot_kernel(const float* __restrict__ H, const float* __
   }
 }
 
+// The partial sums added by one warp in a fixed order (deterministic).
 __global__ void sum_partials_kernel(const double* __restrict__ p, int n, double* __restrict__ out) {
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < n; ++i) s += p[i];
-    *out = s;
-  }
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += 32) s += p[i];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (threadIdx.x == 0) *out = s;
 }
 
 // Export of the block scales into 128-row x 4-column tiles of 512 bytes (the
@@ -161,7 +176,7 @@ int grid_for(int64_t n, int threads) {
   return (int)(b < 8 * kNumSMs ? (b < 1 ? 1 : b) : 8 * kNumSMs);
 }
 
-constexpr int kDotBlocks = 2 * kNumSMs;
+constexpr int kDotBlocks = 8 * kNumSMs;
 
 }  // namespace
 
@@ -237,7 +252,8 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
   nvfp4_status s = gemm_nt_tc_split((int)d_in, (int)d_in, (int)d_out, 1.f, Eh, El, ldE, 0, Eh,
                                     El, ldE, 0, 0.f, G, d_in, 0, nullptr, 0, 0, 1, 1, status, st);
   if (s != NVFP4_OK) return s;
-  sym_tile_dot_kernel<<<kDotBlocks, 256, 0, st>>>(H, G, d_in, part);
+  sym_tile_dot_kernel<<<kDotBlocks, 256, 0, st>>>(H, G, d_in, part,
+                                                  (reinterpret_cast<uintptr_t>(H) & 15) == 0);
   NVFP4_LAUNCH_CHECK();
   sum_partials_kernel<<<1, 32, 0, st>>>(part, kDotBlocks, err);
   NVFP4_LAUNCH_CHECK();

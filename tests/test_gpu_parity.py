@@ -314,6 +314,32 @@ def test_quantize_errors():
 # --------------------------------------------------------------------------
 # whole solve: small layer bit-exact, full-size layer on a row sample
 # --------------------------------------------------------------------------
+def test_layer_error_unaligned_h_equals_aligned():
+    """H at a 4-byte offset (no 16-byte alignment) takes the element-wise
+    path of the weighted dot: the same sum, bit for bit, and the oracle's
+    layer error of the same codes within 1e-6."""
+    W, X = synth.small_outlier(d_out=96, d_in=256, n_tok=512, seed=4)
+    s = gpu_solve(W, X)
+    d_out, d_in = W.shape
+    Wd = W.to(DEV)
+    Hbuf = torch.empty(d_in * d_in + 1, dtype=torch.float32, device=DEV)
+    Hu = Hbuf[1:].view(d_in, d_in)
+    Hu.copy_(s.H)
+    assert Hu.data_ptr() % 16 != 0
+    ws = B.workspace(B.nvfp4_layer_error_workspace_size(d_out, d_in), DEV)
+    e_al = torch.empty(1, dtype=torch.float64, device=DEV)
+    e_un = torch.empty(1, dtype=torch.float64, device=DEV)
+    B.nvfp4_layer_error(Wd, s.codes, s.scales, s.s_g, s.H, e_al, ws)
+    B.nvfp4_layer_error(Wd, s.codes, s.scales, s.s_g, Hu, e_un, ws)
+    torch.cuda.synchronize()
+    assert e_al.item() == e_un.item()
+    codes = unpack_codes(s.codes.cpu().numpy())
+    scales = s.scales.cpu().numpy().astype(np.int64)
+    Q = O.dequant(codes, scales, np.float32(s.s_g.item())).astype(np.float64)
+    L = O.layer_error(W.double().numpy(), Q, s.H.cpu().numpy().astype(np.float64))
+    assert abs(e_al.item() - L) <= 1e-6 * L
+
+
 def test_solve_small_outlier_bitexact():
     W, X = synth.small_outlier()
     ref = O.solve_layer(W.double().numpy(), X.double().numpy())
