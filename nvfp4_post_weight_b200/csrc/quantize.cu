@@ -24,8 +24,11 @@
 // replay kernel walks the batch's 8 blocks for every row (a half-warp per row,
 // lane = candidate scale) with the row's 128 batch values in shared memory,
 // and applies each chosen block's deltas to the rest of the batch; it writes
-// the batch's deltas.  The trailing update then applies the whole batch to
-// every later column at once: W~[:, e:] -= Delta U[batch, e:].
+// the batch's deltas as tf32 hi/lo pairs.  The trailing update W~[:, e:] -=
+// Delta U[batch, e:] is two-level (super_width below): each batch updates
+// the rest of its super-batch at once (update_tc), and each super-batch
+// updates every column beyond it with K = 1024 (the 3xTF32 GEMM on the same
+// hi/lo pairs of Delta and of U's rows).
 #include <math.h>
 
 #include "common.cuh"
