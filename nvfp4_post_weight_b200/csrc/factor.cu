@@ -466,11 +466,6 @@ PrepLayout prep_layout(void* ws, int64_t d) {
   return L;
 }
 
-int grid_for(int64_t n, int threads) {
-  int64_t b = (n + threads - 1) / threads;
-  return (int)(b < 8 * kNumSMs ? (b < 1 ? 1 : b) : 8 * kNumSMs);
-}
-
 }  // namespace
 
 size_t prepare_ws_bytes(int64_t d) {

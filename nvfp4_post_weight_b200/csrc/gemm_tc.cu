@@ -258,7 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;
     const int h = (warp - 6) >> 2;      // column half of the tile
     int g = 0;
     bool ok = true;
