@@ -158,6 +158,12 @@ nvfp4_status nvfp4_hessian_status(nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* a2-a4  damping + upper Cholesky factor of the damped inverse              */
+/* "Replay the Curvature", Abstract, sentence on why the scale choice is     */
+/* hard in GPTQ: quantizing a column updates the columns after it; the       */
+/* update weights are the rows of U, the upper factor of the damped inverse  */
+/* Hessian (H_d^-1 = U^T U), and 1 / U_jj^2 is the Schur complement that the  */
+/* Schur Replay score weights each column's error with (Abstract, sentence   */
+/* introducing Schur Replay).                                                */
 /* ------------------------------------------------------------------------ */
 /* Bytes of workspace nvfp4_gptq_prepare needs for dimension d. */
 size_t nvfp4_prepare_workspace_size(int64_t d);
@@ -179,6 +185,11 @@ nvfp4_status nvfp4_gptq_prepare(const float* H, int64_t d, float damp, float* U,
 
 /* ------------------------------------------------------------------------ */
 /* a5-a8  GPTQ with Schur Replay block-scale selection                       */
+/* "Replay the Curvature", Abstract: the NVFP4 sentence (16 E2M1 codes per   */
+/* block under one E4M3 scale), the sentence on why the scale choice is hard */
+/* in GPTQ (column-sequential updates) and the sentence introducing Schur    */
+/* Replay (each candidate scale scored by replaying the in-block GPTQ        */
+/* updates it causes, after compensation by the unquantized columns).        */
 /* ------------------------------------------------------------------------ */
 /* Bytes of workspace nvfp4_gptq_schur_replay_quantize needs. */
 size_t nvfp4_quantize_workspace_size(int64_t d_out, int64_t d_in,
@@ -231,7 +242,10 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize(
  *   - The device current on the calling thread must be the stream's device.
  *     The first call on a device looks up the array's device address (once
  *     per device, under a lock); make that first call before any stream
- *     capture.
+ *     capture.  Under CUDA's lazy module loading (the default) that first
+ *     call is also when the library's module holding the array is loaded on
+ *     the device, i.e. when the driver reserves its 16 MiB there; later calls
+ *     reserve nothing.
  *   - All calls on one device share the array and it keeps the previous
  *     call's contents (the call clears what must start at zero itself).  Calls
  *     whose GPU work overlaps, e.g. on two streams without ordering, race and

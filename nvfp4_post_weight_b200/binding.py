@@ -24,9 +24,10 @@ _STATUS = {
 
 
 class Nvfp4Error(RuntimeError):
-    def __init__(self, call, code):
+    def __init__(self, call, code, detail=None):
         self.code = int(code)
-        super().__init__(f"{call}: status {code} ({_STATUS.get(int(code), 'unknown')})")
+        msg = f"{call}: status {code} ({_STATUS.get(int(code), 'unknown')})"
+        super().__init__(msg if detail is None else f"{msg}: {detail}")
 
 
 class SolveParams(ctypes.Structure):
@@ -110,6 +111,67 @@ def _check(call, code):
         raise Nvfp4Error(call, code)
 
 
+NVFP4_ERR_INVALID_ARG = 1
+
+
+def _need(call, t, name, shape=None, dtype=None, numel_min=None, device=True):
+    """Host-side check of one tensor argument before the library is called:
+    present, contiguous, on a CUDA device (or the host, device=False), of the
+    given dtype and shape (or at least numel_min elements).  A mismatch would
+    otherwise become an out-of-bounds device access, so it raises
+    Nvfp4Error(call, NVFP4_ERR_INVALID_ARG)."""
+    def bad(why):
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, f"{name}: {why}")
+    if t is None:
+        bad("missing")
+    if not isinstance(t, torch.Tensor):
+        bad(f"not a tensor ({type(t).__name__})")
+    if device and not t.is_cuda:
+        bad("not a CUDA tensor")
+    if not device and t.is_cuda:
+        bad("must be a host tensor")
+    if not t.is_contiguous():
+        bad("not contiguous")
+    if dtype is not None:
+        dts = dtype if isinstance(dtype, tuple) else (dtype,)
+        if t.dtype not in dts:
+            bad(f"dtype {t.dtype}, expected {' or '.join(str(d) for d in dts)}")
+    if shape is not None and tuple(t.shape) != tuple(int(v) for v in shape):
+        bad(f"shape {tuple(t.shape)}, expected {tuple(int(v) for v in shape)}")
+    if numel_min is not None and t.numel() < numel_min:
+        bad(f"{t.numel()} elements, expected at least {numel_min}")
+    return t
+
+
+def _opt_need(call, t, name, **kw):
+    return None if t is None else _need(call, t, name, **kw)
+
+
+def _matrix(call, t, name, dtype=None, device=True):
+    _need(call, t, name, dtype=dtype, device=device)
+    if t.dim() != 2:
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, f"{name}: expected a matrix")
+    return t.shape
+
+
+_IO_DTYPES = (torch.bfloat16, torch.float32)
+_U8, _F32, _F64, _I32 = torch.uint8, torch.float32, torch.float64, torch.int32
+
+
+def _check_solve_outputs(call, d_out, d_in, codes, scales, global_scale, err_out):
+    _need(call, codes, "codes", (d_out, d_in // 2), _U8)
+    _need(call, scales, "scales", (d_out, d_in // 16), _U8)
+    _need(call, global_scale, "global_scale", (1,), _F32)
+    _opt_need(call, err_out, "err_out", shape=(1,), dtype=_F64)
+
+
+def _ws_bytes(call, ws, need):
+    """Workspace tensor: a contiguous uint8 CUDA tensor of at least `need`
+    bytes (the library also checks its size and alignment)."""
+    _need(call, ws, "workspace", dtype=_U8, numel_min=need)
+    return ws.numel()
+
+
 def _dtype_code(t):
     if t.dtype == torch.bfloat16:
         return NVFP4_BF16
@@ -155,19 +217,20 @@ def nvfp4_hessian_host_workspace_size(d, chunk_tok, dtype=torch.bfloat16) -> int
 def nvfp4_hessian_accumulate_host(H, X_host, chunk_tok, ws, beta=0, stream=None):
     """H (device) (+)= X_host^T X_host with X_host a CPU tensor (pinned for
     overlap), streamed in chunks of chunk_tok tokens through ws."""
-    if X_host.is_cuda:
-        raise ValueError("X_host must be a host (CPU) tensor")
-    if not X_host.is_contiguous():
-        raise ValueError("X_host must be contiguous")
-    n_tok, d = X_host.shape
-    _check("nvfp4_hessian_accumulate_host", lib().nvfp4_hessian_accumulate_host(
+    call = "nvfp4_hessian_accumulate_host"
+    n_tok, d = _matrix(call, X_host, "X_host", _IO_DTYPES, device=False)
+    _need(call, H, "H", (d, d), _F32)
+    nws = _ws_bytes(call, ws, nvfp4_hessian_host_workspace_size(d, chunk_tok, X_host.dtype))
+    _check(call, lib().nvfp4_hessian_accumulate_host(
         _ptr(H), ctypes.c_void_p(X_host.data_ptr()), _dtype_code(X_host), n_tok, d, int(beta),
-        int(chunk_tok), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        int(chunk_tok), _ptr(ws), nws, _stream(stream)))
 
 
 def nvfp4_hessian_accumulate(H, X, beta=0, stream=None):
-    n_tok, d = X.shape
-    _check("nvfp4_hessian_accumulate", lib().nvfp4_hessian_accumulate(
+    call = "nvfp4_hessian_accumulate"
+    n_tok, d = _matrix(call, X, "X", _IO_DTYPES)
+    _need(call, H, "H", (d, d), _F32)
+    _check(call, lib().nvfp4_hessian_accumulate(
         _ptr(H), _ptr(X), _dtype_code(X), n_tok, d, int(beta), _stream(stream)))
 
 
@@ -180,10 +243,16 @@ def nvfp4_prepare_workspace_size(d) -> int:
 
 
 def nvfp4_gptq_prepare(H, damp, U, dead=None, lambda_out=None, ws=None, stream=None):
-    d = H.shape[0]
-    _check("nvfp4_gptq_prepare", lib().nvfp4_gptq_prepare(
-        _ptr(H), d, float(damp), _ptr(U), _ptr(dead), _ptr(lambda_out), _ptr(ws),
-        0 if ws is None else ws.numel(), _stream(stream)))
+    call = "nvfp4_gptq_prepare"
+    d, d2 = _matrix(call, H, "H", _F32)
+    _need(call, H, "H", (d, d))
+    _need(call, U, "U", (d, d), _F32)
+    _opt_need(call, dead, "dead", shape=(d,), dtype=_U8)
+    _opt_need(call, lambda_out, "lambda_out", shape=(1,), dtype=_F32)
+    nws = _ws_bytes(call, ws, nvfp4_prepare_workspace_size(d))
+    _check(call, lib().nvfp4_gptq_prepare(
+        _ptr(H), d, float(damp), _ptr(U), _ptr(dead), _ptr(lambda_out), _ptr(ws), nws,
+        _stream(stream)))
 
 
 def nvfp4_quantize_workspace_size(d_out, d_in, params=None) -> int:
@@ -193,12 +262,17 @@ def nvfp4_quantize_workspace_size(d_out, d_in, params=None) -> int:
 
 def nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, global_scale, err_out=None,
                                      dead=None, ws=None, params=None, stream=None):
-    d_out, d_in = W.shape
+    call = "nvfp4_gptq_schur_replay_quantize"
+    d_out, d_in = _matrix(call, W, "W", _IO_DTYPES)
+    _need(call, U, "U", (d_in, d_in), _F32)
+    _opt_need(call, dead, "dead", shape=(d_in,), dtype=_U8)
+    _check_solve_outputs(call, d_out, d_in, codes, scales, global_scale, err_out)
     p = params if params is not None else default_params()
-    _check("nvfp4_gptq_schur_replay_quantize", lib().nvfp4_gptq_schur_replay_quantize(
+    nws = _ws_bytes(call, ws, nvfp4_quantize_workspace_size(d_out, d_in, p))
+    _check(call, lib().nvfp4_gptq_schur_replay_quantize(
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
-        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
-        0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws), nws,
+        _stream(stream)))
 
 
 def nvfp4_export_scales_size(d_out, d_in) -> int:
@@ -208,25 +282,36 @@ def nvfp4_export_scales_size(d_out, d_in) -> int:
 def nvfp4_export_scales(scales, out, stream=None):
     """scales: (d_out, d_in/16) uint8 device tensor -> out (flat uint8 device
     tensor of nvfp4_export_scales_size bytes) in the 128 x 4 tiled layout."""
-    d_out, nb = scales.shape
-    _check("nvfp4_export_scales", lib().nvfp4_export_scales(
+    call = "nvfp4_export_scales"
+    d_out, nb = _matrix(call, scales, "scales", _U8)
+    _need(call, out, "out", dtype=_U8, numel_min=nvfp4_export_scales_size(d_out, nb * 16))
+    _check(call, lib().nvfp4_export_scales(
         _ptr(scales), d_out, nb * 16, _ptr(out), _stream(stream)))
 
 
 def nvfp4_weight_amax(W, amax_out, dead=None, stream=None):
-    d_out, d_in = W.shape
-    _check("nvfp4_weight_amax", lib().nvfp4_weight_amax(
+    call = "nvfp4_weight_amax"
+    d_out, d_in = _matrix(call, W, "W", _IO_DTYPES)
+    _need(call, amax_out, "amax_out", (1,), _F32)
+    _opt_need(call, dead, "dead", shape=(d_in,), dtype=_U8)
+    _check(call, lib().nvfp4_weight_amax(
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(dead), _ptr(amax_out), _stream(stream)))
 
 
 def nvfp4_gptq_schur_replay_quantize_rows(W, U, amax, codes, scales, global_scale, err_out=None,
                                           dead=None, ws=None, params=None, stream=None):
-    d_out, d_in = W.shape
+    call = "nvfp4_gptq_schur_replay_quantize_rows"
+    d_out, d_in = _matrix(call, W, "W", _IO_DTYPES)
+    _need(call, U, "U", (d_in, d_in), _F32)
+    _need(call, amax, "amax", (1,), _F32)
+    _opt_need(call, dead, "dead", shape=(d_in,), dtype=_U8)
+    _check_solve_outputs(call, d_out, d_in, codes, scales, global_scale, err_out)
     p = params if params is not None else default_params()
-    _check("nvfp4_gptq_schur_replay_quantize_rows", lib().nvfp4_gptq_schur_replay_quantize_rows(
+    nws = _ws_bytes(call, ws, nvfp4_quantize_workspace_size(d_out, d_in, p))
+    _check(call, lib().nvfp4_gptq_schur_replay_quantize_rows(
         _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead), _ptr(amax),
-        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws),
-        0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(ws), nws,
+        _stream(stream)))
 
 
 def nvfp4_gptq_schur_replay_quantize_noalloc(W, U, codes, scales, global_scale, err_out=None,
@@ -234,9 +319,14 @@ def nvfp4_gptq_schur_replay_quantize_noalloc(W, U, codes, scales, global_scale, 
                                              stream=None):
     """The quantize call without a workspace: the library's fixed device
     scratch array is used instead, for callers that cannot allocate."""
-    d_out, d_in = W.shape
+    call = "nvfp4_gptq_schur_replay_quantize_noalloc"
+    d_out, d_in = _matrix(call, W, "W", _IO_DTYPES)
+    _need(call, U, "U", (d_in, d_in), _F32)
+    _opt_need(call, dead, "dead", shape=(d_in,), dtype=_U8)
+    _opt_need(call, status_out, "status_out", shape=(1,), dtype=_I32)
+    _check_solve_outputs(call, d_out, d_in, codes, scales, global_scale, err_out)
     p = params if params is not None else default_params()
-    _check("nvfp4_gptq_schur_replay_quantize_noalloc",
+    _check(call,
            lib().nvfp4_gptq_schur_replay_quantize_noalloc(
                _ptr(W), _dtype_code(W), d_out, d_in, _ptr(U), ctypes.byref(p), _ptr(dead),
                _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(err_out), _ptr(status_out),
@@ -244,8 +334,12 @@ def nvfp4_gptq_schur_replay_quantize_noalloc(W, U, codes, scales, global_scale, 
 
 
 def nvfp4_dequant(codes, scales, global_scale, out, stream=None):
-    d_out, d_in = out.shape
-    _check("nvfp4_dequant", lib().nvfp4_dequant(
+    call = "nvfp4_dequant"
+    d_out, d_in = _matrix(call, out, "out", _IO_DTYPES)
+    _need(call, codes, "codes", (d_out, d_in // 2), _U8)
+    _need(call, scales, "scales", (d_out, d_in // 16), _U8)
+    _need(call, global_scale, "global_scale", (1,), _F32)
+    _check(call, lib().nvfp4_dequant(
         _ptr(codes), _ptr(scales), _ptr(global_scale), d_out, d_in, _ptr(out),
         _dtype_code(out), _stream(stream)))
 
@@ -255,16 +349,36 @@ def nvfp4_layer_error_workspace_size(d_out, d_in) -> int:
 
 
 def nvfp4_layer_error(W, codes, scales, global_scale, H, err_out, ws, stream=None):
-    d_out, d_in = W.shape
-    _check("nvfp4_layer_error", lib().nvfp4_layer_error(
+    call = "nvfp4_layer_error"
+    d_out, d_in = _matrix(call, W, "W", _IO_DTYPES)
+    _need(call, codes, "codes", (d_out, d_in // 2), _U8)
+    _need(call, scales, "scales", (d_out, d_in // 16), _U8)
+    _need(call, global_scale, "global_scale", (1,), _F32)
+    _need(call, H, "H", (d_in, d_in), _F32)
+    _need(call, err_out, "err_out", (1,), _F64)
+    nws = _ws_bytes(call, ws, nvfp4_layer_error_workspace_size(d_out, d_in))
+    _check(call, lib().nvfp4_layer_error(
         _ptr(W), _dtype_code(W), _ptr(codes), _ptr(scales), _ptr(global_scale), _ptr(H),
-        d_out, d_in, _ptr(err_out), _ptr(ws), ws.numel(), _stream(stream)))
+        d_out, d_in, _ptr(err_out), _ptr(ws), nws, _stream(stream)))
 
 
 def nvfp4_gemm_nt_f32(P, Q, C, alpha=1.0, beta=0.0, lower=False, status=None, stream=None):
-    """C = beta C + alpha P Q^T (3xTF32 on the tensor cores); P, Q, C fp32."""
+    """C = beta C + alpha P Q^T (3xTF32 on the tensor cores); P, Q, C fp32
+    matrices with unit column stride (row strides are passed as leading
+    dimensions)."""
+    call = "nvfp4_gemm_nt_f32"
+    for name, t in (("P", P), ("Q", Q), ("C", C)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != _F32 or \
+                t.dim() != 2 or t.stride(1) != 1:
+            raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG,
+                             f"{name}: expected a CUDA fp32 matrix with unit column stride")
     M, K = P.shape
     N = Q.shape[0]
+    if Q.shape[1] != K or tuple(C.shape) != (M, N):
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG,
+                         f"shapes P {tuple(P.shape)}, Q {tuple(Q.shape)}, C {tuple(C.shape)}")
+    if status is not None:
+        _need(call, status, "status", (1,), _I32)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=P.device)
     _check("nvfp4_gemm_nt_f32", lib().nvfp4_gemm_nt_f32(
@@ -295,19 +409,43 @@ def _opt(ts):
     return None if ts is None else _ptrs(ts)
 
 
+def _each(call, n, lists):
+    for name, ts in lists.items():
+        if ts is not None and len(ts) != n:
+            raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, f"{name}: {len(ts)} entries, not {n}")
+
+
 def nvfp4_hessian_accumulate_batched(Hs, Xs, beta=0, stream=None):
+    call = "nvfp4_hessian_accumulate_batched"
     n = len(Hs)
+    _each(call, n, {"X": Xs})
     if len({x.dtype for x in Xs}) > 1:
-        raise TypeError("all X must share one dtype")
-    _check("nvfp4_hessian_accumulate_batched", lib().nvfp4_hessian_accumulate_batched(
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "all X must share one dtype")
+    for i in range(n):
+        _, d = _matrix(call, Xs[i], f"X[{i}]", _IO_DTYPES)
+        _need(call, Hs[i], f"H[{i}]", (d, d), _F32)
+    _check(call, lib().nvfp4_hessian_accumulate_batched(
         n, _ptrs(Hs), _ptrs(Xs), _dtype_code(Xs[0]) if n else 0,
         _i64s([x.shape[0] for x in Xs]), _i64s([x.shape[1] for x in Xs]), int(beta),
         _stream(stream)))
 
 
 def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, wss=None, stream=None):
+    call = "nvfp4_gptq_prepare_batched"
     n = len(Hs)
-    _check("nvfp4_gptq_prepare_batched", lib().nvfp4_gptq_prepare_batched(
+    _each(call, n, {"U": Us, "dead": deads, "lambda_out": lambdas, "ws": wss})
+    if wss is None:
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "workspaces missing")
+    for i in range(n):
+        d, _ = _matrix(call, Hs[i], f"H[{i}]", _F32)
+        _need(call, Hs[i], f"H[{i}]", (d, d))
+        _need(call, Us[i], f"U[{i}]", (d, d), _F32)
+        if deads is not None:
+            _opt_need(call, deads[i], f"dead[{i}]", shape=(d,), dtype=_U8)
+        if lambdas is not None:
+            _opt_need(call, lambdas[i], f"lambda_out[{i}]", shape=(1,), dtype=_F32)
+        _ws_bytes(call, wss[i], nvfp4_prepare_workspace_size(d))
+    _check(call, lib().nvfp4_gptq_prepare_batched(
         n, _ptrs(Hs), _i64s([h.shape[0] for h in Hs]), float(damp), _ptrs(Us), _opt(deads),
         _opt(lambdas), _ptrs(wss), _sizes(wss), _stream(stream)))
 
@@ -315,11 +453,24 @@ def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, wss=None,
 def nvfp4_gptq_schur_replay_quantize_batched(Ws, Us, codes, scales, global_scales,
                                              errs=None, deads=None, wss=None, params=None,
                                              stream=None):
+    call = "nvfp4_gptq_schur_replay_quantize_batched"
     n = len(Ws)
+    _each(call, n, {"U": Us, "codes": codes, "scales": scales, "global_scale": global_scales,
+                    "err_out": errs, "dead": deads, "ws": wss})
+    if wss is None:
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "workspaces missing")
     if len({w.dtype for w in Ws}) > 1:
-        raise TypeError("all W must share one dtype")
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "all W must share one dtype")
     p = params if params is not None else default_params()
-    _check("nvfp4_gptq_schur_replay_quantize_batched",
+    for i in range(n):
+        d_out, d_in = _matrix(call, Ws[i], f"W[{i}]", _IO_DTYPES)
+        _need(call, Us[i], f"U[{i}]", (d_in, d_in), _F32)
+        if deads is not None:
+            _opt_need(call, deads[i], f"dead[{i}]", shape=(d_in,), dtype=_U8)
+        _check_solve_outputs(call, d_out, d_in, codes[i], scales[i], global_scales[i],
+                             None if errs is None else errs[i])
+        _ws_bytes(call, wss[i], nvfp4_quantize_workspace_size(d_out, d_in, p))
+    _check(call,
            lib().nvfp4_gptq_schur_replay_quantize_batched(
                n, _ptrs(Ws), _dtype_code(Ws[0]) if n else 0, _i64s([w.shape[0] for w in Ws]),
                _i64s([w.shape[1] for w in Ws]), _ptrs(Us), ctypes.byref(p), _opt(deads),
@@ -328,10 +479,17 @@ def nvfp4_gptq_schur_replay_quantize_batched(Ws, Us, codes, scales, global_scale
 
 
 def nvfp4_dequant_batched(codes, scales, global_scales, outs, stream=None):
+    call = "nvfp4_dequant_batched"
     n = len(outs)
+    _each(call, n, {"codes": codes, "scales": scales, "global_scale": global_scales})
     if len({o.dtype for o in outs}) > 1:
-        raise TypeError("all outputs must share one dtype")
-    _check("nvfp4_dequant_batched", lib().nvfp4_dequant_batched(
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "all outputs must share one dtype")
+    for i in range(n):
+        d_out, d_in = _matrix(call, outs[i], f"out[{i}]", _IO_DTYPES)
+        _need(call, codes[i], f"codes[{i}]", (d_out, d_in // 2), _U8)
+        _need(call, scales[i], f"scales[{i}]", (d_out, d_in // 16), _U8)
+        _need(call, global_scales[i], f"global_scale[{i}]", (1,), _F32)
+    _check(call, lib().nvfp4_dequant_batched(
         n, _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _i64s([o.shape[0] for o in outs]),
         _i64s([o.shape[1] for o in outs]), _ptrs(outs), _dtype_code(outs[0]) if n else 0,
         _stream(stream)))

@@ -54,7 +54,10 @@ nvfp4_status get_pool(Pool** out) {
 
 // Runs fn(i, stream) for i < count on the pool's streams, ordered after the
 // work already queued on `caller` and joined back into it.  The first failing
-// status is returned (the join is still recorded).
+// status is returned.  Every pool stream that was forked is joined back into
+// `caller` whatever failed in between, so that nothing queued on a pool
+// stream can race with later work on the caller's stream; if the fork itself
+// fails, no problem is issued.
 template <typename F>
 nvfp4_status fan_out(int count, cudaStream_t caller, F fn) {
   if (count <= 0) return NVFP4_OK;
@@ -64,16 +67,32 @@ nvfp4_status fan_out(int count, cudaStream_t caller, F fn) {
   if (st != NVFP4_OK) return st;
   std::lock_guard<std::mutex> lock(g_pool_mu);   // one fan-out per device at a time
   NVFP4_CUDA_TRY(cudaEventRecord(p->fork, caller));
-  const int used = count < kPoolStreams ? count : kPoolStreams;
-  for (int i = 0; i < used; ++i) NVFP4_CUDA_TRY(cudaStreamWaitEvent(p->s[i], p->fork, 0));
+  const int want = count < kPoolStreams ? count : kPoolStreams;
   nvfp4_status first = NVFP4_OK;
-  for (int i = 0; i < count; ++i) {
-    const nvfp4_status s = fn(i, p->s[i % kPoolStreams]);
+  auto keep = [&](nvfp4_status s) {
     if (s != NVFP4_OK && first == NVFP4_OK) first = s;
+  };
+  int forked = 0;
+  for (; forked < want; ++forked) {
+    if (cudaStreamWaitEvent(p->s[forked], p->fork, 0) != cudaSuccess) {
+      cudaGetLastError();
+      keep(NVFP4_ERR_CUDA);
+      break;
+    }
   }
-  for (int i = 0; i < used; ++i) {
-    NVFP4_CUDA_TRY(cudaEventRecord(p->done[i], p->s[i]));
-    NVFP4_CUDA_TRY(cudaStreamWaitEvent(caller, p->done[i], 0));
+  if (forked == want) {
+    for (int i = 0; i < count; ++i) keep(fn(i, p->s[i % kPoolStreams]));
+  }
+  for (int i = 0; i < forked; ++i) {
+    if (cudaEventRecord(p->done[i], p->s[i]) != cudaSuccess ||
+        cudaStreamWaitEvent(caller, p->done[i], 0) != cudaSuccess) {
+      // no device-side join: wait on the host instead, so that the caller's
+      // later work still cannot overlap this pool stream's
+      cudaGetLastError();
+      cudaStreamSynchronize(p->s[i]);
+      cudaGetLastError();
+      keep(NVFP4_ERR_CUDA);
+    }
   }
   return first;
 }

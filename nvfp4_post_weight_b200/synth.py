@@ -15,7 +15,9 @@ for the pages' LLM layers):
                   per channel, 8 "massive" channels x100.
   mlp_down_silu   bf16 W ~ N(0, 0.015^2); bf16 X = SiLU(A) * B, A, B ~ N(0,1).
   lognormal       bf16 W ~ N(0, 0.02^2); bf16 X ~ N(0,1) x lognormal(0, sigma)
-                  per channel (the dense-decoder and MoE-expert layers).
+                  per channel (the dense-decoder and MoE-expert layers; their
+                  large tensors are drawn in float32 by row chunks, each chunk
+                  from its own child stream, on a thread pool).
 """
 from __future__ import annotations
 
@@ -84,23 +86,95 @@ def normal_weights(d_out, d_in, std, rng):
     return _bf16(rng.normal(0.0, std, size=(d_out, d_in)).astype(np.float32))
 
 
+# Large tensors are drawn in row chunks of _CHUNK_ROWS rows, chunk c from the
+# c-th child of the tensor's own SeedSequence, on a thread pool (numpy's
+# generators release the GIL while they fill an array), in float32 precision.
+_CHUNK_ROWS = 1024
+
+
+def _pool():
+    import concurrent.futures as cf
+    import os
+    return cf.ThreadPoolExecutor(max(1, min(32, len(os.sched_getaffinity(0)))))
+
+
+def _fill_rows(out: np.ndarray, ss: np.random.SeedSequence, draw, pool=None) -> None:
+    """out[r0:r1] = draw(rng_c, out[r0:r1]) for every row chunk c, rng_c the
+    chunk's own generator; the chunks are independent, so the result does
+    not depend on the number of threads.  pool: a thread pool, None (a new
+    one) or "serial" (this thread)."""
+    rows = out.shape[0]
+    kids = ss.spawn((rows + _CHUNK_ROWS - 1) // _CHUNK_ROWS)
+
+    def one(c):
+        r0, r1 = c * _CHUNK_ROWS, min(rows, (c + 1) * _CHUNK_ROWS)
+        draw(np.random.default_rng(kids[c]), out[r0:r1])
+
+    if pool == "serial":
+        for c in range(len(kids)):
+            one(c)
+    elif pool is None:
+        with _pool() as p:
+            list(p.map(one, range(len(kids))))
+    else:
+        list(pool.map(one, range(len(kids))))
+
+
+def normal_weights_fast(d_out, d_in, std, ss, pool=None):
+    """bf16 (d_out, d_in) ~ N(0, std^2), drawn in float32 by row chunks."""
+    W = np.empty((d_out, d_in), dtype=np.float32)
+
+    def draw(g, blk):
+        g.standard_normal(out=blk, dtype=np.float32)
+        blk *= np.float32(std)
+
+    _fill_rows(W, ss, draw, pool)
+    return _bf16(W)
+
+
+def lognormal_acts_fast(n_tok, d_in, sigma, ss, pool=None):
+    """bf16 (n_tok, d_in) activations: N(0,1) (float32, by row chunks of the
+    first child of ss) times per-channel lognormal(0, sigma) scales (second
+    child)."""
+    ss_x, ss_s = ss.spawn(2)
+    scale = np.random.default_rng(ss_s).lognormal(0.0, sigma, size=d_in).astype(np.float32)
+    X = np.empty((n_tok, d_in), dtype=np.float32)
+
+    def draw(g, blk):
+        g.standard_normal(out=blk, dtype=np.float32)
+        blk *= scale[None, :]
+
+    _fill_rows(X, ss_x, draw, pool)
+    return _bf16(X)
+
+
+# The 70B-shaped dense decoder layer: its linears, each as (d_out, d_in), in
+# the order they are solved; the Hessian groups share one factor.
+DENSE_70B_SHAPES = {"q": (8192, 8192), "k": (1024, 8192), "v": (1024, 8192),
+                    "o": (8192, 8192), "gate": (28672, 8192), "up": (28672, 8192),
+                    "down": (8192, 28672)}
+DENSE_70B_GROUPS = (("X_attn", ("q", "k", "v")), ("X_o", ("o",)), ("X_mlp", ("gate", "up")),
+                    ("X_down", ("down",)))
+
+
 def dense_decoder_layer(hidden=8192, kv=1024, inter=28672, n_tok=16384, seed=3):
-    """70B-shaped dense decoder layer: q, k, v, o, gate, up, down weights and
-    four independent calibration activations (attention input, o input, MLP
-    input, down input), lognormal(0, 1.5) channel scales.  Returned lazily as
-    a dict of callables so that a caller can build one tensor at a time."""
-    names = ["q", "k", "v", "o", "gate", "up", "down",
-             "X_attn", "S_attn", "X_o", "S_o", "X_mlp", "S_mlp", "X_down", "S_down"]
-    rngs = dict(zip(names, _children(seed, len(names))))
+    """70B-shaped dense decoder layer: q, k, v, o, gate, up, down weights
+    (bf16 ~ N(0, 0.02^2)) and four independent calibration activations
+    (attention input, o input, MLP input, down input: n_tok tokens,
+    N(0,1) x lognormal(0, 1.5) channel scales).  Every tensor has its own
+    child of SeedSequence(seed), in the order q, k, v, o, gate, up, down,
+    X_attn, X_o, X_mlp, X_down.  Returned lazily as a dict of callables so
+    that a caller can build one tensor at a time."""
+    names = ["q", "k", "v", "o", "gate", "up", "down", "X_attn", "X_o", "X_mlp", "X_down"]
+    kids = dict(zip(names, np.random.SeedSequence(seed).spawn(len(names))))
     shapes = {"q": (hidden, hidden), "k": (kv, hidden), "v": (kv, hidden),
               "o": (hidden, hidden), "gate": (inter, hidden), "up": (inter, hidden),
               "down": (hidden, inter)}
     out = {}
     for n, shp in shapes.items():
-        out[n] = (lambda shp=shp, r=rngs[n]: normal_weights(shp[0], shp[1], 0.02, r))
+        out[n] = (lambda shp=shp, ss=kids[n]: normal_weights_fast(shp[0], shp[1], 0.02, ss))
     for x, d in (("attn", hidden), ("o", hidden), ("mlp", hidden), ("down", inter)):
-        out["X_" + x] = (lambda d=d, rx=rngs["X_" + x], rs=rngs["S_" + x]:
-                         lognormal_acts(n_tok, d, 1.5, rx, rs))
+        out["X_" + x] = (lambda d=d, ss=kids["X_" + x]: lognormal_acts_fast(n_tok, d, 1.5, ss))
     return out
 
 
@@ -132,23 +206,34 @@ def zipf_token_counts(n_experts=128, total=65536, alpha=1.1, lo=64, hi=4096):
 
 def moe_layer(n_experts=128, hidden=4096, inter=1536, total_tokens=65536, seed=4):
     """MoE layer of independent experts (gate/up hidden->inter, down
-    inter->hidden).  Returns (counts, make_expert) where make_expert(e)
-    draws expert e's tensors from its own child streams."""
+    inter->hidden, bf16 ~ N(0, 0.02^2); activations N(0,1) x lognormal(0, 1)
+    channel scales).  Returns (counts, make_expert) where make_expert(e)
+    draws expert e's tensors from the children of the e-th child of
+    SeedSequence(seed), in the order gate, up, down, X_in, X_mid."""
     counts = zipf_token_counts(n_experts, total_tokens)
     roots = np.random.SeedSequence(seed).spawn(n_experts)
 
-    def make_expert(e):
-        g = [np.random.default_rng(s) for s in roots[e].spawn(7)]
+    def make_expert(e, pool=None):
+        g = roots[e].spawn(5)
         n = int(counts[e])
         return dict(
-            gate=normal_weights(inter, hidden, 0.02, g[0]),
-            up=normal_weights(inter, hidden, 0.02, g[1]),
-            down=normal_weights(hidden, inter, 0.02, g[2]),
-            X_in=lognormal_acts(n, hidden, 1.0, g[3], g[4]),
-            X_mid=lognormal_acts(n, inter, 1.0, g[5], g[6]),
+            gate=normal_weights_fast(inter, hidden, 0.02, g[0], pool),
+            up=normal_weights_fast(inter, hidden, 0.02, g[1], pool),
+            down=normal_weights_fast(hidden, inter, 0.02, g[2], pool),
+            X_in=lognormal_acts_fast(n, hidden, 1.0, g[3], pool),
+            X_mid=lognormal_acts_fast(n, inter, 1.0, g[4], pool),
         )
 
     return counts, make_expert
+
+
+def moe_all_experts(n_experts=128, **kw):
+    """counts and the list of every expert's tensors of moe_layer (drawn on
+    one thread pool)."""
+    counts, make = moe_layer(n_experts=n_experts, **kw)
+    with _pool() as p:
+        experts = list(p.map(lambda e: make(e, "serial"), range(n_experts)))
+    return counts, experts
 
 
 WORKLOADS = {

@@ -66,9 +66,13 @@ def classify(ref: dict, U: np.ndarray, s_g: float, codes_gpu: np.ndarray,
     """Compare GPU codes/scales with the oracle's (ref from
     oracle.schur_replay_gptq(..., return_diag=True)) on the given oracle rows.
 
-    Returns a dict: n_blocks, n_mismatch, frac, rows_affected, and
-    bad_first: list of (row, block, margin, midpoint_dist) for rows whose first
-    differing block is not at a near-tie."""
+    Returns a dict: n_blocks, n_mismatch, frac, rows_affected; for the first
+    differing block of every affected row, which clause excused it:
+    first_scale_tie (the oracle's top two scores within NEAR_TIE, the rule the
+    acceptance criterion states) or first_midpoint (a replayed value within
+    NEAR_TIE of an E2M1 rounding midpoint, this suite's reading of the same
+    kind of event for the codes); and bad_first: list of (row, block, margin,
+    midpoint_dist) for rows whose first differing block is neither."""
     oc = ref["codes"]
     os_ = ref["scales"]
     gc = codes_gpu
@@ -80,13 +84,15 @@ def classify(ref: dict, U: np.ndarray, s_g: float, codes_gpu: np.ndarray,
     mism = ~blk_eq
     res = dict(n_blocks=int(blk_eq.size), n_mismatch=int(mism.sum()),
                frac=float(mism.mean()) if blk_eq.size else 0.0,
-               rows_affected=int(mism.any(axis=1).sum()), bad_first=[])
+               rows_affected=int(mism.any(axis=1).sum()), first_scale_tie=0,
+               first_midpoint=0, bad_first=[])
     sg = float(np.float32(s_g))
     for r in np.nonzero(mism.any(axis=1))[0]:
         b = int(np.argmax(mism[r]))
         margin = float(ref["margin"][r, b]) if "margin" in ref else \
             float(top2_margin(ref["scores"][r, b]))
         if margin < NEAR_TIE:
+            res["first_scale_tie"] += 1
             continue
         Ublk = U[16 * b:16 * b + 16, 16 * b:16 * b + 16]
         s_or = O.e4m3_value(os_[r, b]) * sg
@@ -95,6 +101,18 @@ def classify(ref: dict, U: np.ndarray, s_g: float, codes_gpu: np.ndarray,
             s_gp = O.e4m3_value(gs[r, b]) * sg
             dist = min(dist, midpoint_distance(ref["wblock"][r, b], Ublk, s_gp))
         if dist < NEAR_TIE:
+            res["first_midpoint"] += 1
             continue
         res["bad_first"].append((int(r if rows is None else rows[r]), b, margin, dist))
     return res
+
+
+def report(label: str, c: dict) -> str:
+    """One line of what a comparison found (printed by the parity tests; run
+    pytest with -s to see them)."""
+    line = (f"PARITY {label}: blocks={c['n_blocks']} mismatched={c['n_mismatch']} "
+            f"({c['frac']:.2e}) rows_affected={c['rows_affected']} "
+            f"first_excused_scale_tie={c['first_scale_tie']} "
+            f"first_excused_midpoint={c['first_midpoint']} bad_first={len(c['bad_first'])}")
+    print(line, flush=True)
+    return line

@@ -26,7 +26,7 @@ import torch
 import oracle as O
 from nvfp4_post_weight_b200 import binding as B
 from nvfp4_post_weight_b200 import synth
-from parity import classify, unpack_codes
+from parity import classify, report, unpack_codes
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -96,6 +96,7 @@ def check_group(layer, x_name, w_names, seed):
         s_g = scales[rows].cpu().numpy().astype(np.int64)
         ref = O.schur_replay_gptq(W64[rows], Uo, sg, return_diag=True)
         c = classify(ref, Uo, sg, c_g, s_g, rows)
+        report(f"dense_decoder_70b {name}", c)
         assert c["frac"] <= 1e-3, (name, c)
         assert not c["bad_first"], (name, c)
         Q = O.dequant(c_g, s_g, sg).astype(np.float64)

@@ -25,7 +25,7 @@ import torch
 import oracle as O
 from nvfp4_post_weight_b200 import binding as B
 from nvfp4_post_weight_b200 import synth
-from parity import classify, unpack_codes
+from parity import classify, report, unpack_codes
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -93,6 +93,7 @@ def test_expert_hessians(moe):
 def check_rows(W64, U, sg, codes, scales, H, Q_gpu, label):
     ref = O.schur_replay_gptq(W64, U, sg, return_diag=True)
     c = classify(ref, U, sg, codes, scales)
+    report(f"moe {label}", c)
     assert c["frac"] <= 1e-3, (label, c)
     assert not c["bad_first"], (label, c)
     Q = O.dequant(codes, scales, sg)

@@ -18,7 +18,7 @@ import oracle as O
 from nvfp4_post_weight_b200 import binding as B
 from nvfp4_post_weight_b200 import synth
 from nvfp4_post_weight_b200.layer import LayerSolver
-from parity import classify, unpack_codes, pack_codes
+from parity import classify, report, unpack_codes, pack_codes
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -383,12 +383,15 @@ def test_solve_attn_4096_all_rows():
     codes = unpack_codes(s.codes.cpu().numpy()[rows])
     scales = s.scales.cpu().numpy()[rows].astype(np.int64)
     c = classify(ref, U, sg, codes, scales, rows)
+    report("attn_massive_4096x4096 all rows", c)
     assert c["frac"] <= 1e-3, c
     assert not c["bad_first"], c
     Q = O.dequant(codes, scales, sg).astype(np.float64)
     L_gpu = O.layer_error(W64[rows], Q, H)
     L_ref = O.layer_error(W64[rows], ref["q"], H)
     assert abs(L_gpu - L_ref) <= 1e-4 * L_ref
+    # the library's own layer error (Gram form on the tensor cores)
+    assert abs(s.layer_err.item() - L_ref) <= 1e-4 * L_ref
 
 
 def test_solve_mlp_down_14336_given_hessian_row_sample():
@@ -422,6 +425,7 @@ def test_solve_mlp_down_14336_given_hessian_row_sample():
     rows = np.sort(np.random.default_rng(102).choice(d_out, 512, replace=False))
     ref = O.schur_replay_gptq(W64[rows], Uo, sg, return_diag=True)
     c = classify(ref, Uo, sg, codes[rows], scales[rows], rows)
+    report("mlp_down_silu_4096x14336 given H, 512 rows", c)
     assert c["frac"] <= 1e-3, c
     assert not c["bad_first"], c
     Q = O.dequant(codes[rows], scales[rows], sg).astype(np.float64)

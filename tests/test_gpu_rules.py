@@ -16,7 +16,7 @@ import oracle as O
 from nvfp4_post_weight_b200 import binding as B
 from nvfp4_post_weight_b200 import synth
 from nvfp4_post_weight_b200.layer import LayerSolver
-from parity import classify, unpack_codes
+from parity import classify, report, unpack_codes
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -104,6 +104,7 @@ def test_rule_attn_4096_all_rows(attn_layer, rule):
     codes = unpack_codes(s.codes.cpu().numpy())
     scales = s.scales.cpu().numpy().astype(np.int64)
     c = classify(ref, U, sg, codes, scales)
+    report(f"attn_massive_4096x4096 rule {rule}", c)
     assert c["frac"] <= 1e-3, c
     assert not c["bad_first"], c
     Q = O.dequant(codes, scales, sg).astype(np.float64)

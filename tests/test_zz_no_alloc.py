@@ -83,6 +83,25 @@ def test_noalloc_matches_workspace_call_twice():
         assert abs(got[3] - ref[3]) <= 1e-9 * abs(ref[3])
 
 
+def test_noalloc_reserves_nothing_after_its_first_call():
+    """The first call on a device loads the library module that holds the
+    fixed scratch array (lazy module loading); from then on a call changes
+    the device's free memory by nothing."""
+    W, X = synth.small_outlier(d_out=128, d_in=256, n_tok=512, seed=13)
+    U = _factor(X, 256)
+    Wd = W.to(DEV)
+    codes, scales, sg, err = _outputs(128, 256)
+    status = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+    B.nvfp4_gptq_schur_replay_quantize_noalloc(Wd, U, codes, scales, sg, err, status)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(2):
+        B.nvfp4_gptq_schur_replay_quantize_noalloc(Wd, U, codes, scales, sg, err, status)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert status.item() == 0
+
+
 def test_noalloc_rejects_layers_beyond_its_scratch():
     d_out, d_in = 4096, 4096   # needs far more than the fixed 16 MiB
     assert B.nvfp4_quantize_workspace_size(d_out, d_in) > (16 << 20)
