@@ -338,8 +338,7 @@ class MoELayer:
         self.solver.step(self.Wd, self.Xd)
 
     def status_ok(self):
-        ws, h = self.solver.status()
-        return all(v == 0 for v in ws) and h == 0
+        return self.solver.status() == (0, 0, 0)
 
 
 WORKLOADS = {

@@ -83,17 +83,30 @@ typedef enum {
   NVFP4_RULE_BLOCK_MSE = 2
 } nvfp4_scale_rule;
 
-/* Solve parameters.  n_candidates, cand_lo and lazy_batch support only the
- * defaults below (n_candidates = 16, cand_lo = -8, lazy_batch = 128); other
- * values, or a scale_rule outside nvfp4_scale_rule, return
- * NVFP4_ERR_UNSUPPORTED.  The candidate window is the n_candidates
- * consecutive E4M3 codes starting at k0 + cand_lo, shifted into 1..126,
- * where k0 = e4m3_rn(amax_block / (6 s_g)) (at least 1). */
+/* Arithmetic of the solve (nvfp4_solve_params.precision).
+ * NVFP4_PRECISION_FP64_REPLAY (the default and the only value this build
+ *   supports): the working copy W~ and the Schur Replay are fp64, the
+ *   trailing-update products 3xTF32 on the tensor cores (fp32-level
+ *   products, accumulated into the fp64 W~), the factor U fp64-accurate and
+ *   stored fp32.  The codes are discrete decisions taken on values every
+ *   earlier column's update has moved, so an fp32 working copy or replay flips
+ *   decisions that are not near ties; this is the cheapest arithmetic measured
+ *   to keep them on the exact solve's. */
+typedef enum { NVFP4_PRECISION_FP64_REPLAY = 0 } nvfp4_precision;
+
+/* Solve parameters.  n_candidates, cand_lo, lazy_batch and precision support
+ * only the defaults below (n_candidates = 16, cand_lo = -8, lazy_batch = 128,
+ * precision = NVFP4_PRECISION_FP64_REPLAY); other values, or a scale_rule
+ * outside nvfp4_scale_rule, return NVFP4_ERR_UNSUPPORTED.  The candidate
+ * window is the n_candidates consecutive E4M3 codes starting at
+ * k0 + cand_lo, shifted into 1..126, where k0 = e4m3_rn(amax_block / (6 s_g))
+ * (at least 1). */
 typedef struct {
   int n_candidates; /* 16 */
   int cand_lo;      /* -8 */
   int lazy_batch;   /* 128: columns per batch of the trailing update */
   int scale_rule;   /* nvfp4_scale_rule, default NVFP4_RULE_SCHUR_REPLAY */
+  int precision;    /* nvfp4_precision, default NVFP4_PRECISION_FP64_REPLAY */
 } nvfp4_solve_params;
 
 /* Fills *p with the defaults above. */
@@ -342,14 +355,44 @@ nvfp4_status nvfp4_layer_error(const void* W, nvfp4_dtype w_dtype, const uint8_t
 /* ------------------------------------------------------------------------ */
 /* Every array argument is a HOST array of length count holding the per-problem
  * value of the argument of the same name in the single-problem call (device
- * pointers, sizes, workspaces); the per-problem rules, layouts and status words
- * are those of the single-problem call.  Optional per-problem pointers
- * (dead, lambda_out, err_out) may be given as a NULL array.  The problems run
- * concurrently on an internal pool of 8 streams per device that fork from and
- * join back into `stream`: when the call returns, all of the work is ordered
- * before anything later queued on `stream`.  The first failing problem's host
- * status is returned (later problems are still issued).  count == 0 is a
- * no-op; count < 0 or a NULL required array is NVFP4_ERR_INVALID_ARG. */
+ * pointers and sizes); the per-problem rules and layouts are those of the
+ * single-problem call, and every result equals the single call's bit for bit.
+ * Optional per-problem pointers (dead, lambda_out, err_out) may be given as a
+ * NULL array.
+ *
+ * Problems of equal shape (d; or d_out and d_in) are solved together: each
+ * kernel launch of the call covers all problems of one shape (up to 256; a
+ * larger set makes one group per 256), so the number of launches grows with
+ * the number of distinct shapes, not with count.  Problems are grouped in
+ * their order of appearance.
+ *
+ * Scratch: ONE device workspace for the whole call (256-byte aligned), of
+ * nvfp4_prepare_batched_workspace_size() / nvfp4_quantize_batched_workspace_
+ * size() bytes for the same count and sizes -- the sum of the problems'
+ * single-call workspaces, so split a call whose total does not fit.  It
+ * starts with a status header: nvfp4_workspace_status() on it returns the
+ * first non-OK status of any problem, nvfp4_batched_workspace_status() also
+ * each problem's own (a timed-out wait inside a launch that serves several
+ * problems is reported for each of them).
+ *
+ * Every argument is checked on the host before anything is launched: the
+ * first problem that fails a check decides the returned status and then
+ * nothing is queued.  count == 0 is a no-op; count < 0 or a NULL required
+ * array is NVFP4_ERR_INVALID_ARG. */
+size_t nvfp4_prepare_batched_workspace_size(int count, const int64_t* d);
+size_t nvfp4_quantize_batched_workspace_size(int count, const int64_t* d_out,
+                                             const int64_t* d_in,
+                                             const nvfp4_solve_params* params);
+
+/* Synchronizes `stream`, writes problem i's status word to status[i] (host
+ * array of count ints, may be NULL) and returns the first non-OK status of
+ * any problem of the batched call that last used ws. */
+nvfp4_status nvfp4_batched_workspace_status(const void* ws, int count, int* status,
+                                            nvfp4_stream_t stream);
+
+/* Tensor-core problems (bf16 tokens, d >= 256, n_tok >= 64, 16-byte aligned)
+ * of one d run in one launch per 128 problems, heaviest token counts first;
+ * any other problem runs on its own.  No workspace. */
 nvfp4_status nvfp4_hessian_accumulate_batched(int count, float* const* H, const void* const* X,
                                               nvfp4_dtype x_dtype, const int64_t* n_tok,
                                               const int64_t* d, int beta,
@@ -357,16 +400,17 @@ nvfp4_status nvfp4_hessian_accumulate_batched(int count, float* const* H, const 
 
 nvfp4_status nvfp4_gptq_prepare_batched(int count, const float* const* H, const int64_t* d,
                                         float damp, float* const* U, uint8_t* const* dead,
-                                        float* const* lambda_out, void* const* ws,
-                                        const size_t* ws_bytes, nvfp4_stream_t stream);
+                                        float* const* lambda_out, void* ws, size_t ws_bytes,
+                                        nvfp4_stream_t stream);
 
 nvfp4_status nvfp4_gptq_schur_replay_quantize_batched(
     int count, const void* const* W, nvfp4_dtype w_dtype, const int64_t* d_out,
     const int64_t* d_in, const float* const* U, const nvfp4_solve_params* params,
     const uint8_t* const* dead, uint8_t* const* codes, uint8_t* const* scales,
-    float* const* global_scale, double* const* err_out, void* const* ws,
-    const size_t* ws_bytes, nvfp4_stream_t stream);
+    float* const* global_scale, double* const* err_out, void* ws, size_t ws_bytes,
+    nvfp4_stream_t stream);
 
+/* No workspace. */
 nvfp4_status nvfp4_dequant_batched(int count, const uint8_t* const* codes,
                                    const uint8_t* const* scales,
                                    const float* const* global_scale, const int64_t* d_out,
@@ -392,6 +436,22 @@ nvfp4_status nvfp4_gemm_nt_f32(int64_t M, int64_t N, int64_t K, float alpha, con
 /* Number of kernels this library has launched since it was loaded (all
  * threads, all devices).  Host-only; never fails. */
 long long nvfp4_launch_count(void);
+
+/* Failure-detection support (the paper has no counterpart).  Sets, for the
+ * current device, how long a pipeline wait inside the library's tensor-core
+ * kernels (a TMA copy to land, an MMA stage or accumulator to be released)
+ * may spin before the kernel gives up: ns nanoseconds of wall time, 0 for the
+ * default of 4 s.  A wait that runs out records NVFP4_ERR_TIMEOUT in the
+ * call's status word; the kernel then waits (always with the 4 s bound) for
+ * the copies and MMAs it has already issued, frees its tensor memory and
+ * returns, so the context stays usable.  A limit shorter than a kernel's
+ * normal waits makes it time out: that is how the timeout path is tested;
+ * with ns = 1 a wait gives up as soon as one non-blocking probe finds that
+ * what it waits for has not happened yet (the first copy of a kernel always
+ * takes longer), so every tensor-core kernel then times out.
+ * Synchronous (it writes the limit to device memory); returns NVFP4_ERR_CUDA
+ * if that write fails.  Not for use while library kernels run. */
+nvfp4_status nvfp4_set_wait_limit_ns(unsigned long long ns);
 
 /* Phases reported by nvfp4_profile_end, in this order. */
 enum {

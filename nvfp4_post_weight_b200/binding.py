@@ -32,7 +32,8 @@ class Nvfp4Error(RuntimeError):
 
 class SolveParams(ctypes.Structure):
     _fields_ = [("n_candidates", ctypes.c_int), ("cand_lo", ctypes.c_int),
-                ("lazy_batch", ctypes.c_int), ("scale_rule", ctypes.c_int)]
+                ("lazy_batch", ctypes.c_int), ("scale_rule", ctypes.c_int),
+                ("precision", ctypes.c_int)]
 
 
 _lib = None
@@ -74,16 +75,21 @@ def lib():
                 [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, vp,
                  sz, vp], i32),
             "nvfp4_hessian_accumulate_batched": ([i32, vp, vp, i32, vp, vp, i32, vp], i32),
-            "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, vp, vp], i32),
+            "nvfp4_prepare_batched_workspace_size": ([i32, vp], sz),
+            "nvfp4_quantize_batched_workspace_size": ([i32, vp, vp, ctypes.POINTER(SolveParams)],
+                                                      sz),
+            "nvfp4_batched_workspace_status": ([vp, i32, vp, vp], i32),
+            "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_gptq_schur_replay_quantize_batched": (
                 [i32, vp, i32, vp, vp, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
-                 vp, vp], i32),
+                 sz, vp], i32),
             "nvfp4_dequant_batched": ([i32, vp, vp, vp, vp, vp, vp, i32, vp], i32),
             "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
                                    vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
             "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
             "nvfp4_launch_count": ([], ctypes.c_longlong),
+            "nvfp4_set_wait_limit_ns": ([ctypes.c_ulonglong], i32),
             "nvfp4_profile_begin": ([], i32),
             "nvfp4_profile_end": ([vp, vp, i32], i32),
             "nvfp4_profile_work": ([vp, i32], i32),
@@ -401,10 +407,6 @@ def _i64s(vals):
     return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])
 
 
-def _sizes(ws):
-    return (ctypes.c_size_t * len(ws))(*[w.numel() for w in ws])
-
-
 def _opt(ts):
     return None if ts is None else _ptrs(ts)
 
@@ -430,12 +432,32 @@ def nvfp4_hessian_accumulate_batched(Hs, Xs, beta=0, stream=None):
         _stream(stream)))
 
 
-def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, wss=None, stream=None):
+def nvfp4_prepare_batched_workspace_size(ds) -> int:
+    return int(lib().nvfp4_prepare_batched_workspace_size(len(ds), _i64s(ds)))
+
+
+def nvfp4_quantize_batched_workspace_size(shapes, params=None) -> int:
+    """shapes: [(d_out, d_in)] of the problems."""
+    p = params if params is not None else default_params()
+    return int(lib().nvfp4_quantize_batched_workspace_size(
+        len(shapes), _i64s([s[0] for s in shapes]), _i64s([s[1] for s in shapes]),
+        ctypes.byref(p)))
+
+
+def nvfp4_batched_workspace_status(ws, count, stream=None):
+    """(first non-OK status of any problem, [status of each problem])."""
+    st = (ctypes.c_int * max(count, 1))()
+    r = int(lib().nvfp4_batched_workspace_status(_ptr(ws), int(count), st, _stream(stream)))
+    return r, [int(st[i]) for i in range(count)]
+
+
+def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, ws=None, stream=None):
+    """All factors in one call; ws: one workspace of
+    nvfp4_prepare_batched_workspace_size bytes for the whole call."""
     call = "nvfp4_gptq_prepare_batched"
     n = len(Hs)
-    _each(call, n, {"U": Us, "dead": deads, "lambda_out": lambdas, "ws": wss})
-    if wss is None:
-        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "workspaces missing")
+    _each(call, n, {"U": Us, "dead": deads, "lambda_out": lambdas})
+    ds = []
     for i in range(n):
         d, _ = _matrix(call, Hs[i], f"H[{i}]", _F32)
         _need(call, Hs[i], f"H[{i}]", (d, d))
@@ -444,24 +466,26 @@ def nvfp4_gptq_prepare_batched(Hs, damp, Us, deads=None, lambdas=None, wss=None,
             _opt_need(call, deads[i], f"dead[{i}]", shape=(d,), dtype=_U8)
         if lambdas is not None:
             _opt_need(call, lambdas[i], f"lambda_out[{i}]", shape=(1,), dtype=_F32)
-        _ws_bytes(call, wss[i], nvfp4_prepare_workspace_size(d))
+        ds.append(d)
+    nws = _ws_bytes(call, ws, nvfp4_prepare_batched_workspace_size(ds)) if n else 0
     _check(call, lib().nvfp4_gptq_prepare_batched(
-        n, _ptrs(Hs), _i64s([h.shape[0] for h in Hs]), float(damp), _ptrs(Us), _opt(deads),
-        _opt(lambdas), _ptrs(wss), _sizes(wss), _stream(stream)))
+        n, _ptrs(Hs), _i64s(ds), float(damp), _ptrs(Us), _opt(deads), _opt(lambdas), _ptr(ws),
+        nws, _stream(stream)))
 
 
 def nvfp4_gptq_schur_replay_quantize_batched(Ws, Us, codes, scales, global_scales,
-                                             errs=None, deads=None, wss=None, params=None,
+                                             errs=None, deads=None, ws=None, params=None,
                                              stream=None):
+    """All weight matrices in one call; ws: one workspace of
+    nvfp4_quantize_batched_workspace_size bytes for the whole call."""
     call = "nvfp4_gptq_schur_replay_quantize_batched"
     n = len(Ws)
     _each(call, n, {"U": Us, "codes": codes, "scales": scales, "global_scale": global_scales,
-                    "err_out": errs, "dead": deads, "ws": wss})
-    if wss is None:
-        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "workspaces missing")
+                    "err_out": errs, "dead": deads})
     if len({w.dtype for w in Ws}) > 1:
         raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "all W must share one dtype")
     p = params if params is not None else default_params()
+    shapes = []
     for i in range(n):
         d_out, d_in = _matrix(call, Ws[i], f"W[{i}]", _IO_DTYPES)
         _need(call, Us[i], f"U[{i}]", (d_in, d_in), _F32)
@@ -469,13 +493,14 @@ def nvfp4_gptq_schur_replay_quantize_batched(Ws, Us, codes, scales, global_scale
             _opt_need(call, deads[i], f"dead[{i}]", shape=(d_in,), dtype=_U8)
         _check_solve_outputs(call, d_out, d_in, codes[i], scales[i], global_scales[i],
                              None if errs is None else errs[i])
-        _ws_bytes(call, wss[i], nvfp4_quantize_workspace_size(d_out, d_in, p))
+        shapes.append((d_out, d_in))
+    nws = _ws_bytes(call, ws, nvfp4_quantize_batched_workspace_size(shapes, p)) if n else 0
     _check(call,
            lib().nvfp4_gptq_schur_replay_quantize_batched(
-               n, _ptrs(Ws), _dtype_code(Ws[0]) if n else 0, _i64s([w.shape[0] for w in Ws]),
-               _i64s([w.shape[1] for w in Ws]), _ptrs(Us), ctypes.byref(p), _opt(deads),
-               _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _opt(errs), _ptrs(wss),
-               _sizes(wss), _stream(stream)))
+               n, _ptrs(Ws), _dtype_code(Ws[0]) if n else 0, _i64s([s[0] for s in shapes]),
+               _i64s([s[1] for s in shapes]), _ptrs(Us), ctypes.byref(p), _opt(deads),
+               _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _opt(errs), _ptr(ws), nws,
+               _stream(stream)))
 
 
 def nvfp4_dequant_batched(codes, scales, global_scales, outs, stream=None):
@@ -493,3 +518,9 @@ def nvfp4_dequant_batched(codes, scales, global_scales, outs, stream=None):
         n, _ptrs(codes), _ptrs(scales), _ptrs(global_scales), _i64s([o.shape[0] for o in outs]),
         _i64s([o.shape[1] for o in outs]), _ptrs(outs), _dtype_code(outs[0]) if n else 0,
         _stream(stream)))
+
+
+def nvfp4_set_wait_limit_ns(ns: int) -> None:
+    """Pipeline-wait limit of the library's tensor-core kernels on the
+    current device (0: the default 4 s); for testing the timeout path."""
+    _check("nvfp4_set_wait_limit_ns", lib().nvfp4_set_wait_limit_ns(int(ns)))

@@ -15,7 +15,8 @@ namespace {
 bool params_ok(const nvfp4_solve_params* p) {
   if (!p) return true;
   return p->n_candidates == kCand && p->cand_lo == -8 && p->lazy_batch == kLazyBatch &&
-         p->scale_rule >= NVFP4_RULE_SCHUR_REPLAY && p->scale_rule <= NVFP4_RULE_BLOCK_MSE;
+         p->scale_rule >= NVFP4_RULE_SCHUR_REPLAY && p->scale_rule <= NVFP4_RULE_BLOCK_MSE &&
+         p->precision == NVFP4_PRECISION_FP64_REPLAY;
 }
 
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
@@ -36,6 +37,7 @@ void nvfp4_default_params(nvfp4_solve_params* p) {
   p->cand_lo = -8;
   p->lazy_batch = kLazyBatch;
   p->scale_rule = NVFP4_RULE_SCHUR_REPLAY;
+  p->precision = NVFP4_PRECISION_FP64_REPLAY;
 }
 
 const char* nvfp4_status_string(nvfp4_status s) {

@@ -24,6 +24,36 @@ __device__ __forceinline__ void flag_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ---- groups: several problems of one shape in every launch ------------------
+// A group is P <= kMaxGroup problems of the same shape.  Its scratch lives in
+// one region: a 256-byte group header whose first int is the group's sticky
+// status word, per-problem headers, then every scratch array as P copies a
+// uniform stride apart, so that one launch (grid dimension or GEMM batch)
+// covers all P problems.  The single-problem calls are groups of one: their
+// workspace is one group region, and its first int is the status word
+// nvfp4_workspace_status() reads.  Caller-owned buffers reach the kernels as
+// per-problem pointer arrays (kernel parameters, or a table in the region).
+constexpr int kMaxGroup = 256;
+template <typename T>
+struct PtrArr {
+  T p[kMaxGroup];
+};
+
+// Batched calls: one workspace for all problems -- a batch header (the first
+// int: the first non-OK status of any problem; then one status word per
+// problem in the caller's order), then one group region per run of problems
+// of equal shape (problems grouped by shape in their order of appearance, at
+// most kMaxGroup per group).
+__host__ __device__ inline size_t batch_header_bytes(int count) {
+  return align256(sizeof(int) * (1 + (size_t)count));
+}
+// Copies each group problem's status (its own word, else the group's word)
+// into the batch header at the problem's index in the call: idx[i] for
+// problem i of the group; per_problem_status[i] points at problem i's word.
+nvfp4_status gather_group_status(int* batch_hdr, const int* group_status,
+                                 const PtrArr<const int*>& per_problem_status,
+                                 const PtrArr<int>& idx, int P, cudaStream_t st);
+
 inline cudaStream_t as_cuda(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // ---- launch accounting and optional per-phase event timing (runtime.cu) ----
@@ -134,6 +164,10 @@ nvfp4_status launch_hessian_host(float* H, const void* X_host, nvfp4_dtype xt, i
                                  cudaStream_t st);
 nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
                                cudaStream_t st);
+// P problems of one dimension d, each hessian_tc_supported (ragged n_tok).
+nvfp4_status launch_hessian_tc_group(int P, float* const* H, const void* const* X,
+                                     const int64_t* n_tok, int64_t d, int beta,
+                                     cudaStream_t st);
 int hessian_tc_take_status(cudaStream_t st);
 
 // TMA descriptors of the tensor-core trailing update: Delta = Dh + Dl
@@ -144,20 +178,37 @@ struct UpdateMaps {
 };
 // Maps of the update operands: Dh/Dl (d_out x kcols) and Uh/Ul (d_in x kcols)
 // hold deltas and U rows K-contiguous, kcols K values per row.
+// P problems of a group: each array repeats P times, a whole matrix apart.
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
                       const float* Ul, const double* Wt, int64_t d_out, int64_t d_in,
-                      int64_t kcols);
+                      int64_t kcols, int P);
 // W~[:, e:e_end] -= sum over nkb 128-deep K blocks from K offset kofs of
 // (Dh + Dl)(Uh + Ul)^T (3xTF32, fp64 W~); keep_w keeps W~ in L2 (evict last)
 // instead of streaming it.  A timed-out wait sets NVFP4_ERR_TIMEOUT in *status.
 nvfp4_status launch_update_tc(const UpdateMaps& m, int64_t d_out, int64_t d_in, int64_t e,
-                              int64_t e_end, int kofs, int nkb, bool keep_w, int* status,
+                              int64_t e_end, int kofs, int nkb, bool keep_w, int P, int* status,
                               cudaStream_t st);
 nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                             int64_t d, int beta, cudaStream_t st);
 nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,
                             uint8_t* dead, float* lambda_out, void* ws, cudaStream_t st);
 size_t prepare_ws_bytes(int64_t d);
+// Groups of P problems of one shape (kernels launched once for all P); ws is
+// the group region of *_group_ws_bytes() bytes.
+size_t prepare_group_ws_bytes(int64_t d, int P);
+nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t d, float damp,
+                                  const PtrArr<float*>& U, const PtrArr<uint8_t*>& dead,
+                                  const PtrArr<float*>& lambda_out, void* ws, cudaStream_t st);
+const int* prepare_group_problem_status(const void* ws, int i);
+size_t quantize_group_ws_bytes(int64_t d_out, int64_t d_in, int P);
+nvfp4_status launch_quantize_group(int P, const PtrArr<const void*>& W, nvfp4_dtype wt,
+                                   int64_t d_out, int64_t d_in, const PtrArr<const float*>& U,
+                                   const PtrArr<const uint8_t*>& dead, int rule,
+                                   const PtrArr<uint8_t*>& codes, const PtrArr<uint8_t*>& scales,
+                                   const PtrArr<float*>& sg, const PtrArr<double*>& err,
+                                   const PtrArr<const float*>& amax_in, void* ws,
+                                   cudaStream_t st);
+const int* quantize_group_problem_status(const void* ws, int i);
 nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
                              const float* U, const uint8_t* dead, int rule, uint8_t* codes,
                              uint8_t* scales, float* sg, double* err, void* ws,
@@ -171,6 +222,10 @@ size_t quantize_ws_bytes(int64_t d_out, int64_t d_in);
 nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* sg,
                             int64_t d_out, int64_t d_in, void* out, nvfp4_dtype ot,
                             cudaStream_t st);
+nvfp4_status launch_dequant_group(int P, const PtrArr<const uint8_t*>& codes,
+                                  const PtrArr<const uint8_t*>& scales,
+                                  const PtrArr<const float*>& sg, const PtrArr<void*>& out,
+                                  int64_t d_out, int64_t d_in, nvfp4_dtype ot, cudaStream_t st);
 nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* codes,
                                 const uint8_t* scales, const float* sg, const float* H,
                                 int64_t d_out, int64_t d_in, double* err, void* ws,

@@ -24,38 +24,62 @@ __device__ __forceinline__ uint16_t bf16_of_product(float cs, float sg) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(hi));
 }
 
-// One thread per 16-weight block: 8 code bytes + 1 scale byte in, 16 values out.
+// The 16 dequantized values of one block: code bytes c (low nibble first),
+// scale code sc, written to o (16 bf16 = 32 bytes, or 16 fp32 = 64 bytes).
 template <bool kBF16>
-__global__ void dequant_kernel(const uint8_t* __restrict__ codes,
-                               const uint8_t* __restrict__ scales,
-                               const float* __restrict__ sg_ptr, int64_t nblocks,
-                               void* __restrict__ out) {
-  const float sg = *sg_ptr;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks;
-       b += (int64_t)gridDim.x * blockDim.x) {
-    const uint2 c = reinterpret_cast<const uint2*>(codes)[b];
-    const float sb = (float)e4m3_value(scales[b] & 0x7F);
-    const uint64_t p = ((uint64_t)c.y << 32) | c.x;
-    float cs[16];
+__device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, void* o) {
+  const float sb = (float)e4m3_value(sc & 0x7F);
+  const uint64_t p = ((uint64_t)c.y << 32) | c.x;
+  float cs[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) cs[j] = e2m1_value((uint32_t)(p >> (4 * j)) & 0xF) * sb;
-    if constexpr (kBF16) {
-      uint32_t h[8];
+  for (int j = 0; j < 16; ++j) cs[j] = e2m1_value((uint32_t)(p >> (4 * j)) & 0xF) * sb;
+  if constexpr (kBF16) {
+    uint32_t h[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        h[j] = (uint32_t)bf16_of_product(cs[2 * j], sg) |
-               ((uint32_t)bf16_of_product(cs[2 * j + 1], sg) << 16);
-      uint4* o = reinterpret_cast<uint4*>(out) + 2 * b;
-      o[0] = make_uint4(h[0], h[1], h[2], h[3]);
-      o[1] = make_uint4(h[4], h[5], h[6], h[7]);
-    } else {
-      float4* o = reinterpret_cast<float4*>(out) + 4 * b;
+    for (int j = 0; j < 8; ++j)
+      h[j] = (uint32_t)bf16_of_product(cs[2 * j], sg) |
+             ((uint32_t)bf16_of_product(cs[2 * j + 1], sg) << 16);
+    uint4* q = reinterpret_cast<uint4*>(o);
+    q[0] = make_uint4(h[0], h[1], h[2], h[3]);
+    q[1] = make_uint4(h[4], h[5], h[6], h[7]);
+  } else {
+    float4* q = reinterpret_cast<float4*>(o);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        o[q] = make_float4(cs[4 * q] * sg, cs[4 * q + 1] * sg, cs[4 * q + 2] * sg,
-                           cs[4 * q + 3] * sg);
-    }
+    for (int k = 0; k < 4; ++k)
+      q[k] = make_float4(cs[4 * k] * sg, cs[4 * k + 1] * sg, cs[4 * k + 2] * sg,
+                         cs[4 * k + 3] * sg);
   }
+}
+
+// Problem blockIdx.y of a group.  Each thread step takes four consecutive
+// 16-weight blocks (32 code bytes + 4 scale bytes in, their 64 values out),
+// all loads issued before any use; a tail of fewer than four blocks goes one
+// block per thread.
+template <bool kBF16>
+__global__ void dequant_kernel(PtrArr<const uint8_t*> codes_a, PtrArr<const uint8_t*> scales_a,
+                               PtrArr<const float*> sg_a, PtrArr<void*> out_a,
+                               int64_t nblocks) {
+  const int pb = blockIdx.y;
+  const uint2* __restrict__ codes = reinterpret_cast<const uint2*>(codes_a.p[pb]);
+  const uint8_t* __restrict__ scales = scales_a.p[pb];
+  uint8_t* out = static_cast<uint8_t*>(out_a.p[pb]);
+  constexpr int kOut = kBF16 ? 32 : 64;   // output bytes per block
+  const float sg = *sg_a.p[pb];
+  const int64_t nq = nblocks / 4;
+  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t step = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t q = t0; q < nq; q += step) {
+    uint2 c[4];
+    uint32_t sc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) c[k] = codes[4 * q + k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sc[k] = scales[4 * q + k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dequant_block<kBF16>(c[k], sc[k], sg, out + (4 * q + k) * kOut);
+  }
+  for (int64_t b = 4 * nq + t0; b < nblocks; b += step)
+    dequant_block<kBF16>(codes[b], scales[b], sg, out + b * kOut);
 }
 
 // Et = (W - Q)^T in fp32 (W bf16 or fp32) for a 64 x 64 tile of W: one
@@ -180,18 +204,35 @@ constexpr int kDotBlocks = 8 * kNumSMs;
 
 }  // namespace
 
-nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* sg,
-                            int64_t d_out, int64_t d_in, void* out, nvfp4_dtype ot,
-                            cudaStream_t st) {
+// P problems of one shape (codes, scales, s_g and outputs per problem).
+nvfp4_status launch_dequant_group(int P, const PtrArr<const uint8_t*>& codes,
+                                  const PtrArr<const uint8_t*>& scales,
+                                  const PtrArr<const float*>& sg, const PtrArr<void*>& out,
+                                  int64_t d_out, int64_t d_in, nvfp4_dtype ot, cudaStream_t st) {
   const int64_t nb = d_out * (d_in / kBlock);
-  if (nb == 0) return NVFP4_OK;
+  if (nb == 0 || P < 1) return NVFP4_OK;
+  int g = grid_for((nb + 3) / 4, 256) / P;
+  const dim3 grid((unsigned)(g < 1 ? 1 : g), (unsigned)P);
   if (ot == NVFP4_BF16)
-    dequant_kernel<true><<<grid_for(nb, 256), 256, 0, st>>>(codes, scales, sg, nb, out);
+    dequant_kernel<true><<<grid, 256, 0, st>>>(codes, scales, sg, out, nb);
   else
-    dequant_kernel<false><<<grid_for(nb, 256), 256, 0, st>>>(codes, scales, sg, nb, out);
+    dequant_kernel<false><<<grid, 256, 0, st>>>(codes, scales, sg, out, nb);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;
+}
+
+nvfp4_status launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* sg,
+                            int64_t d_out, int64_t d_in, void* out, nvfp4_dtype ot,
+                            cudaStream_t st) {
+  PtrArr<const uint8_t*> c, s;
+  PtrArr<const float*> g;
+  PtrArr<void*> o;
+  c.p[0] = codes;
+  s.p[0] = scales;
+  g.p[0] = sg;
+  o.p[0] = out;
+  return launch_dequant_group(1, c, s, g, o, d_out, d_in, ot, st);
 }
 
 int64_t et_ld(int64_t d_out) { return (d_out + 31) / 32 * 32; }

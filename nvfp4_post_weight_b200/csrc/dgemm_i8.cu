@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kIThreads, 1)
       }
     }
     for (int i = g - kIStages < 0 ? 0 : g - kIStages; i < g; ++i)
-      mbar_wait(&sm->full[i % kIStages], (i / kIStages) & 1);
+      mbar_wait_drain(&sm->full[i % kIStages], (i / kIStages) & 1);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     int g = 0, lt = 0;
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kIThreads, 1)
     // nothing of this thread's may still run on the tensor cores when TMEM is
     // freed, also after a wait ran out
     mma_commit(&sm->done);
-    mbar_wait(&sm->done, 0);
+    mbar_wait_drain(&sm->done, 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // (1) the levels of each row are summed in fp64 straight out of TMEM,

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(Cfg<TL>::kThreads)
       }
       // whatever happened, no copy may still be in flight when the CTA exits
       for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
-        mbar_wait(&bars->full[i % kStages], (i / kStages) & 1);
+        mbar_wait_drain(&bars->full[i % kStages], (i / kStages) & 1);
     }
     return;
   }

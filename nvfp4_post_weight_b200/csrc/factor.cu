@@ -20,7 +20,7 @@ namespace {
 
 constexpr int NB = 64;  // diagonal block (panel) width
 
-struct PrepHeader {   // lives in the workspace header (first 256 bytes)
+struct PrepHeader {   // one per problem of a group
   int status;
   int pad;
   double diag_sum;
@@ -28,17 +28,25 @@ struct PrepHeader {   // lives in the workspace header (first 256 bytes)
   double lambda64;    // used for the damping
 };
 
-// Sum of the diagonal (dead entries counted as 1), dead flags, lambda.
-__global__ void diag_stats_kernel(const float* __restrict__ H, int64_t d, float damp,
-                                  uint8_t* __restrict__ dead, float* __restrict__ lambda_out,
-                                  PrepHeader* hdr) {
+// Sum of the diagonal (dead entries counted as 1), dead flags, lambda.  One
+// CTA per problem of the group (blockIdx.x).
+__global__ void diag_stats_kernel(PtrArr<const float*> Hs, int64_t d, float damp,
+                                  PtrArr<uint8_t*> deads, PtrArr<float*> lambdas,
+                                  PrepHeader* hdrs, int* gstatus) {
   __shared__ double part[32];
+  const int pb = blockIdx.x;
+  const float* __restrict__ H = Hs.p[pb];
+  uint8_t* dead = deads.p[pb];
+  PrepHeader* hdr = hdrs + pb;
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < d; i += blockDim.x) {
     const float h = H[i * d + i];
     const bool is_dead = (h == 0.f);
     if (dead) dead[i] = is_dead ? 1 : 0;
-    if (!isfinite(h)) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+    if (!isfinite(h)) {
+      flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+      flag_status(gstatus, NVFP4_ERR_NONFINITE);
+    }
     s += is_dead ? 1.0 : (double)h;
   }
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -53,18 +61,27 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int64_t d, float 
       const float lam = (float)lam64;
       hdr->lambda = lam;
       hdr->lambda64 = lam64;
-      if (lambda_out) *lambda_out = lam;
+      if (lambdas.p[pb]) *lambdas.p[pb] = lam;
     }
   }
 }
 
 // A[i][j] = H_d[d-1-i][d-1-j]; dead diagonal entries become 1 + lambda.
-// Also zero-fills X (the inverse is built from its block diagonal outward).
-// Rows blockIdx.y, + gridDim.y, ...; four consecutive columns per thread (d
-// is a multiple of 16); H read as float4 when it is 16-byte aligned (vec).
-__global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
-                                    double* __restrict__ A, double* __restrict__ X,
-                                    PrepHeader* hdr, int vec) {
+// Also zero-fills X and Y (the inverse is built from its block diagonal
+// outward).  Rows blockIdx.y, + gridDim.y, ...; four consecutive columns per
+// thread (d is a multiple of 16); H read as float4 when it is 16-byte aligned.
+// Problem blockIdx.z of the group: its matrices sa elements after the
+// previous problem's.
+__global__ void reverse_damp_kernel(PtrArr<const float*> Hs, int64_t d, double* __restrict__ A,
+                                    double* __restrict__ X, double* __restrict__ Y, int64_t sa,
+                                    PrepHeader* hdrs, int* gstatus) {
+  const int pb = blockIdx.z;
+  const float* __restrict__ H = Hs.p[pb];
+  PrepHeader* hdr = hdrs + pb;
+  A += pb * sa;
+  X += pb * sa;
+  Y += pb * sa;
+  const bool vec = (reinterpret_cast<uintptr_t>(H) & 15) == 0;
   const double lam = hdr->lambda64;
   const int64_t j = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
   if (j >= d) return;
@@ -87,13 +104,19 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int64_t d,
       a[q] = (double)hv[q];
       if (i == j + q) a[q] = (hv[q] == 0.f ? 1.0 : a[q]) + lam;
     }
-    if (bad) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+    if (bad) {
+      flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+      flag_status(gstatus, NVFP4_ERR_NONFINITE);
+    }
     double2* Ar = reinterpret_cast<double2*>(A + i * d + j);   // workspace: aligned
     double2* Xr = reinterpret_cast<double2*>(X + i * d + j);
+    double2* Yr = reinterpret_cast<double2*>(Y + i * d + j);
     Ar[0] = make_double2(a[0], a[1]);
     Ar[1] = make_double2(a[2], a[3]);
     Xr[0] = make_double2(0.0, 0.0);
     Xr[1] = make_double2(0.0, 0.0);
+    Yr[0] = make_double2(0.0, 0.0);
+    Yr[1] = make_double2(0.0, 0.0);
   }
 }
 
@@ -152,7 +175,7 @@ constexpr size_t kPanelSmem = sizeof(double) * ((3 * NB + kSlice) * kPitch + NB)
 // (lower part) and write L_KK back into S (zeros above) and 1/L_jj into invd.
 // A non-positive pivot is flagged and taken as 1.
 __device__ __forceinline__ void factor_16(double (*S)[kPitch], double* invd, int o,
-                                          PrepHeader* hdr) {
+                                          PrepHeader* hdr, int* gstatus) {
   const int lane = threadIdx.x & 31;
   const int i = lane & 15;
   const unsigned full = 0xffffffffu;
@@ -175,7 +198,10 @@ __device__ __forceinline__ void factor_16(double (*S)[kPitch], double* invd, int
       r[l] = fma(-a, cl, r[l]);
     }
   }
-  if (bad && lane == 0) flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
+  if (bad && lane == 0) {
+    flag_status(&hdr->status, NVFP4_ERR_NOT_PD);
+    flag_status(gstatus, NVFP4_ERR_NOT_PD);
+  }
   // L[i][l] = r[l] / sqrt(p_l) (l < i), L[i][i] = sqrt(p_i)
   double sq[kSub], isq[kSub];
 #pragma unroll
@@ -269,7 +295,13 @@ __device__ __forceinline__ void doubling_level(double (*S)[kPitch], double (*Xd)
 
 __global__ void __launch_bounds__(kPanelThreads)
     chol_panel_kernel(double* __restrict__ A, int64_t d, int64_t k, int kb,
-                      double* __restrict__ X, double* __restrict__ Y, PrepHeader* hdr) {
+                      double* __restrict__ X, double* __restrict__ Y, int64_t sa,
+                      PrepHeader* hdrs, int* gstatus) {
+  // problem blockIdx.y of the group
+  A += blockIdx.y * sa;
+  X += blockIdx.y * sa;
+  Y += blockIdx.y * sa;
+  PrepHeader* hdr = hdrs + blockIdx.y;
   extern __shared__ double dsm[];
   double(*S)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm);             // A11 -> L11
   double(*Xd)[kPitch] = reinterpret_cast<double(*)[kPitch]>(dsm + NB * kPitch);   // X11
@@ -316,7 +348,7 @@ __global__ void __launch_bounds__(kPanelThreads)
 #pragma unroll 1
   for (int K = 0; K < NB / kSub; ++K) {
     const int o = K * kSub;
-    if (warp == 0) factor_16(S, invd, o, hdr);
+    if (warp == 0) factor_16(S, invd, o, hdr, gstatus);
     __syncthreads();
     const int nb = NB - o - kSub;   // rows below the sub-block (48, 32, 16 or 0)
     if (nb == 0) break;
@@ -409,8 +441,11 @@ __global__ void __launch_bounds__(kPanelThreads)
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.  Rows
 // blockIdx.y, + gridDim.y, ...; four consecutive columns per thread, U
 // written as float4 when it is 16-byte aligned (vec).
-__global__ void reverse_to_upper_kernel(const double* __restrict__ X, int64_t d,
-                                        float* __restrict__ U, int vec) {
+__global__ void reverse_to_upper_kernel(const double* __restrict__ X, int64_t d, int64_t sa,
+                                        PtrArr<float*> Us) {
+  float* __restrict__ U = Us.p[blockIdx.z];   // problem blockIdx.z of the group
+  X += blockIdx.z * sa;
+  const bool vec = (reinterpret_cast<uintptr_t>(U) & 15) == 0;
   const int64_t j = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
   if (j >= d) return;
   for (int64_t i = blockIdx.y; i < d; i += gridDim.y) {
@@ -433,61 +468,88 @@ __global__ void reverse_to_upper_kernel(const double* __restrict__ X, int64_t d,
   }
 }
 
+// A group region of the prepare: the group header (its first int the status
+// word), P problem headers, then P copies each of A, X, Y (sa = d (d + 1)
+// elements apart: one d x d matrix and d elements of padding, so that the
+// pairs of the inverse doubling of all P problems sit one stride apart when
+// 2b divides d), the doubling scratch T and the int8-slice scratch.
 struct PrepLayout {
+  int* gstatus;
   PrepHeader* hdr;
-  double* A;   // J H_d J, then its Cholesky factor L (lower)
-  double* X;   // L^-1 (lower)
-  double* Y;   // L^-T (upper)
-  double* T;   // scratch of the inverse doubling
-  void* S8;    // int8 slices of the tensor-core fp64 GEMMs
+  int64_t sa;   // elements between the problems' A (X, Y) matrices
+  double* A;    // J H_d J, then its Cholesky factor L (lower)
+  double* X;    // L^-1 (lower)
+  double* Y;    // L^-T (upper)
+  double* T;    // scratch of the inverse doubling
+  void* S8;     // int8 slices of the tensor-core fp64 GEMMs
   size_t s8_bytes;
 };
 
-// Slice scratch of the int8-slice GEMMs: the largest operand pair of a call
-// (trailing update: d x 256 twice; doubling level b: d/2b pairs of b x b,
-// twice) is below the bound for M = N = d, K = d/2.
-size_t slice_scratch_bytes(int64_t d) { return dgemm_i8_scratch_bytes(d, d, (d / 2 + 15) / 16 * 16 + 256, 1); }
+// Doubling scratch per problem: a level's pairs (d / 2b of b x b) or its
+// ragged pair (b x rr, rr < b), at most d^2 / 4; plus room for d x NB.
+int64_t t_elems(int64_t d) { return (d * d + 3) / 4 + d * NB; }
 
-PrepLayout prep_layout(void* ws, int64_t d) {
+// Slice scratch of the int8-slice GEMMs for P problems: the largest operand
+// pair of a call (trailing update: d x 512 twice; doubling level b: d/2b
+// pairs of b x b, twice) per problem is below the bound for M = N = d,
+// K = d/2.
+size_t slice_scratch_bytes(int64_t d, int P) {
+  return dgemm_i8_scratch_bytes(d, d, (d / 2 + 15) / 16 * 16 + 256, P);
+}
+
+size_t prep_group_bytes(int64_t d, int P) {
+  const int64_t sa = d * (d + 1);
+  return kWsHeader + align256(sizeof(PrepHeader) * P) + 3 * align256(sizeof(double) * sa * P) +
+         align256(sizeof(double) * (size_t)t_elems(d) * P) + align256(slice_scratch_bytes(d, P));
+}
+
+PrepLayout prep_layout(void* ws, int64_t d, int P) {
   char* p = static_cast<char*>(ws);
   PrepLayout L;
-  L.hdr = reinterpret_cast<PrepHeader*>(p);
+  L.gstatus = reinterpret_cast<int*>(p);
   size_t off = kWsHeader;
+  L.hdr = reinterpret_cast<PrepHeader*>(p + off);
+  off += align256(sizeof(PrepHeader) * P);
+  L.sa = d * (d + 1);
   L.A = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * d * d);
+  off += align256(sizeof(double) * L.sa * P);
   L.X = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * d * d);
+  off += align256(sizeof(double) * L.sa * P);
   L.Y = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * d * d);
+  off += align256(sizeof(double) * L.sa * P);
   L.T = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB));
+  off += align256(sizeof(double) * (size_t)t_elems(d) * P);
   L.S8 = p + off;
-  L.s8_bytes = slice_scratch_bytes(d);
+  L.s8_bytes = slice_scratch_bytes(d, P);
   return L;
 }
 
 }  // namespace
 
-size_t prepare_ws_bytes(int64_t d) {
-  return kWsHeader + 3 * align256(sizeof(double) * d * d) +
-         align256(sizeof(double) * (size_t)((d * d + 3) / 4 + d * NB)) +
-         align256(slice_scratch_bytes(d));
-}
+size_t prepare_ws_bytes(int64_t d) { return prep_group_bytes(d, 1); }
+size_t prepare_group_ws_bytes(int64_t d, int P) { return prep_group_bytes(d, P); }
 
-nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uint8_t* dead,
-                            float* lambda_out, void* ws, cudaStream_t st) {
-  PrepLayout L = prep_layout(ws, d);
-  NVFP4_CUDA_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(PrepHeader), st));
-  diag_stats_kernel<<<1, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr);
+// The prepare of a group of P problems of dimension d (every launch covers all
+// P): ws is the group region (prepare_group_ws_bytes(d, P) bytes).  A problem
+// whose factor meets a non-positive pivot or a non-finite H has its own
+// header's status set; the group word at the start of ws collects the first
+// status of any problem and the GEMMs' timeouts.
+nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t d, float damp,
+                                  const PtrArr<float*>& U, const PtrArr<uint8_t*>& dead,
+                                  const PtrArr<float*>& lambda_out, void* ws,
+                                  cudaStream_t st) {
+  if (P < 1 || P > kMaxGroup) return NVFP4_ERR_INVALID_ARG;
+  PrepLayout L = prep_layout(ws, d, P);
+  NVFP4_CUDA_TRY(cudaMemsetAsync(ws, 0, kWsHeader + align256(sizeof(PrepHeader) * P), st));
+  diag_stats_kernel<<<P, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr, L.gstatus);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-  const dim3 rgrid((unsigned)((d / 4 + 255) / 256), (unsigned)(d < 65535 ? d : 65535));
-  reverse_damp_kernel<<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.hdr,
-                                             (reinterpret_cast<uintptr_t>(H) & 15) == 0);
+  const dim3 rgrid((unsigned)((d / 4 + 255) / 256), (unsigned)(d < 65535 ? d : 65535),
+                   (unsigned)P);
+  reverse_damp_kernel<<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.Y, L.sa, L.hdr, L.gstatus);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-
-  NVFP4_CUDA_TRY(cudaMemsetAsync(L.Y, 0, sizeof(double) * d * d, st));
+  const int64_t sa = L.sa;
 
   // Blocked right-looking Cholesky of A (lower), two levels: 64-column panels
   // (one fused panel kernel each: diagonal factor + inverse + panel solve)
@@ -501,15 +563,15 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
   // levels from 256) go to the int8-slice tensor-core engine, the small and
   // narrow ones to mma.sync fp64, whose latency is lower
   constexpr int64_t kBigGemm = 512;
-  auto gemm = [&](bool big, int M, int N, int K, double alpha, const double* P, int64_t ldp,
+  auto gemm = [&](bool big, int M, int N, int K, double alpha, const double* Pm, int64_t ldp,
                   int64_t sP, const double* Q, int64_t ldq, int64_t sQ, double beta, double* C,
                   int64_t ldc, int64_t sC, double* C2, int64_t ldc2, int64_t sC2, int batch,
                   int lower, int ktri) {
     if (big && K < (1 << 16))
-      return dgemm_i8(M, N, K, alpha, P, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2,
-                      batch, lower, ktri, L.S8, L.s8_bytes, &L.hdr->status, st);
-    return dgemm_nt(M, N, K, alpha, P, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2, batch,
-                    lower, ktri, &L.hdr->status, st);
+      return dgemm_i8(M, N, K, alpha, Pm, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2,
+                      batch, lower, ktri, L.S8, L.s8_bytes, L.gstatus, st);
+    return dgemm_nt(M, N, K, alpha, Pm, ldp, sP, Q, ldq, sQ, beta, C, ldc, sC, C2, ldc2, sC2,
+                    batch, lower, ktri, L.gstatus, st);
   };
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(chol_panel_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -523,61 +585,103 @@ nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uin
       {
         ProfileScope ps(kPhasePanel, st);
         // Cholesky and inverse of the kb x kb block, and the m x kb slice solve
-        add_phase_work(2.0 * kb * kb * kb / 3.0 + (double)m * kb * kb);
-        NVFP4_CUDA_TRY(launch_chained(chol_panel_kernel, dim3(grid), dim3(kPanelThreads),
-                                      kPanelSmem, st, L.A, d, k, kb, L.X, L.Y, L.hdr));
+        add_phase_work(P * (2.0 * kb * kb * kb / 3.0 + (double)m * kb * kb));
+        NVFP4_CUDA_TRY(launch_chained(chol_panel_kernel, dim3(grid, P), dim3(kPanelThreads),
+                                      kPanelSmem, st, L.A, d, k, kb, L.X, L.Y, sa, L.hdr,
+                                      L.gstatus));
         count_launches(1);
       }
       const int64_t nc = kend - (k + kb);   // columns of the outer block still to come
       if (m <= 0 || nc <= 0) continue;
       const double* L21 = L.A + (k + kb) * d + k;
-      nvfp4_status s = dgemm_nt((int)m, (int)nc, kb, -1.0, L21, d, 0, L21, d, 0, 1.0,
-                                L.A + (k + kb) * (d + 1), d, 0, nullptr, 0, 0, 1, 0, 0, &L.hdr->status, st);
+      nvfp4_status s = dgemm_nt((int)m, (int)nc, kb, -1.0, L21, d, sa, L21, d, sa, 1.0,
+                                L.A + (k + kb) * (d + 1), d, sa, nullptr, 0, 0, P, 0, 0,
+                                L.gstatus, st);
       if (s != NVFP4_OK) return s;
     }
     const int64_t m2 = d - kend;
     if (m2 > 0) {
       const double* Lb = L.A + kend * d + k0;
-      nvfp4_status s = gemm(m2 >= kBigGemm, (int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, 0,
-                            Lb, d, 0, 1.0, L.A + kend * (d + 1), d, 0, nullptr, 0, 0, 1, 1, 0);
+      nvfp4_status s = gemm(m2 >= kBigGemm, (int)m2, (int)m2, (int)(kend - k0), -1.0, Lb, d, sa,
+                            Lb, d, sa, 1.0, L.A + kend * (d + 1), d, sa, nullptr, 0, 0, P, 1, 0);
       if (s != NVFP4_OK) return s;
     }
   }
 
   // X = L^-1 by recursive doubling over pairs of adjacent diagonal blocks of
-  // size b (all pairs of one level at once):  with L = [L11 0; L21 L22],
+  // size b (all pairs of one level, of all P problems, at once):  with
+  // L = [L11 0; L21 L22],
   //   T^T = Y11 L21^T,  X21 = -X22 T,  Y12 = X21^T   (Y = X^T throughout),
-  // so every product is of the form P Q^T with K-contiguous operands.
+  // so every product is of the form P Q^T with K-contiguous operands.  The
+  // pairs of a level lie 2b (d + 1) apart inside a problem; across problems
+  // that is still one stride when 2b divides d (sa = (d / 2b) 2b (d + 1)) or
+  // when there is one pair per problem (stride sa); otherwise the level runs
+  // problem by problem.
+  auto level = [&](int64_t b, int64_t npairs, const double* base_off_A, int nbatch,
+                   int64_t stride, double* T) -> nvfp4_status {
+    const bool big = b >= kBigGemm / 2;
+    const int64_t o = base_off_A - L.A;   // element offset of the first pair's block
+    nvfp4_status s = gemm(big, (int)b, (int)b, (int)b, 1.0, L.Y + o, d, stride,
+                          L.A + o + b * d, d, stride, 0.0, T, b, b * b, nullptr, 0, 0, nbatch,
+                          0, 1);
+    if (s != NVFP4_OK) return s;
+    (void)npairs;
+    return gemm(big, (int)b, (int)b, (int)b, -1.0, L.X + o + b * (d + 1), d, stride, T, b,
+                b * b, 0.0, L.X + o + b * d, d, stride, L.Y + o + b, d, stride, nbatch, 0, 2);
+  };
   for (int64_t b = NB; b < d; b *= 2) {
     const int64_t npairs = d / (2 * b);
     const int64_t stride = 2 * b * (d + 1);
-    const bool big = b >= kBigGemm / 2;
     if (npairs > 0) {
-      nvfp4_status s = gemm(big, (int)b, (int)b, (int)b, 1.0, L.Y, d, stride, L.A + b * d, d,
-                            stride, 0.0, L.T, b, b * b, nullptr, 0, 0, (int)npairs, 0, 1);
-      if (s != NVFP4_OK) return s;
-      s = gemm(big, (int)b, (int)b, (int)b, -1.0, L.X + b * (d + 1), d, stride, L.T, b, b * b,
-               0.0, L.X + b * d, d, stride, L.Y + b, d, stride, (int)npairs, 0, 2);
+      nvfp4_status s;
+      if (P == 1 || d % (2 * b) == 0) {
+        s = level(b, npairs, L.A, (int)(npairs * P), stride, L.T);
+      } else if (npairs == 1) {
+        s = level(b, npairs, L.A, P, sa, L.T);
+      } else {
+        s = NVFP4_OK;
+        for (int pb = 0; pb < P && s == NVFP4_OK; ++pb)
+          s = level(b, npairs, L.A + pb * sa, (int)npairs, stride, L.T + pb * npairs * b * b);
+      }
       if (s != NVFP4_OK) return s;
     }
     const int64_t r0 = npairs * 2 * b;   // a ragged pair: full left block, rr rows right
     const int64_t rr = d - r0 - b;
     if (rr > 0) {
       const int64_t o = r0 * (d + 1);
-      nvfp4_status s = gemm(big, (int)b, (int)rr, (int)b, 1.0, L.Y + o, d, 0, L.A + o + b * d, d,
-                            0, 0.0, L.T, rr, 0, nullptr, 0, 0, 1, 0, 1);
+      nvfp4_status s = gemm(b >= kBigGemm / 2, (int)b, (int)rr, (int)b, 1.0, L.Y + o, d, sa,
+                            L.A + o + b * d, d, sa, 0.0, L.T, rr, b * rr, nullptr, 0, 0, P, 0,
+                            1);
       if (s != NVFP4_OK) return s;
       // X21 (rr x b) = -X22 (rr x rr) T (rr x b): P = X22, Q = T^T (b x rr)
-      s = gemm(big, (int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, 0, L.T, rr, 0,
-               0.0, L.X + o + b * d, d, 0, L.Y + o + b, d, 0, 1, 0, 2);
+      s = gemm(b >= kBigGemm / 2, (int)rr, (int)b, (int)rr, -1.0, L.X + o + b * (d + 1), d, sa,
+               L.T, rr, b * rr, 0.0, L.X + o + b * d, d, sa, L.Y + o + b, d, sa, P, 0, 2);
       if (s != NVFP4_OK) return s;
     }
   }
-  reverse_to_upper_kernel<<<rgrid, 256, 0, st>>>(L.X, d, U,
-                                                 (reinterpret_cast<uintptr_t>(U) & 15) == 0);
+  reverse_to_upper_kernel<<<rgrid, 256, 0, st>>>(L.X, d, sa, U);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   return NVFP4_OK;
+}
+
+// The single-problem prepare: a group of one whose region is ws.
+nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uint8_t* dead,
+                            float* lambda_out, void* ws, cudaStream_t st) {
+  PtrArr<const float*> h;
+  PtrArr<float*> u, lam;
+  PtrArr<uint8_t*> dd;
+  h.p[0] = H;
+  u.p[0] = U;
+  dd.p[0] = dead;
+  lam.p[0] = lambda_out;
+  return launch_prepare_group(1, h, d, damp, u, dd, lam, ws, st);
+}
+
+// Problem i's status word of a prepare group region.
+const int* prepare_group_problem_status(const void* ws, int i) {
+  const char* p = static_cast<const char*>(ws) + kWsHeader;
+  return reinterpret_cast<const int*>(p + sizeof(PrepHeader) * i);
 }
 
 }  // namespace nvfp4

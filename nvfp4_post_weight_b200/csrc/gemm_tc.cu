@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s = kStages - 1;
           ph ^= 1;
         }
-        mbar_wait(&sm->full[s], ph);
+        mbar_wait_drain(&sm->full[s], ph);
       }
     }
   } else if (warp >= 2 && warp < 6 && !presplit) {
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     mma_commit(&sm->drain);
-    mbar_wait(&sm->drain, 0);
+    mbar_wait_drain(&sm->drain, 0);
   } else if (warp >= 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;

@@ -50,6 +50,18 @@ constexpr size_t kSmem = kStages * kStageBytes + 1024 + 256;
 
 __device__ int g_hessian_status;
 
+// Up to kHessGroup problems of the same dimension d in one launch: their
+// token maps, outputs and token counts (a kernel parameter, 18 KB).  Tile t
+// of the launch is band tile t % per of problem t / per; the host orders the
+// problems by decreasing token count, so the longest tiles come first.
+constexpr int kHessGroup = 128;
+struct HessGroup {
+  CUtensorMap map[kHessGroup];
+  float* H[kHessGroup];
+  int n_tok[kHessGroup];
+  int P;
+};
+
 struct BandTiles {   // 128 x 256 tiles (I, J) with J >= I / 2, row-major
   int nI, nJ;
   __host__ __device__ int row_count(int I) const { return nJ - (I >> 1); }
@@ -88,15 +100,15 @@ __device__ __forceinline__ bool aborted(Smem* sm) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, float* __restrict__ H, int d,
-                      int n_tok, int beta, BandTiles band) {
+    hessian_tc_kernel(const __grid_constant__ HessGroup grp, int d, int beta, BandTiles band) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(tiles + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = band.total();
-  const int nk = (n_tok + BK - 1) / BK;
+  const int per = band.total();
+  const int n_tiles = per * grp.P;
+  auto nk_of = [&](int pb) { return (grp.n_tok[pb] + BK - 1) / BK; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -119,13 +131,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    tma_prefetch(&tmX);
     int s = 0;
     uint32_t ph = 0;
     int issued = 0;
     for (int t = blockIdx.x; t < n_tiles && !aborted(sm); t += gridDim.x) {
+      const int pb = t / per;
+      const CUtensorMap* tmX = &grp.map[pb];
+      const int nk = nk_of(pb);
       int I, J;
-      band.get(t, I, J);
+      band.get(t - pb * per, I, J);
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait(&sm->empty[s], ph ^ 1)) {
           give_up(sm);
@@ -135,9 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* a = tiles + s * kStageBytes;
         uint8_t* b = a + kABytes;
         for (int x = 0; x < BM / kBox; ++x)
-          tma_load_2d(a + x * kBoxBytes, &tmX, &sm->full[s], I * BM + x * kBox, kb * BK);
+          tma_load_2d(a + x * kBoxBytes, tmX, &sm->full[s], I * BM + x * kBox, kb * BK);
         for (int x = 0; x < BN / kBox; ++x)
-          tma_load_2d(b + x * kBoxBytes, &tmX, &sm->full[s], J * BN + x * kBox, kb * BK);
+          tma_load_2d(b + x * kBoxBytes, tmX, &sm->full[s], J * BN + x * kBox, kb * BK);
         ++issued;
         if (++s == kStages) {
           s = 0;
@@ -152,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s = kStages - 1;
           ph ^= 1;
         }
-        mbar_wait(&sm->full[s], ph);
+        mbar_wait_drain(&sm->full[s], ph);
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -163,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;   // chunks issued by this CTA
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
+      const int nk = nk_of(t / per);
       for (int kb0 = 0; ok && kb0 < nk; kb0 += kChunkStages, ++g) {
         const int acc = g & 1;
         if (!mbar_wait(&sm->accempty[acc], ((g >> 1) & 1) ^ 1)) {
@@ -201,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // every MMA issued above completes before TMEM is released
     mma_commit(&sm->drain);
-    mbar_wait(&sm->drain, 0);
+    mbar_wait_drain(&sm->drain, 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may read
@@ -213,6 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !__any_sync(0xffffffffu, aborted(sm));
          t += gridDim.x) {
+      const int pb = t / per;
+      const int nk = nk_of(pb);
+      float* __restrict__ H = grp.H[pb];
       float sum[128];
 #pragma unroll
       for (int k = 0; k < 128; ++k) sum[k] = 0.f;
@@ -237,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       int I, J;
-      band.get(t, I, J);
+      band.get(t - pb * per, I, J);
       const int i = I * BM + r;
       const bool row_ok = i < d;
       float* hrow = H + (size_t)i * d;
@@ -293,25 +311,53 @@ bool hessian_tc_supported(const float* H, const void* X, nvfp4_dtype xt, int64_t
          (reinterpret_cast<uintptr_t>(X) & 15) == 0 && (reinterpret_cast<uintptr_t>(H) & 15) == 0;
 }
 
-nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
-                               cudaStream_t st) {
-  CUtensorMap tm;
-  const uint64_t dims[2] = {(uint64_t)d, (uint64_t)n_tok};
-  const uint64_t strides[1] = {(uint64_t)d * 2};
-  const uint32_t box[2] = {(uint32_t)kBox, (uint32_t)BK};
-  if (!encode_tmap_2d(&tm, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return NVFP4_ERR_CUDA;
+// H_p (+)= X_p^T X_p for P problems of dimension d (bf16 tokens, each
+// hessian_tc_supported), up to kHessGroup per launch.
+nvfp4_status launch_hessian_tc_group(int P, float* const* H, const void* const* X,
+                                     const int64_t* n_tok, int64_t d, int beta,
+                                     cudaStream_t st) {
+  // heaviest problems first
+  int order[kMaxGroup];
+  if (P < 1 || P > kMaxGroup) return NVFP4_ERR_INVALID_ARG;
+  for (int i = 0; i < P; ++i) order[i] = i;
+  for (int i = 1; i < P; ++i)   // stable insertion sort by decreasing n_tok
+    for (int j = i; j > 0 && n_tok[order[j]] > n_tok[order[j - 1]]; --j) {
+      const int t = order[j];
+      order[j] = order[j - 1];
+      order[j - 1] = t;
+    }
   BandTiles band{(int)((d + BM - 1) / BM), (int)((d + BN - 1) / BN)};
-  const int n_tiles = band.total();
+  const int per = band.total();
   const int sms = num_sms();
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-  hessian_tc_kernel<<<n_tiles < sms ? n_tiles : sms, kThreads, kSmem, st>>>(
-      tm, H, (int)d, (int)n_tok, beta, band);
-  NVFP4_LAUNCH_CHECK();
-  count_launches(1);
+  static thread_local HessGroup grp;   // 18 KB: kept off the stack
+  for (int c0 = 0; c0 < P; c0 += kHessGroup) {
+    const int n = (P - c0) < kHessGroup ? (P - c0) : kHessGroup;
+    grp.P = n;
+    for (int i = 0; i < n; ++i) {
+      const int q = order[c0 + i];
+      const uint64_t dims[2] = {(uint64_t)d, (uint64_t)n_tok[q]};
+      const uint64_t strides[1] = {(uint64_t)d * 2};
+      const uint32_t box[2] = {(uint32_t)kBox, (uint32_t)BK};
+      if (!encode_tmap_2d(&grp.map[i], X[q], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides,
+                          box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return NVFP4_ERR_CUDA;
+      grp.H[i] = H[q];
+      grp.n_tok[i] = (int)n_tok[q];
+    }
+    const int n_tiles = per * n;
+    hessian_tc_kernel<<<n_tiles < sms ? n_tiles : sms, kThreads, kSmem, st>>>(grp, (int)d,
+                                                                              beta, band);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(1);
+  }
   return NVFP4_OK;
+}
+
+nvfp4_status launch_hessian_tc(float* H, const void* X, int64_t n_tok, int64_t d, int beta,
+                               cudaStream_t st) {
+  return launch_hessian_tc_group(1, &H, &X, &n_tok, d, beta, st);
 }
 
 int hessian_tc_take_status(cudaStream_t st) {

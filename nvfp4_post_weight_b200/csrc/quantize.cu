@@ -38,9 +38,22 @@
 namespace nvfp4 {
 namespace {
 
-struct QuantHeader {   // workspace header (first 256 bytes)
+struct QuantHeader {   // one per problem of a group
   int status;
   unsigned amax_bits;  // max |W| as fp32 bits (non-negative floats order as uints)
+};
+
+// The caller's buffers of every problem of a group, written into the group
+// region once per call (init_group_kernel) and read by the kernels.
+struct QuantTable {
+  const void* W[kMaxGroup];
+  const float* U[kMaxGroup];
+  const uint8_t* dead[kMaxGroup];
+  uint8_t* codes[kMaxGroup];
+  uint8_t* scales[kMaxGroup];
+  float* sg[kMaxGroup];
+  double* err[kMaxGroup];
+  const float* amax_in[kMaxGroup];
 };
 
 // Columns per super-batch.  Inside a super-batch every lazy batch updates only
@@ -51,10 +64,15 @@ struct QuantHeader {   // workspace header (first 256 bytes)
 // super-batch (the plain lazy-batch scheme).
 int64_t super_width(int64_t d_in) { return d_in >= 2048 ? 8 * kLazyBatch : kLazyBatch; }
 
+// A group region of the quantize: the group header (its first int the status
+// word), the pointer table, P problem headers, then P copies each (uniform
+// strides) of the arrays below.
 struct QuantLayout {
+  int* gstatus;
+  QuantTable* tab;
   QuantHeader* hdr;
   int64_t S;       // super-batch width (K values per row of the four below)
-  double* Wt;      // d_out x d_in working copy
+  double* Wt;      // d_out x d_in working copy (stride d_out d_in)
   float* Dh;       // d_out x S: the super-batch's deltas, tf32-rounded part
   float* Dl;       // d_out x S: remainder (delta - Dh)
   float* Uh;       // d_in x S: the super-batch's rows of U transposed, tf32 part
@@ -62,32 +80,61 @@ struct QuantLayout {
   double* rowerr;  // d_out
 };
 
-QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in) {
+size_t quant_group_bytes(int64_t d_out, int64_t d_in, int P) {
+  const int64_t S = super_width(d_in);
+  return kWsHeader + align256(sizeof(QuantTable)) + align256(sizeof(QuantHeader) * P) +
+         align256(sizeof(double) * d_out * d_in * P) + 2 * align256(sizeof(float) * d_out * S * P) +
+         2 * align256(sizeof(float) * S * d_in * P) + align256(sizeof(double) * d_out * P);
+}
+
+QuantLayout quant_layout(void* ws, int64_t d_out, int64_t d_in, int P) {
   char* p = static_cast<char*>(ws);
   QuantLayout L;
-  L.hdr = reinterpret_cast<QuantHeader*>(p);
+  L.gstatus = reinterpret_cast<int*>(p);
   L.S = super_width(d_in);
   size_t off = kWsHeader;
+  L.tab = reinterpret_cast<QuantTable*>(p + off);
+  off += align256(sizeof(QuantTable));
+  L.hdr = reinterpret_cast<QuantHeader*>(p + off);
+  off += align256(sizeof(QuantHeader) * P);
   L.Wt = reinterpret_cast<double*>(p + off);
-  off += align256(sizeof(double) * d_out * d_in);
+  off += align256(sizeof(double) * d_out * d_in * P);
   L.Dh = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d_out * L.S);
+  off += align256(sizeof(float) * d_out * L.S * P);
   L.Dl = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * d_out * L.S);
+  off += align256(sizeof(float) * d_out * L.S * P);
   L.Uh = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * L.S * d_in);
+  off += align256(sizeof(float) * L.S * d_in * P);
   L.Ul = reinterpret_cast<float*>(p + off);
-  off += align256(sizeof(float) * L.S * d_in);
+  off += align256(sizeof(float) * L.S * d_in * P);
   L.rowerr = reinterpret_cast<double*>(p + off);
   return L;
 }
 
+// Clears the group's status word and problem headers and stores the pointer
+// table (one CTA).
+__global__ void init_group_kernel(QuantTable t, QuantTable* dst, int* gstatus, QuantHeader* hdr,
+                                  int P) {
+  if (threadIdx.x == 0) *gstatus = 0;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) hdr[i] = QuantHeader{0, 0u};
+  const uint64_t* src = reinterpret_cast<const uint64_t*>(&t);
+  uint64_t* out = reinterpret_cast<uint64_t*>(dst);
+  for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 8); i += blockDim.x) out[i] = src[i];
+}
+
 // a5 + a6: W~ = fp64(W) with dead columns zeroed, amax |W~|, non-finite check.
-// Eight consecutive elements per thread step (d_in is a multiple of 16).
+// Eight consecutive elements per thread step (d_in is a multiple of 16);
+// problem blockIdx.y of the group.
 template <typename T>
-__global__ void wprep_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_in,
-                             const uint8_t* __restrict__ dead, double* __restrict__ Wt,
-                             double* __restrict__ rowerr, QuantHeader* hdr) {
+__global__ void wprep_kernel(const QuantTable* __restrict__ tab, int64_t d_out, int64_t d_in,
+                             double* __restrict__ Wt, double* __restrict__ rowerr,
+                             QuantHeader* hdrs, int* gstatus) {
+  const int pb = blockIdx.y;
+  const T* __restrict__ W = static_cast<const T*>(tab->W[pb]);
+  const uint8_t* __restrict__ dead = tab->dead[pb];
+  QuantHeader* hdr = hdrs + pb;
+  Wt += pb * d_out * d_in;
+  rowerr += pb * d_out;
   const int64_t n8 = d_out * d_in / 8;
   float m = 0.f;
   bool bad = false;
@@ -127,7 +174,10 @@ __global__ void wprep_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_i
        r += (int64_t)gridDim.x * blockDim.x)
     rowerr[r] = 0.0;
   if (__any_sync(0xffffffffu, bad)) {
-    if ((threadIdx.x & 31) == 0) flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+    if ((threadIdx.x & 31) == 0) {
+      flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
+      flag_status(gstatus, NVFP4_ERR_NONFINITE);
+    }
   }
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) atomicMax(&hdr->amax_bits, __float_as_uint(m));
@@ -135,10 +185,14 @@ __global__ void wprep_kernel(const T* __restrict__ W, int64_t d_out, int64_t d_i
 
 // s_g = amax / (6 * 448) correctly rounded to fp32, 1 when W == 0; amax is
 // this call's own max |W~| unless the caller gives the layer's (row shards).
-__global__ void global_scale_kernel(QuantHeader* hdr, const float* __restrict__ amax_in,
-                                    float* __restrict__ sg) {
-  const float amax = amax_in ? *amax_in : __uint_as_float(hdr->amax_bits);
-  *sg = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+// One thread per problem of the group.
+__global__ void global_scale_kernel(const QuantTable* __restrict__ tab, const QuantHeader* hdrs,
+                                    int P) {
+  const int pb = threadIdx.x;
+  if (pb >= P) return;
+  const float* amax_in = tab->amax_in[pb];
+  const float amax = amax_in ? *amax_in : __uint_as_float(hdrs[pb].amax_bits);
+  *tab->sg[pb] = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
 }
 
 // max |W| (dead columns as 0) into *amax_bits (fp32 bits; non-negative floats
@@ -178,13 +232,17 @@ __device__ __forceinline__ int utile(int p, int q) { return p * (2 * kNb - 1 - p
 // Uh[j][k] + Ul[j][k] = U[cs + k][j] (tf32 part and remainder): the per-batch
 // updates read the super-batch's own columns, the super-batch update the
 // columns beyond it.  32 x 32 tiles transposed through shared memory.
-__global__ void __launch_bounds__(256) split_u_rows_kernel(const float* __restrict__ U,
+// Problem blockIdx.z of the group.
+__global__ void __launch_bounds__(256) split_u_rows_kernel(const QuantTable* __restrict__ tab,
                                                            int64_t d_in, int64_t cs, int nk,
                                                            int64_t j0, int64_t S,
                                                            float* __restrict__ Uh,
                                                            float* __restrict__ Ul) {
   __shared__ float t[32][33];
   pdl_wait();
+  const float* __restrict__ U = tab->U[blockIdx.z];
+  Uh += blockIdx.z * d_in * S;
+  Ul += blockIdx.z * d_in * S;
   const int64_t jb = j0 + (int64_t)blockIdx.x * 32;
   const int k0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -277,12 +335,10 @@ constexpr int kRuleSchurReplay = 0, kRuleAmax = 1, kRuleBlockMse = 2;
 // shared memory as 16x16 fp64 tiles, the rows' batch values next to it.
 template <int kRule>
 __global__ void __launch_bounds__(kReplayThreads)
-    schur_replay_batch_kernel(double* __restrict__ Wt, const float* __restrict__ U,
+    schur_replay_batch_kernel(const QuantTable* __restrict__ tab, double* __restrict__ Wt_all,
                               int64_t d_out, int64_t d_in, int c0, int bw,
-                              const float* __restrict__ sg_ptr, uint8_t* __restrict__ codes,
-                              uint8_t* __restrict__ scales, float* __restrict__ Dh,
-                              float* __restrict__ Dl, int64_t ldD,
-                              int kofs, double* __restrict__ rowerr) {
+                              float* __restrict__ Dh_all, float* __restrict__ Dl_all,
+                              int64_t ldD, int kofs, double* __restrict__ rowerr_all) {
   extern __shared__ double4 smem_d4[];
   double* Ut = reinterpret_cast<double*>(smem_d4);           // kUTiles x 256
   double* invd = Ut + kUTiles * 256;                         // 128
@@ -290,8 +346,31 @@ __global__ void __launch_bounds__(kReplayThreads)
   double* inv_tab = s_tab + 128;                             // 1 / s_tab[k]
   double* rows = inv_tab + 128;                              // kRowsPerCta x 128
   const int nblk = bw / kBlock;
+  // problem blockIdx.y of the group; its buffers are read (volatile: not kept
+  // in registers) from shared memory where they are used
+  const int pb = blockIdx.y;
+  __shared__ volatile struct {
+    double* Wt;
+    float* Dh;
+    float* Dl;
+    double* rowerr;
+    uint8_t* codes;
+    uint8_t* scales;
+    double six_sg;
+  } cp;
   pdl_wait();
   {
+    const float* __restrict__ U = tab->U[pb];
+    const float* sg_ptr = tab->sg[pb];
+    if (threadIdx.x == 0) {
+      cp.Wt = Wt_all + (int64_t)pb * d_out * d_in;
+      cp.Dh = Dh_all + (int64_t)pb * d_out * ldD;
+      cp.Dl = Dl_all + (int64_t)pb * d_out * ldD;
+      cp.rowerr = rowerr_all + (int64_t)pb * d_out;
+      cp.codes = tab->codes[pb];
+      cp.scales = tab->scales[pb];
+      cp.six_sg = 6.0 * (double)*sg_ptr;
+    }
     // Stage the batch's upper block-triangular part of U as 16 x 16 fp64
     // tiles: thread t < 256 handles element e = t of every tile and issues
     // all its loads before any store.  The other threads fill the candidate
@@ -323,8 +402,6 @@ __global__ void __launch_bounds__(kReplayThreads)
   }
   __syncthreads();
 
-  const double sg = (double)*sg_ptr;
-  const double six_sg = 6.0 * sg;
   const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
   const int warp = threadIdx.x >> 5;
   const int rloc = warp * 2 + half;
@@ -337,7 +414,10 @@ __global__ void __launch_bounds__(kReplayThreads)
     const int64_t r = rb + rloc;
     const bool valid = r < d_out;
     // stage the row's batch values
-    for (int c = hl; c < bw; c += 16) row[c] = valid ? Wt[r * d_in + c0 + c] : 0.0;
+    {
+      const double* __restrict__ Wt = cp.Wt;
+      for (int c = hl; c < bw; c += 16) row[c] = valid ? Wt[r * d_in + c0 + c] : 0.0;
+    }
     __syncwarp();
     double rowsum = 0.0;
 
@@ -349,7 +429,7 @@ __global__ void __launch_bounds__(kReplayThreads)
         v[i] = row[16 * b + i];
         amax = fmax(amax, fabs(v[i]));
       }
-      const int k0 = max(e4m3_code_rn(amax / six_sg), 1);
+      const int k0 = max(e4m3_code_rn(amax / cp.six_sg), 1);
       const int lo = min(max(k0 - 8, 1), 127 - kCand);
       const double s = s_tab[lo + hl];   // e4m3_value * s_g, exact: 4 + 24 significant bits
       const double inv_s = inv_tab[lo + hl];
@@ -415,9 +495,9 @@ __global__ void __launch_bounds__(kReplayThreads)
           hi_w |= __shfl_xor_sync(FULL, hi_w, o, 16);
         }
         if (valid && hl == 0) {
-          *reinterpret_cast<uint2*>(codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
+          *reinterpret_cast<uint2*>(cp.codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
               make_uint2(lo_w, hi_w);
-          scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
+          cp.scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
         }
       }
       // later columns of the batch absorb the chosen block's deltas
@@ -440,21 +520,27 @@ __global__ void __launch_bounds__(kReplayThreads)
       __syncwarp();
     }
     if (valid) {
+      float* __restrict__ Dh = cp.Dh;
+      float* __restrict__ Dl = cp.Dl;
       for (int c = hl; c < bw; c += 16) {
         const double x = row[c];
         const float h = sm100::tf32_rn((float)x);
         Dh[r * ldD + kofs + c] = h;
         Dl[r * ldD + kofs + c] = (float)(x - (double)h);
       }
-      if (hl == 0) rowerr[r] += rowsum;
+      if (hl == 0) cp.rowerr[r] += rowsum;
     }
     __syncwarp();
   }
 }
 
-__global__ void sum_rows_kernel(const double* __restrict__ rowerr, int64_t n,
-                                double* __restrict__ out) {
+// One CTA per problem of the group: err = sum of its rows' delta^2.
+__global__ void sum_rows_kernel(const QuantTable* __restrict__ tab,
+                                const double* __restrict__ rowerr_all, int64_t n) {
   __shared__ double part[32];
+  double* out = tab->err[blockIdx.x];
+  if (!out) return;
+  const double* rowerr = rowerr_all + (int64_t)blockIdx.x * n;
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += rowerr[i];
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -478,11 +564,14 @@ constexpr size_t kReplaySmem =
 
 }  // namespace
 
-size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) {
-  const int64_t S = super_width(d_in);
-  return kWsHeader + align256(sizeof(double) * d_out * d_in) +
-         2 * align256(sizeof(float) * d_out * S) + 2 * align256(sizeof(float) * S * d_in) +
-         align256(sizeof(double) * d_out);
+size_t quantize_ws_bytes(int64_t d_out, int64_t d_in) { return quant_group_bytes(d_out, d_in, 1); }
+size_t quantize_group_ws_bytes(int64_t d_out, int64_t d_in, int P) {
+  return quant_group_bytes(d_out, d_in, P);
+}
+
+const int* quantize_group_problem_status(const void* ws, int i) {
+  const char* p = static_cast<const char*>(ws) + kWsHeader + align256(sizeof(QuantTable));
+  return reinterpret_cast<const int*>(p + sizeof(QuantHeader) * i);
 }
 
 nvfp4_status launch_weight_amax(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
@@ -502,30 +591,65 @@ nvfp4_status launch_weight_amax(const void* W, nvfp4_dtype wt, int64_t d_out, in
   return NVFP4_OK;
 }
 
-nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
-                             const float* U, const uint8_t* dead, int rule, uint8_t* codes,
-                             uint8_t* scales, float* sg, double* err, void* ws,
-                             cudaStream_t st, const float* amax_in) {
-  QuantLayout L = quant_layout(ws, d_out, d_in);
-  NVFP4_CUDA_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(QuantHeader), st));
-  if (d_out == 0 || d_in == 0) {
-    global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, amax_in, sg);
+// GPTQ with Schur Replay for a group of P weight matrices of one shape (each
+// with its own U, outputs and global scale; every launch covers all P): ws is
+// the group region (quantize_group_ws_bytes(d_out, d_in, P) bytes).
+nvfp4_status launch_quantize_group(int P, const PtrArr<const void*>& W, nvfp4_dtype wt,
+                                   int64_t d_out, int64_t d_in, const PtrArr<const float*>& U,
+                                   const PtrArr<const uint8_t*>& dead, int rule,
+                                   const PtrArr<uint8_t*>& codes, const PtrArr<uint8_t*>& scales,
+                                   const PtrArr<float*>& sg, const PtrArr<double*>& err,
+                                   const PtrArr<const float*>& amax_in, void* ws,
+                                   cudaStream_t st) {
+  if (P < 1 || P > kMaxGroup) return NVFP4_ERR_INVALID_ARG;
+  QuantLayout L = quant_layout(ws, d_out, d_in, P);
+  {
+    QuantTable t;
+    for (int i = 0; i < P; ++i) {
+      t.W[i] = W.p[i];
+      t.U[i] = U.p[i];
+      t.dead[i] = dead.p[i];
+      t.codes[i] = codes.p[i];
+      t.scales[i] = scales.p[i];
+      t.sg[i] = sg.p[i];
+      t.err[i] = err.p[i];
+      t.amax_in[i] = amax_in.p[i];
+    }
+    for (int i = P; i < kMaxGroup; ++i) {
+      t.W[i] = t.U[i] = nullptr;
+      t.dead[i] = nullptr;
+      t.codes[i] = t.scales[i] = nullptr;
+      t.sg[i] = nullptr;
+      t.err[i] = nullptr;
+      t.amax_in[i] = nullptr;
+    }
+    init_group_kernel<<<1, 256, 0, st>>>(t, L.tab, L.gstatus, L.hdr, P);
     NVFP4_LAUNCH_CHECK();
     count_launches(1);
-    if (err) NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
+  }
+  if (d_out == 0 || d_in == 0) {
+    global_scale_kernel<<<1, kMaxGroup, 0, st>>>(L.tab, L.hdr, P);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(1);
+    for (int i = 0; i < P; ++i)
+      if (err.p[i]) NVFP4_CUDA_TRY(cudaMemsetAsync(err.p[i], 0, sizeof(double), st));
     return NVFP4_OK;
   }
-  const int g = grid_for(d_out * d_in / 8, 256);
-  if (wt == NVFP4_BF16)
-    wprep_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), d_out, d_in,
-                                              dead, L.Wt, L.rowerr, L.hdr);
-  else
-    wprep_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), d_out, d_in, dead,
-                                           L.Wt, L.rowerr, L.hdr);
-  NVFP4_LAUNCH_CHECK();
-  global_scale_kernel<<<1, 1, 0, st>>>(L.hdr, amax_in, sg);
-  NVFP4_LAUNCH_CHECK();
-  count_launches(2);
+  {
+    int g = grid_for(d_out * d_in / 8, 256) / P;
+    g = g < 1 ? 1 : g;
+    const dim3 wg((unsigned)g, (unsigned)P);
+    if (wt == NVFP4_BF16)
+      wprep_kernel<uint16_t><<<wg, 256, 0, st>>>(L.tab, d_out, d_in, L.Wt, L.rowerr, L.hdr,
+                                                 L.gstatus);
+    else
+      wprep_kernel<float><<<wg, 256, 0, st>>>(L.tab, d_out, d_in, L.Wt, L.rowerr, L.hdr,
+                                              L.gstatus);
+    NVFP4_LAUNCH_CHECK();
+    global_scale_kernel<<<1, kMaxGroup, 0, st>>>(L.tab, L.hdr, P);
+    NVFP4_LAUNCH_CHECK();
+    count_launches(2);
+  }
 
   auto* replay_kernel = rule == kRuleAmax       ? schur_replay_batch_kernel<kRuleAmax>
                        : rule == kRuleBlockMse ? schur_replay_batch_kernel<kRuleBlockMse>
@@ -533,10 +657,18 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kReplaySmem));
   UpdateMaps maps;
-  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in, L.S))
+  if (!make_update_maps(&maps, L.Dh, L.Dl, L.Uh, L.Ul, L.Wt, d_out, d_in, L.S, P))
     return NVFP4_ERR_CUDA;
-  const int64_t row_groups = (d_out + kRowsPerCta - 1) / kRowsPerCta;
-  const int rgrid = (int)(row_groups < kNumSMs ? row_groups : kNumSMs);
+  // CTAs per problem: one CTA per SM for a single problem; for a group,
+  // enough CTAs of about 8 row groups each that the tail of the last wave is
+  // a small part of the launch (each CTA stages its problem's U tiles once)
+  const int64_t rg = (d_out + kRowsPerCta - 1) / kRowsPerCta;
+  int64_t want = (rg * P + 7) / 8;
+  if (want < kNumSMs) want = kNumSMs;
+  int64_t per_problem = (want + P - 1) / P;
+  if (per_problem > rg) per_problem = rg;
+  const dim3 rgrid((unsigned)per_problem, (unsigned)P);
+  const int64_t sW = d_out * d_in, sD = d_out * L.S, sU = d_in * L.S;
   for (int64_t cs = 0; cs < d_in; cs += L.S) {
     const int64_t send = (d_in - cs) < L.S ? d_in : cs + L.S;
     const int64_t j0 = cs + kLazyBatch;   // first column any update of this super-batch touches
@@ -544,9 +676,10 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
       ProfileScope ps(kPhaseUpdate, st);
       const int nk = (int)(send - cs);
       NVFP4_CUDA_TRY(launch_chained(split_u_rows_kernel,
-                                    dim3((unsigned)((d_in - j0 + 31) / 32), (unsigned)((nk + 31) / 32)),
-                                    dim3(256), 0, st, U, (int64_t)d_in, cs, nk, j0, L.S,
-                                    L.Uh, L.Ul));
+                                    dim3((unsigned)((d_in - j0 + 31) / 32),
+                                         (unsigned)((nk + 31) / 32), (unsigned)P),
+                                    dim3(256), 0, st, (const QuantTable*)L.tab, (int64_t)d_in,
+                                    cs, nk, j0, L.S, L.Uh, L.Ul));
       count_launches(1);
     }
     for (int64_t c0 = cs; c0 < send; c0 += kLazyBatch) {
@@ -554,17 +687,17 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
       const int kofs = (int)(c0 - cs);
       {
         ProfileScope ps(kPhaseReplay, st);
-        NVFP4_CUDA_TRY(launch_chained(replay_kernel, dim3(rgrid), dim3(kReplayThreads),
-                                      kReplaySmem, st, L.Wt, U, d_out, d_in, (int)c0, bw, sg,
-                                      codes, scales, L.Dh, L.Dl, L.S, kofs, L.rowerr));
+        NVFP4_CUDA_TRY(launch_chained(replay_kernel, rgrid, dim3(kReplayThreads),
+                                      kReplaySmem, st, (const QuantTable*)L.tab, L.Wt, d_out,
+                                      d_in, (int)c0, bw, L.Dh, L.Dl, L.S, kofs, L.rowerr));
         count_launches(1);
       }
       const int64_t e = c0 + bw;
       if (e < send) {
         // the batch's deltas into the rest of the super-batch (W~ slab kept in L2)
         ProfileScope ps(kPhaseUpdate, st);
-        nvfp4_status s = launch_update_tc(maps, d_out, d_in, e, send, kofs, 1, true,
-                                          &L.hdr->status, st);
+        nvfp4_status s = launch_update_tc(maps, d_out, d_in, e, send, kofs, 1, true, P,
+                                          L.gstatus, st);
         if (s != NVFP4_OK) return s;
       }
     }
@@ -572,21 +705,41 @@ nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64
       // the whole super-batch's deltas into every later column, K = send - cs:
       // the 3xTF32 GEMM engine on the deltas' and U's hi/lo parts (128 x 128
       // tiles, 128-deep partials summed in fp32 registers), added to the fp64
-      // working copy in its epilogue
+      // working copy in its epilogue; one batch entry per problem
       ProfileScope ps(kPhaseUpdate, st);
       nvfp4_status s = gemm_nt_tc_split(
-          (int)d_out, (int)(d_in - send), (int)(send - cs), -1.f, L.Dh, L.Dl, L.S, 0,
-          L.Uh + send * L.S, L.Ul + send * L.S, L.S, 0, 0.f, nullptr, d_in, 0, nullptr, 0, 0, 1,
-          0, &L.hdr->status, st, L.Wt + send);
+          (int)d_out, (int)(d_in - send), (int)(send - cs), -1.f, L.Dh, L.Dl, L.S, sD,
+          L.Uh + send * L.S, L.Ul + send * L.S, L.S, sU, 0.f, nullptr, d_in, sW, nullptr, 0, 0,
+          P, 0, L.gstatus, st, L.Wt + send);
       if (s != NVFP4_OK) return s;
     }
   }
-  if (err) {
-    sum_rows_kernel<<<1, 1024, 0, st>>>(L.rowerr, d_out, err);
-    NVFP4_LAUNCH_CHECK();
-    count_launches(1);
-  }
+  sum_rows_kernel<<<P, 1024, 0, st>>>(L.tab, L.rowerr, d_out);
+  NVFP4_LAUNCH_CHECK();
+  count_launches(1);
   return NVFP4_OK;
+}
+
+// The single-problem quantize: a group of one whose region is ws.
+nvfp4_status launch_quantize(const void* W, nvfp4_dtype wt, int64_t d_out, int64_t d_in,
+                             const float* U, const uint8_t* dead, int rule, uint8_t* codes,
+                             uint8_t* scales, float* sg, double* err, void* ws,
+                             cudaStream_t st, const float* amax_in) {
+  PtrArr<const void*> w;
+  PtrArr<const float*> u, am;
+  PtrArr<const uint8_t*> dd;
+  PtrArr<uint8_t*> c, sc;
+  PtrArr<float*> g;
+  PtrArr<double*> e;
+  w.p[0] = W;
+  u.p[0] = U;
+  dd.p[0] = dead;
+  c.p[0] = codes;
+  sc.p[0] = scales;
+  g.p[0] = sg;
+  e.p[0] = err;
+  am.p[0] = amax_in;
+  return launch_quantize_group(1, w, wt, d_out, d_in, u, dd, rule, c, sc, g, e, am, ws, st);
 }
 
 }  // namespace nvfp4

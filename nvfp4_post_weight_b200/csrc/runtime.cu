@@ -52,6 +52,24 @@ void count_launches(int n) {
   g_phase_launches[p].fetch_add(n, std::memory_order_relaxed);
 }
 
+// Setters of every device module's pipeline-wait limit (sm100.cuh), one per
+// .cu file, registered while the library loads.
+using WaitSetter = cudaError_t (*)(unsigned long long);
+static std::vector<WaitSetter>& wait_setters() {
+  static std::vector<WaitSetter> v;   // constructed on first use: load order safe
+  return v;
+}
+static std::mutex& wait_setters_mu() {
+  static std::mutex m;
+  return m;
+}
+
+int register_wait_limit_setter(cudaError_t (*setter)(unsigned long long ns)) {
+  std::lock_guard<std::mutex> lk(wait_setters_mu());
+  wait_setters().push_back(setter);
+  return (int)wait_setters().size();
+}
+
 void add_phase_work(double work) {
   if (!g_profiling.load(std::memory_order_relaxed)) return;
   const int p = t_phase >= 0 ? t_phase : kPhaseOther;
@@ -144,6 +162,18 @@ using namespace nvfp4;
 extern "C" {
 
 long long nvfp4_launch_count(void) { return g_launches.load(); }
+
+nvfp4_status nvfp4_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long v = ns == 0 ? 4000000000ull : ns;
+  std::lock_guard<std::mutex> lk(wait_setters_mu());
+  for (WaitSetter f : wait_setters()) {
+    if (f(v) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+  }
+  return NVFP4_OK;
+}
 
 nvfp4_status nvfp4_profile_begin(void) {
   std::lock_guard<std::mutex> lk(g_mu);

@@ -1,19 +1,38 @@
 // sm_100a building blocks: mbarriers, TMA tile loads, TMEM allocation,
 // tcgen05 MMAs and TMEM loads, as thin inline-PTX wrappers.
 //
-// Every wait here is bounded: mbar_wait() gives up after kWaitNs of wall time
-// (read from %globaltimer) and returns false, so a kernel that loses a
+// Every wait here is bounded: mbar_wait() gives up after the pipeline-wait
+// limit of wall time (read from %globaltimer; 4 s unless the host set another
+// with nvfp4_set_wait_limit_ns) and returns false, so a kernel that loses a
 // partner never spins forever; the caller records NVFP4_ERR_TIMEOUT and
-// drains what it has in flight before it exits.
+// drains what it has in flight before it exits.  The drain's own waits
+// (mbar_wait_drain: copies and MMAs already issued) always keep the 4 s bound,
+// so that a short pipeline limit never lets a CTA exit with a copy or an MMA
+// still writing its shared or tensor memory.
 #pragma once
 
 #include <cuda.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace nvfp4 {
+
+// Registers a setter of one compiled module's pipeline-wait limit (runtime.cu);
+// nvfp4_set_wait_limit_ns calls every registered setter.
+int register_wait_limit_setter(cudaError_t (*setter)(unsigned long long ns));
+
 namespace sm100 {
 
 constexpr uint64_t kWaitNs = 4000000000ull;  // 4 s
+
+// The pipeline-wait limit of this module (every .cu file that includes this
+// header is its own device module, with its own copy, set through its own
+// registered setter).
+static __device__ unsigned long long g_wait_limit_ns = kWaitNs;
+static cudaError_t set_module_wait_limit(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
+static const int g_wait_limit_registered = register_wait_limit_setter(&set_module_wait_limit);
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -70,15 +89,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitNs) return false;
+    if (globaltimer() - t0 > limit) return false;
   }
+}
+
+// Waits for the phase with the given parity to complete; false once the
+// pipeline-wait limit has passed.  A limit of 1 ns or less means no waiting
+// at all: the wait fails unless one non-blocking probe finds the phase
+// complete (try_wait itself may block until completion, so it is not used
+// then).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long limit = __ldg(&g_wait_limit_ns);
+  if (limit <= 1) return mbar_test_wait(bar, parity);
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_for(bar, parity, limit);
+}
+
+// The same with the fixed 4 s bound: the waits of a drain (copies and MMAs
+// already issued, which complete on their own).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitNs);
 }
 
 // ---- TMA (no multicast) -------------------------------------------------------

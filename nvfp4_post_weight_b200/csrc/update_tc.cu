@@ -91,23 +91,24 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
-__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map,
-                                                 uint64_t* bar, int c0, int c1,
+// The operands are 3-D: (columns, rows, problem of the group).
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map,
+                                                 uint64_t* bar, int c0, int c1, int c2,
                                                  uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 
 // TMA tile store from shared memory (out-of-range parts are not written).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0,
-                                             int c1, uint64_t policy) {
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1, int c2, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint"
-      " [%0, {%2, %3}], [%1], %4;" ::"l"(map),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "l"(policy)
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4}], [%1], %5;" ::"l"(map),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
@@ -125,8 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmDl,
                      const __grid_constant__ CUtensorMap tmUh,
                      const __grid_constant__ CUtensorMap tmUl,
-                     const __grid_constant__ CUtensorMap tmW, int e, int n_rb, int n_tiles,
-                     int kofs, int nkb, int keep_w, int* status) {
+                     const __grid_constant__ CUtensorMap tmW, int e, int n_rb, int n_cols,
+                     int n_tiles, int kofs, int nkb, int keep_w, int* status) {
+  // tile t: problem t / (n_rb n_cols), then column tile, then row block (the
+  // CTAs running at once share a U tile in L2)
+  const int per = n_rb * n_cols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
-      const int rb = t % n_rb, tn = t / n_rb;
+      const int pb = t / per, rb = (t % per) % n_rb, tn = (t % per) / n_rb;
       for (int h = 0; h < 2; ++h, ++hw) {   // the W~ tile first: the long HBM latency
         const int wb = hw % kWBufs;
         if (!mbar_wait(&sm->w_empty[wb], ((hw / kWBufs) & 1) ^ 1)) {
@@ -183,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&sm->w_full[wb], kWHalf);
         for (int q = 0; q < 2; ++q)
-          tma_load_2d_hint(Wbuf + wb * kWHalf + q * kWBox, &tmW, &sm->w_full[wb],
-                           e + tn * UN + h * 32 + q * WBOX, rb * UM, w_pol);
+          tma_load_3d_hint(Wbuf + wb * kWHalf + q * kWBox, &tmW, &sm->w_full[wb],
+                           e + tn * UN + h * 32 + q * WBOX, rb * UM, pb, w_pol);
       }
       for (int kk = 0; ok && kk < nkb * kNChunks; ++kk) {
         const int kx = kofs + kk * KC;   // K coordinate of this chunk
@@ -195,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&sm->full[s], kStage);
         uint8_t* st = ring + s * kStage;
-        tma_load_2d_hint(st, &tmDh, &sm->full[s], kx, rb * UM, keep_pol);
-        tma_load_2d_hint(st + kAPart, &tmDl, &sm->full[s], kx, rb * UM, keep_pol);
-        tma_load_2d_hint(st + 2 * kAPart, &tmUh, &sm->full[s], kx, e + tn * UN, keep_pol);
-        tma_load_2d_hint(st + 2 * kAPart + kBPart, &tmUl, &sm->full[s], kx, e + tn * UN,
+        tma_load_3d_hint(st, &tmDh, &sm->full[s], kx, rb * UM, pb, keep_pol);
+        tma_load_3d_hint(st + kAPart, &tmDl, &sm->full[s], kx, rb * UM, pb, keep_pol);
+        tma_load_3d_hint(st + 2 * kAPart, &tmUh, &sm->full[s], kx, e + tn * UN, pb, keep_pol);
+        tma_load_3d_hint(st + 2 * kAPart + kBPart, &tmUl, &sm->full[s], kx, e + tn * UN, pb,
                          keep_pol);
         ++issued;
         if (++s == kStages) {
@@ -213,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           s = kStages - 1;
           ph ^= 1;
         }
-        mbar_wait(&sm->full[s], ph);
+        mbar_wait_drain(&sm->full[s], ph);
       }
       for (int k = 1; k <= kWBufs && k <= hw; ++k)
-        mbar_wait(&sm->w_full[(hw - k) % kWBufs], ((hw - k) / kWBufs) & 1);
+        mbar_wait_drain(&sm->w_full[(hw - k) % kWBufs], ((hw - k) / kWBufs) & 1);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&sm->acc_full[buf]);
     }
     mma_commit(&sm->drain);
-    mbar_wait(&sm->drain, 0);
+    mbar_wait_drain(&sm->drain, 0);
   } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t w_pol = keep_w ? policy_evict_last() : policy_evict_first();
     int hw = 0, prev = -1;
     for (int t = blockIdx.x; t < n_tiles && !aborted(sm); t += gridDim.x) {
-      const int rb = t % n_rb, tn = t / n_rb;
+      const int pb = t / per, rb = (t % per) % n_rb, tn = (t % per) / n_rb;
       bool ok = true;
       for (int h = 0; h < 2; ++h, ++hw) {
         const int wb = hw % kWBufs;
@@ -331,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         for (int qb = 0; qb < 2; ++qb)
-          tma_store_2d(&tmW, Wbuf + wb * kWHalf + qb * kWBox, e + tn * UN + h * 32 + qb * WBOX,
-                       rb * UM, w_pol);
+          tma_store_3d(&tmW, Wbuf + wb * kWHalf + qb * kWBox, e + tn * UN + h * 32 + qb * WBOX,
+                       rb * UM, pb, w_pol);
         bulk_commit();
         bulk_wait_read_all_but_one();   // the previous half's store has read its buffer
         if (prev >= 0) mbar_arrive(&sm->w_empty[prev]);
@@ -352,46 +356,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// 3-D map (columns, rows, problem): rows ld elements apart, problems
+// `stride` elements apart.
+static bool map3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
+                 int64_t cols, int64_t rows, int64_t ld, int P, int64_t stride, uint32_t box0,
+                 uint32_t box1) {
+  const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)P};
+  const uint64_t strides[2] = {(uint64_t)ld * esize, (uint64_t)stride * esize};
+  const uint32_t box[3] = {box0, box1, 1u};
+  return encode_tmap_nd(m, base, dt, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 bool make_update_maps(UpdateMaps* m, const float* Dh, const float* Dl, const float* Uh,
                       const float* Ul, const double* Wt, int64_t d_out, int64_t d_in,
-                      int64_t kcols) {
-  const uint64_t dw[2] = {(uint64_t)d_in, (uint64_t)d_out};
-  const uint64_t sw[1] = {(uint64_t)d_in * 8};
-  const uint32_t bw[2] = {(uint32_t)WBOX, (uint32_t)UM};
-  const uint64_t da[2] = {(uint64_t)kcols, (uint64_t)d_out};
-  const uint64_t sa[1] = {(uint64_t)kcols * 4};
-  const uint32_t ba[2] = {(uint32_t)KC, (uint32_t)UM};
-  const uint64_t db[2] = {(uint64_t)kcols, (uint64_t)d_in};
-  const uint64_t sb[1] = {(uint64_t)kcols * 4};
-  const uint32_t bb[2] = {(uint32_t)KC, (uint32_t)UN};
-  return encode_tmap_2d(&m->Dh, Dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, da, sa, ba,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tmap_2d(&m->Dl, Dl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, da, sa, ba,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tmap_2d(&m->Uh, Uh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, db, sb, bb,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tmap_2d(&m->Ul, Ul, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, db, sb, bb,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tmap_2d(&m->W, Wt, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, dw, sw, bw,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+                      int64_t kcols, int P) {
+  constexpr CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  return map3(&m->Dh, Dh, F32, 4, kcols, d_out, kcols, P, d_out * kcols, KC, UM) &&
+         map3(&m->Dl, Dl, F32, 4, kcols, d_out, kcols, P, d_out * kcols, KC, UM) &&
+         map3(&m->Uh, Uh, F32, 4, kcols, d_in, kcols, P, d_in * kcols, KC, UN) &&
+         map3(&m->Ul, Ul, F32, 4, kcols, d_in, kcols, P, d_in * kcols, KC, UN) &&
+         map3(&m->W, Wt, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, 8, d_in, d_out, d_in, P, d_out * d_in,
+              WBOX, UM);
 }
 
 nvfp4_status launch_update_tc(const UpdateMaps& m, int64_t d_out, int64_t d_in, int64_t e,
-                              int64_t e_end, int kofs, int nkb, bool keep_w, int* status,
+                              int64_t e_end, int kofs, int nkb, bool keep_w, int P, int* status,
                               cudaStream_t st) {
   const int n = (int)(e_end - e);
-  if (n <= 0 || d_out <= 0 || nkb <= 0) return NVFP4_OK;
+  if (n <= 0 || d_out <= 0 || nkb <= 0 || P < 1) return NVFP4_OK;
   // a tile may not reach past e_end unless e_end is the last column (the
   // tensor map clips there): tiles are UN columns wide
   if (e_end < d_in && n % UN != 0) return NVFP4_ERR_INVALID_ARG;
   const int n_rb = (int)((d_out + UM - 1) / UM);
-  const int n_tiles = n_rb * ((n + UN - 1) / UN);
+  const int n_cols = (n + UN - 1) / UN;
+  const int n_tiles = n_rb * n_cols * P;
   const int sms = num_sms();
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(update_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   NVFP4_CUDA_TRY(launch_chained(update_tc_kernel, dim3(n_tiles < sms ? n_tiles : sms),
                                 dim3(kThreads), kSmem, st, m.Dh, m.Dl, m.Uh, m.Ul, m.W, (int)e,
-                                n_rb, n_tiles, kofs, nkb, keep_w ? 1 : 0, status));
+                                n_rb, n_cols, n_tiles, kofs, nkb, keep_w ? 1 : 0, status));
   count_launches(1);
   return NVFP4_OK;
 }

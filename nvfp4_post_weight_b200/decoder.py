@@ -174,7 +174,7 @@ class MoELayerSolver:
         self.dims = [d for _ in range(E) for d in (hidden, inter)]
         self.H = [torch.empty((d, d), dtype=torch.float32, device=dev) for d in self.dims]
         self.U = [torch.empty((d, d), dtype=torch.float32, device=dev) for d in self.dims]
-        self.ws_prep = [_flat(B.nvfp4_prepare_workspace_size(d), dev) for d in self.dims]
+        self.ws_prep = _flat(B.nvfp4_prepare_batched_workspace_size(self.dims), dev)
         # weights: [gate_0, up_0, down_0, gate_1, ...]; factor index of each
         self.wshape = [s for _ in range(E) for s in ((inter, hidden), (inter, hidden),
                                                     (hidden, inter))]
@@ -184,19 +184,23 @@ class MoELayerSolver:
                        for o, i in self.wshape]
         self.s_g = [torch.empty(1, dtype=torch.float32, device=dev) for _ in self.wshape]
         self.err = [torch.empty(1, dtype=torch.float64, device=dev) for _ in self.wshape]
-        self.ws_quant = [_flat(B.nvfp4_quantize_workspace_size(o, i), dev) for o, i in self.wshape]
+        self.ws_quant = _flat(B.nvfp4_quantize_batched_workspace_size(self.wshape, self.params),
+                              dev)
         self.Q = [torch.empty(s, dtype=out_dtype, device=dev) for s in self.wshape]
 
     def step(self, Ws, Xs, stream=None):
         """Ws: [gate_0, up_0, down_0, ...] device weights; Xs: [X_in_0,
         X_mid_0, X_in_1, ...] device tokens."""
         B.nvfp4_hessian_accumulate_batched(self.H, Xs, 0, stream)
-        B.nvfp4_gptq_prepare_batched(self.H, self.damp, self.U, wss=self.ws_prep, stream=stream)
+        B.nvfp4_gptq_prepare_batched(self.H, self.damp, self.U, ws=self.ws_prep, stream=stream)
         B.nvfp4_gptq_schur_replay_quantize_batched(
             Ws, [self.U[f] for f in self.wfac], self.codes, self.scales, self.s_g, self.err,
-            wss=self.ws_quant, params=self.params, stream=stream)
+            ws=self.ws_quant, params=self.params, stream=stream)
         B.nvfp4_dequant_batched(self.codes, self.scales, self.s_g, self.Q, stream)
 
     def status(self, stream=None):
-        return ([B.nvfp4_workspace_status(w, stream) for w in self.ws_prep + self.ws_quant],
+        """(prepare status, quantize status, Hessian status): the first non-OK
+        status of any problem of each batched call."""
+        return (B.nvfp4_workspace_status(self.ws_prep, stream),
+                B.nvfp4_workspace_status(self.ws_quant, stream),
                 B.nvfp4_hessian_status(stream))

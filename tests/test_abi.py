@@ -77,9 +77,26 @@ def test_host_side_checks_need_no_device():
         null) == 3
     # batched forms: count < 0 or missing arrays are rejected on the host
     assert L.nvfp4_hessian_accumulate_batched(-1, null, null, 0, null, null, 0, null) == 1
-    assert L.nvfp4_gptq_prepare_batched(2, null, null, 0.01, null, null, null, null, null,
+    assert L.nvfp4_gptq_prepare_batched(2, null, null, 0.01, null, null, null, null, 0,
                                         null) == 1
     assert L.nvfp4_dequant_batched(0, null, null, null, null, null, null, 0, null) == 0
+    # a batched workspace that is too small -> NVFP4_ERR_WORKSPACE (nothing queued)
+    H = (ctypes.c_void_p * 2)(256, 512)
+    d = (ctypes.c_int64 * 2)(32, 32)
+    assert L.nvfp4_gptq_prepare_batched(2, H, d, 0.01, H, null, null, ctypes.c_void_p(256), 16,
+                                        null) == 3
+    # a problem with a bad shape decides the status before anything is queued
+    d_bad = (ctypes.c_int64 * 2)(32, 20)
+    assert L.nvfp4_gptq_prepare_batched(2, H, d_bad, 0.01, H, null, null, ctypes.c_void_p(256),
+                                        1 << 30, null) == 2
+    # an unsupported precision -> NVFP4_ERR_UNSUPPORTED
+    p = B.default_params()
+    assert p.precision == 0
+    p.precision = 1
+    assert L.nvfp4_gptq_schur_replay_quantize(
+        ctypes.c_void_p(256), 0, 4, 32, ctypes.c_void_p(256), ctypes.byref(p), null,
+        ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), null,
+        ctypes.c_void_p(256), 1 << 20, null) == 8
     assert L.nvfp4_status_string(5) == b"damped Hessian is not positive definite"
     assert L.nvfp4_prepare_workspace_size(-1) == 0
 
@@ -89,3 +106,40 @@ def test_workspace_sizes_grow_with_the_layer(d_out, d_in):
     q = B.nvfp4_quantize_workspace_size(d_out, d_in)
     assert q >= 8 * d_out * d_in
     assert B.nvfp4_prepare_workspace_size(d_in) >= 4 * d_in * d_in
+
+
+def test_batched_workspace_covers_the_problems():
+    """One workspace for a batched call: at least every problem's own scratch
+    arrays, at most the single-call workspaces plus the status header."""
+    ds = [4096, 1536, 4096, 4096, 1536]
+    b = B.nvfp4_prepare_batched_workspace_size(ds)
+    singles = sum(B.nvfp4_prepare_workspace_size(d) for d in ds)
+    assert sum(3 * 8 * d * d for d in ds) <= b <= singles + 256 * (len(ds) + 1)
+    shapes = [(1536, 4096), (1536, 4096), (4096, 1536)] * 3
+    q = B.nvfp4_quantize_batched_workspace_size(shapes)
+    qs = sum(B.nvfp4_quantize_workspace_size(*s) for s in shapes)
+    assert sum(8 * o * i for o, i in shapes) <= q <= qs + 256 * (len(shapes) + 1)
+    assert B.nvfp4_prepare_batched_workspace_size([]) > 0   # the status header
+
+
+def test_binding_rejects_bad_buffers_on_the_host():
+    """Tensor arguments are checked before the library is called: a buffer of
+    the wrong kind is NVFP4_ERR_INVALID_ARG, not a device access."""
+    import torch
+    codes = torch.zeros((4, 16), dtype=torch.uint8)
+    scales = torch.zeros((4, 2), dtype=torch.uint8)
+    sg = torch.zeros(1)
+    out = torch.zeros((4, 32))
+    with pytest.raises(B.Nvfp4Error) as e:
+        B.nvfp4_dequant(codes, scales, sg, out)     # host tensors
+    assert e.value.code == 1 and "CUDA" in str(e.value)
+    with pytest.raises(B.Nvfp4Error) as e:
+        B._need("call", torch.zeros((4, 8), dtype=torch.uint8), "codes", (4, 16), torch.uint8,
+                device=False)
+    assert e.value.code == 1 and "shape" in str(e.value)
+    with pytest.raises(B.Nvfp4Error):
+        B._need("call", torch.zeros((4, 16)).t(), "W", device=False)   # not contiguous
+    with pytest.raises(B.Nvfp4Error):
+        B._need("call", torch.zeros(3), "ws", dtype=torch.uint8, device=False)
+    with pytest.raises(B.Nvfp4Error):
+        B._need("call", torch.zeros(8, dtype=torch.uint8), "ws", numel_min=16, device=False)
