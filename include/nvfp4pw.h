@@ -163,6 +163,28 @@ nvfp4_status nvfp4_hessian_accumulate_host(float* H, const void* X_host, nvfp4_d
                                            int64_t chunk_tok, void* ws, size_t ws_bytes,
                                            nvfp4_stream_t stream);
 
+/* The same accumulation kept to fp64 accuracy, into an fp64 H: every product
+ * of two token values and their sums are exact to fp64 rounding (the tokens
+ * are transposed into fp64 channel rows, zero-padded, and the product runs on
+ * the int8-slice tensor-core GEMM of the factorisation: channel rows scaled
+ * by powers of two, cut into 7-bit slices, slice products exact in int32,
+ * levels summed in fp64; 8192 tokens per pass, passes added in fp64).
+ * For layers with fewer calibration tokens than channels: their damped
+ * Hessian's condition number (1e4 and more) amplifies the fp32 rounding of H
+ * (relative 6e-8) into factor errors that move decisions beyond near ties;
+ * with this H and nvfp4_gptq_prepare_f64 the factor is as accurate as for a
+ * well-conditioned layer.  About ten times the work of the bf16 tensor-core
+ * Hessian.
+ * H   : d x d fp64, full symmetric (both triangles written).
+ * ws  : nvfp4_hessian_f64_workspace_size(n_tok, d) bytes, 256-byte aligned;
+ *       a timed-out wait sets NVFP4_ERR_TIMEOUT in its status word
+ *       (nvfp4_workspace_status).
+ * Other arguments, layouts and errors as nvfp4_hessian_accumulate. */
+size_t nvfp4_hessian_f64_workspace_size(int64_t n_tok, int64_t d);
+nvfp4_status nvfp4_hessian_accumulate_f64(double* H, const void* X, nvfp4_dtype x_dtype,
+                                          int64_t n_tok, int64_t d, int beta, void* ws,
+                                          size_t ws_bytes, nvfp4_stream_t stream);
+
 /* Synchronizes `stream` and returns, then clears, the status word of the
  * Hessian calls on the current device: NVFP4_ERR_TIMEOUT if a tensor-core
  * Hessian kernel gave up on a bounded wait since the last query, NVFP4_OK
@@ -195,6 +217,13 @@ size_t nvfp4_prepare_workspace_size(int64_t d);
 nvfp4_status nvfp4_gptq_prepare(const float* H, int64_t d, float damp, float* U,
                                 uint8_t* dead, float* lambda_out, void* ws,
                                 size_t ws_bytes, nvfp4_stream_t stream);
+
+/* nvfp4_gptq_prepare from an fp64 H (as nvfp4_hessian_accumulate_f64 writes
+ * it): the same factorisation, which runs in fp64 throughout, reads H without
+ * rounding it to fp32 first.  Same workspace size and errors. */
+nvfp4_status nvfp4_gptq_prepare_f64(const double* H, int64_t d, float damp, float* U,
+                                    uint8_t* dead, float* lambda_out, void* ws,
+                                    size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* a5-a8  GPTQ with Schur Replay block-scale selection                       */

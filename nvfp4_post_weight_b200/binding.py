@@ -59,6 +59,9 @@ def lib():
             "nvfp4_hessian_accumulate_host": ([vp, vp, i32, i64, i64, i32, i64, vp, sz, vp],
                                               i32),
             "nvfp4_prepare_workspace_size": ([i64], sz),
+            "nvfp4_hessian_f64_workspace_size": ([i64, i64], sz),
+            "nvfp4_hessian_accumulate_f64": ([vp, vp, i32, i64, i64, i32, vp, sz, vp], i32),
+            "nvfp4_gptq_prepare_f64": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
             "nvfp4_gptq_schur_replay_quantize": (
@@ -238,6 +241,34 @@ def nvfp4_hessian_accumulate(H, X, beta=0, stream=None):
     _need(call, H, "H", (d, d), _F32)
     _check(call, lib().nvfp4_hessian_accumulate(
         _ptr(H), _ptr(X), _dtype_code(X), n_tok, d, int(beta), _stream(stream)))
+
+
+def nvfp4_hessian_f64_workspace_size(n_tok, d) -> int:
+    return int(lib().nvfp4_hessian_f64_workspace_size(int(n_tok), int(d)))
+
+
+def nvfp4_hessian_accumulate_f64(H, X, ws, beta=0, stream=None):
+    """H (fp64, d x d) (+)= X^T X to fp64 accuracy (int8-slice tensor cores)."""
+    call = "nvfp4_hessian_accumulate_f64"
+    n_tok, d = _matrix(call, X, "X", _IO_DTYPES)
+    _need(call, H, "H", (d, d), _F64)
+    nws = _ws_bytes(call, ws, nvfp4_hessian_f64_workspace_size(n_tok, d))
+    _check(call, lib().nvfp4_hessian_accumulate_f64(
+        _ptr(H), _ptr(X), _dtype_code(X), n_tok, d, int(beta), _ptr(ws), nws, _stream(stream)))
+
+
+def nvfp4_gptq_prepare_f64(H, damp, U, dead=None, lambda_out=None, ws=None, stream=None):
+    """nvfp4_gptq_prepare from an fp64 H."""
+    call = "nvfp4_gptq_prepare_f64"
+    d, _ = _matrix(call, H, "H", _F64)
+    _need(call, H, "H", (d, d))
+    _need(call, U, "U", (d, d), _F32)
+    _opt_need(call, dead, "dead", shape=(d,), dtype=_U8)
+    _opt_need(call, lambda_out, "lambda_out", shape=(1,), dtype=_F32)
+    nws = _ws_bytes(call, ws, nvfp4_prepare_workspace_size(d))
+    _check(call, lib().nvfp4_gptq_prepare_f64(
+        _ptr(H), d, float(damp), _ptr(U), _ptr(dead), _ptr(lambda_out), _ptr(ws), nws,
+        _stream(stream)))
 
 
 def nvfp4_hessian_status(stream=None) -> int:

@@ -117,7 +117,37 @@ nvfp4_status nvfp4_gptq_prepare(const float* H, int64_t d, float damp, float* U,
   if (!ws || !aligned256(ws) || ws_bytes < prepare_ws_bytes(d)) return NVFP4_ERR_WORKSPACE;
   if (d == 0) return NVFP4_OK;
   ProfileScope ps(kPhasePrepare, as_cuda(stream));
-  return launch_prepare(H, d, damp, U, dead, lambda_out, ws, as_cuda(stream));
+  return launch_prepare(H, false, d, damp, U, dead, lambda_out, ws, as_cuda(stream));
+}
+
+nvfp4_status nvfp4_gptq_prepare_f64(const double* H, int64_t d, float damp, float* U,
+                                    uint8_t* dead, float* lambda_out, void* ws, size_t ws_bytes,
+                                    nvfp4_stream_t stream) {
+  if (!H || !U || d < 0 || !(damp >= 0.f)) return NVFP4_ERR_INVALID_ARG;
+  if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (!ws || !aligned256(ws) || ws_bytes < prepare_ws_bytes(d)) return NVFP4_ERR_WORKSPACE;
+  if (d == 0) return NVFP4_OK;
+  ProfileScope ps(kPhasePrepare, as_cuda(stream));
+  return launch_prepare(H, true, d, damp, U, dead, lambda_out, ws, as_cuda(stream));
+}
+
+size_t nvfp4_hessian_f64_workspace_size(int64_t n_tok, int64_t d) {
+  if (n_tok < 0 || d < 0) return 0;
+  return hessian_f64_ws_bytes(n_tok, d);
+}
+
+nvfp4_status nvfp4_hessian_accumulate_f64(double* H, const void* X, nvfp4_dtype x_dtype,
+                                          int64_t n_tok, int64_t d, int beta, void* ws,
+                                          size_t ws_bytes, nvfp4_stream_t stream) {
+  if (!H || n_tok < 0 || d < 0 || (n_tok > 0 && !X)) return NVFP4_ERR_INVALID_ARG;
+  if (x_dtype != NVFP4_BF16 && x_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  if (beta != 0 && beta != 1) return NVFP4_ERR_INVALID_ARG;
+  if (d % 16 || d > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (d == 0) return NVFP4_OK;
+  if (!ws || !aligned256(ws) || ws_bytes < hessian_f64_ws_bytes(n_tok, d))
+    return NVFP4_ERR_WORKSPACE;
+  ProfileScope ps(kPhaseHessian, as_cuda(stream));
+  return launch_hessian_f64(H, X, x_dtype, n_tok, d, beta, ws, as_cuda(stream));
 }
 
 size_t nvfp4_quantize_workspace_size(int64_t d_out, int64_t d_in,

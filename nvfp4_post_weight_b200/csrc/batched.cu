@@ -177,7 +177,7 @@ nvfp4_status nvfp4_gptq_prepare_batched(int count, const float* const* H, const 
     const int P = (int)g.size();
     const int64_t dd = d[g[0]];
     if (dd > 0) {
-      PtrArr<const float*> h;
+      PtrArr<const void*> h;
       PtrArr<float*> u, lam;
       PtrArr<uint8_t*> de;
       for (int k = 0; k < P; ++k) {
@@ -186,7 +186,7 @@ nvfp4_status nvfp4_gptq_prepare_batched(int count, const float* const* H, const 
         de.p[k] = dead ? dead[g[k]] : nullptr;
         lam.p[k] = lambda_out ? lambda_out[g[k]] : nullptr;
       }
-      nvfp4_status s = launch_prepare_group(P, h, dd, damp, u, de, lam, region, st);
+      nvfp4_status s = launch_prepare_group(P, h, false, dd, damp, u, de, lam, region, st);
       if (s != NVFP4_OK) return s;
       PtrArr<const int*> ps_;
       PtrArr<int> idx;

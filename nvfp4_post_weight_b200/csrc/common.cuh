@@ -190,15 +190,20 @@ nvfp4_status launch_update_tc(const UpdateMaps& m, int64_t d_out, int64_t d_in, 
                               cudaStream_t st);
 nvfp4_status launch_hessian(float* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
                             int64_t d, int beta, cudaStream_t st);
-nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U,
+// H: fp32 (h64 false) or fp64 (h64 true), d x d.
+nvfp4_status launch_prepare(const void* H, bool h64, int64_t d, float damp, float* U,
                             uint8_t* dead, float* lambda_out, void* ws, cudaStream_t st);
+size_t hessian_f64_ws_bytes(int64_t n_tok, int64_t d);
+nvfp4_status launch_hessian_f64(double* H, const void* X, nvfp4_dtype xt, int64_t n_tok,
+                                int64_t d, int beta, void* ws, cudaStream_t st);
 size_t prepare_ws_bytes(int64_t d);
 // Groups of P problems of one shape (kernels launched once for all P); ws is
 // the group region of *_group_ws_bytes() bytes.
 size_t prepare_group_ws_bytes(int64_t d, int P);
-nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t d, float damp,
-                                  const PtrArr<float*>& U, const PtrArr<uint8_t*>& dead,
-                                  const PtrArr<float*>& lambda_out, void* ws, cudaStream_t st);
+nvfp4_status launch_prepare_group(int P, const PtrArr<const void*>& H, bool h64, int64_t d,
+                                  float damp, const PtrArr<float*>& U,
+                                  const PtrArr<uint8_t*>& dead, const PtrArr<float*>& lambda_out,
+                                  void* ws, cudaStream_t st);
 const int* prepare_group_problem_status(const void* ws, int i);
 size_t quantize_group_ws_bytes(int64_t d_out, int64_t d_in, int P);
 nvfp4_status launch_quantize_group(int P, const PtrArr<const void*>& W, nvfp4_dtype wt,

@@ -29,19 +29,20 @@ struct PrepHeader {   // one per problem of a group
 };
 
 // Sum of the diagonal (dead entries counted as 1), dead flags, lambda.  One
-// CTA per problem of the group (blockIdx.x).
-__global__ void diag_stats_kernel(PtrArr<const float*> Hs, int64_t d, float damp,
+// CTA per problem of the group (blockIdx.x).  H is fp32 or fp64 (T).
+template <typename T>
+__global__ void diag_stats_kernel(PtrArr<const void*> Hs, int64_t d, float damp,
                                   PtrArr<uint8_t*> deads, PtrArr<float*> lambdas,
                                   PrepHeader* hdrs, int* gstatus) {
   __shared__ double part[32];
   const int pb = blockIdx.x;
-  const float* __restrict__ H = Hs.p[pb];
+  const T* __restrict__ H = static_cast<const T*>(Hs.p[pb]);
   uint8_t* dead = deads.p[pb];
   PrepHeader* hdr = hdrs + pb;
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < d; i += blockDim.x) {
-    const float h = H[i * d + i];
-    const bool is_dead = (h == 0.f);
+    const T h = H[i * d + i];
+    const bool is_dead = (h == T(0));
     if (dead) dead[i] = is_dead ? 1 : 0;
     if (!isfinite(h)) {
       flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
@@ -69,40 +70,41 @@ __global__ void diag_stats_kernel(PtrArr<const float*> Hs, int64_t d, float damp
 // A[i][j] = H_d[d-1-i][d-1-j]; dead diagonal entries become 1 + lambda.
 // Also zero-fills X and Y (the inverse is built from its block diagonal
 // outward).  Rows blockIdx.y, + gridDim.y, ...; four consecutive columns per
-// thread (d is a multiple of 16); H read as float4 when it is 16-byte aligned.
-// Problem blockIdx.z of the group: its matrices sa elements after the
-// previous problem's.
-__global__ void reverse_damp_kernel(PtrArr<const float*> Hs, int64_t d, double* __restrict__ A,
+// thread (d is a multiple of 16); an fp32 H is read as float4 when it is
+// 16-byte aligned.  Problem blockIdx.z of the group: its matrices sa elements
+// after the previous problem's.  H is fp32 or fp64 (T).
+template <typename T>
+__global__ void reverse_damp_kernel(PtrArr<const void*> Hs, int64_t d, double* __restrict__ A,
                                     double* __restrict__ X, double* __restrict__ Y, int64_t sa,
                                     PrepHeader* hdrs, int* gstatus) {
   const int pb = blockIdx.z;
-  const float* __restrict__ H = Hs.p[pb];
+  const T* __restrict__ H = static_cast<const T*>(Hs.p[pb]);
   PrepHeader* hdr = hdrs + pb;
   A += pb * sa;
   X += pb * sa;
   Y += pb * sa;
-  const bool vec = (reinterpret_cast<uintptr_t>(H) & 15) == 0;
+  const bool vec = sizeof(T) == 4 && (reinterpret_cast<uintptr_t>(H) & 15) == 0;
   const double lam = hdr->lambda64;
   const int64_t j = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
   if (j >= d) return;
   for (int64_t i = blockIdx.y; i < d; i += gridDim.y) {
     // H row d-1-i, columns d-4-j .. d-1-j, i.e. hv[3..0] for A's columns j .. j+3
-    const float* hr = H + (d - 1 - i) * d + (d - 4 - j);
-    float hv[4];
+    const T* hr = H + (d - 1 - i) * d + (d - 4 - j);
+    double hv[4];
     if (vec) {
       const float4 h4 = *reinterpret_cast<const float4*>(hr);
       hv[0] = h4.w, hv[1] = h4.z, hv[2] = h4.y, hv[3] = h4.x;
     } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) hv[q] = hr[3 - q];
+      for (int q = 0; q < 4; ++q) hv[q] = (double)hr[3 - q];
     }
     double a[4];
     bool bad = false;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       bad |= !isfinite(hv[q]);
-      a[q] = (double)hv[q];
-      if (i == j + q) a[q] = (hv[q] == 0.f ? 1.0 : a[q]) + lam;
+      a[q] = hv[q];
+      if (i == j + q) a[q] = (hv[q] == 0.0 ? 1.0 : a[q]) + lam;
     }
     if (bad) {
       flag_status(&hdr->status, NVFP4_ERR_NONFINITE);
@@ -417,8 +419,13 @@ __global__ void __launch_bounds__(kPanelThreads)
     }
     return;
   }
-  // ---- L21 slice = A21 slice X11^T: 32 x 64 = 4 x 8 tiles, 4 per warp
-  {
+  // ---- L21 slice = A21 slice X11^T: 32 x 64 = 4 x 8 tiles, 4 per warp; then
+  // the CTA's further slices (gridDim.x - 1 slices apart), each loaded after
+  // the previous one is written (the diagonal block is factored once per CTA)
+  int64_t rs = r0;
+  int nrows = rows;
+  const int64_t slice_step = (int64_t)(gridDim.x - 1) * kSlice;
+  for (;;) {
     const int ti = warp & 3, tj0 = (warp >> 2) * 4;
     double acc[4][2] = {};
     for (int kk = 0; kk < NB; kk += 4) {
@@ -433,9 +440,48 @@ __global__ void __launch_bounds__(kPanelThreads)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int c = 8 * (tj0 + j) + fc2 + h;
-        if (i < rows && c < kb) A[(r0 + i) * d + k + c] = acc[j][h];
+        if (i < nrows && c < kb) A[(rs + i) * d + k + c] = acc[j][h];
       }
+    rs += slice_step;
+    if (rs >= d) break;
+    nrows = (int)((d - rs) < kSlice ? (d - rs) : kSlice);
+    constexpr int kPerS = kSlice * NB / kPanelThreads;   // 8
+    double a21[kPerS];
+#pragma unroll
+    for (int q = 0; q < kPerS; ++q) {
+      const int idx = tid + q * kPanelThreads, ii = idx / NB, l = idx % NB;
+      a21[q] = (ii < nrows && l < kb) ? A[(rs + ii) * d + k + l] : 0.0;
+    }
+    __syncthreads();   // every warp is done reading the previous slice
+#pragma unroll
+    for (int q = 0; q < kPerS; ++q) {
+      const int idx = tid + q * kPanelThreads, ii = idx / NB, l = idx % NB;
+      R[ii][l] = a21[q];
+    }
+    __syncthreads();
   }
+}
+
+// CTAs that solve a panel's slices, per problem of a group of P: every CTA
+// factors the diagonal block (a fixed chain of about kChainUnits time units)
+// before it solves its slices (about one unit each), and the panel kernel
+// runs one CTA per SM; so take the count of slice CTAs that minimises waves x
+// time per CTA.
+constexpr int kChainUnits = 8;
+int panel_slice_ctas(int64_t nslices, int P, int sms) {
+  if (nslices <= 0) return 0;
+  int best = 1;
+  double best_t = 1e300;
+  for (int64_t c = 1; c <= nslices; ++c) {
+    const int64_t waves = ((int64_t)P * (1 + c) + sms - 1) / sms;
+    const double t = (double)waves * (kChainUnits + (double)((nslices + c - 1) / c));
+    if (t < best_t) {
+      best_t = t;
+      best = (int)c;
+    }
+    if ((int64_t)P * (1 + c) > 64LL * sms) break;
+  }
+  return best;
 }
 
 // U[i][j] = X[d-1-i][d-1-j] for j >= i, 0 below the diagonal.  Rows
@@ -534,19 +580,29 @@ size_t prepare_group_ws_bytes(int64_t d, int P) { return prep_group_bytes(d, P);
 // whose factor meets a non-positive pivot or a non-finite H has its own
 // header's status set; the group word at the start of ws collects the first
 // status of any problem and the GEMMs' timeouts.
-nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t d, float damp,
-                                  const PtrArr<float*>& U, const PtrArr<uint8_t*>& dead,
-                                  const PtrArr<float*>& lambda_out, void* ws,
-                                  cudaStream_t st) {
+nvfp4_status launch_prepare_group(int P, const PtrArr<const void*>& H, bool h64, int64_t d,
+                                  float damp, const PtrArr<float*>& U,
+                                  const PtrArr<uint8_t*>& dead, const PtrArr<float*>& lambda_out,
+                                  void* ws, cudaStream_t st) {
   if (P < 1 || P > kMaxGroup) return NVFP4_ERR_INVALID_ARG;
   PrepLayout L = prep_layout(ws, d, P);
   NVFP4_CUDA_TRY(cudaMemsetAsync(ws, 0, kWsHeader + align256(sizeof(PrepHeader) * P), st));
-  diag_stats_kernel<<<P, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr, L.gstatus);
+  if (h64)
+    diag_stats_kernel<double><<<P, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr,
+                                                  L.gstatus);
+  else
+    diag_stats_kernel<float><<<P, 1024, 0, st>>>(H, d, damp, dead, lambda_out, L.hdr,
+                                                 L.gstatus);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   const dim3 rgrid((unsigned)((d / 4 + 255) / 256), (unsigned)(d < 65535 ? d : 65535),
                    (unsigned)P);
-  reverse_damp_kernel<<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.Y, L.sa, L.hdr, L.gstatus);
+  if (h64)
+    reverse_damp_kernel<double><<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.Y, L.sa, L.hdr,
+                                                       L.gstatus);
+  else
+    reverse_damp_kernel<float><<<rgrid, 256, 0, st>>>(H, d, L.A, L.X, L.Y, L.sa, L.hdr,
+                                                      L.gstatus);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
   const int64_t sa = L.sa;
@@ -581,7 +637,7 @@ nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t 
     for (int64_t k = k0; k < kend; k += NB) {
       const int kb = (int)((d - k) < NB ? (d - k) : NB);
       const int64_t m = d - k - kb;
-      const int grid = 1 + (int)((m + kSlice - 1) / kSlice);
+      const int grid = 1 + panel_slice_ctas((m + kSlice - 1) / kSlice, P, num_sms());
       {
         ProfileScope ps(kPhasePanel, st);
         // Cholesky and inverse of the kb x kb block, and the m x kb slice solve
@@ -665,17 +721,18 @@ nvfp4_status launch_prepare_group(int P, const PtrArr<const float*>& H, int64_t 
   return NVFP4_OK;
 }
 
-// The single-problem prepare: a group of one whose region is ws.
-nvfp4_status launch_prepare(const float* H, int64_t d, float damp, float* U, uint8_t* dead,
-                            float* lambda_out, void* ws, cudaStream_t st) {
-  PtrArr<const float*> h;
+// The single-problem prepare: a group of one whose region is ws; H is fp32,
+// or fp64 when h64.
+nvfp4_status launch_prepare(const void* H, bool h64, int64_t d, float damp, float* U,
+                            uint8_t* dead, float* lambda_out, void* ws, cudaStream_t st) {
+  PtrArr<const void*> h;
   PtrArr<float*> u, lam;
   PtrArr<uint8_t*> dd;
   h.p[0] = H;
   u.p[0] = U;
   dd.p[0] = dead;
   lam.p[0] = lambda_out;
-  return launch_prepare_group(1, h, d, damp, u, dd, lam, ws, st);
+  return launch_prepare_group(1, h, h64, d, damp, u, dd, lam, ws, st);
 }
 
 // Problem i's status word of a prepare group region.

@@ -346,31 +346,18 @@ __global__ void __launch_bounds__(kReplayThreads)
   double* inv_tab = s_tab + 128;                             // 1 / s_tab[k]
   double* rows = inv_tab + 128;                              // kRowsPerCta x 128
   const int nblk = bw / kBlock;
-  // problem blockIdx.y of the group; its buffers are read (volatile: not kept
-  // in registers) from shared memory where they are used
+  // problem blockIdx.y of the group: its buffers
   const int pb = blockIdx.y;
-  __shared__ volatile struct {
-    double* Wt;
-    float* Dh;
-    float* Dl;
-    double* rowerr;
-    uint8_t* codes;
-    uint8_t* scales;
-    double six_sg;
-  } cp;
+  const float* __restrict__ U = tab->U[pb];
+  const float* __restrict__ sg_ptr = tab->sg[pb];
+  double* __restrict__ Wt = Wt_all + (int64_t)pb * d_out * d_in;
+  float* __restrict__ Dh = Dh_all + (int64_t)pb * d_out * ldD;
+  float* __restrict__ Dl = Dl_all + (int64_t)pb * d_out * ldD;
+  double* __restrict__ rowerr = rowerr_all + (int64_t)pb * d_out;
+  uint8_t* __restrict__ codes = tab->codes[pb];
+  uint8_t* __restrict__ scales = tab->scales[pb];
   pdl_wait();
   {
-    const float* __restrict__ U = tab->U[pb];
-    const float* sg_ptr = tab->sg[pb];
-    if (threadIdx.x == 0) {
-      cp.Wt = Wt_all + (int64_t)pb * d_out * d_in;
-      cp.Dh = Dh_all + (int64_t)pb * d_out * ldD;
-      cp.Dl = Dl_all + (int64_t)pb * d_out * ldD;
-      cp.rowerr = rowerr_all + (int64_t)pb * d_out;
-      cp.codes = tab->codes[pb];
-      cp.scales = tab->scales[pb];
-      cp.six_sg = 6.0 * (double)*sg_ptr;
-    }
     // Stage the batch's upper block-triangular part of U as 16 x 16 fp64
     // tiles: thread t < 256 handles element e = t of every tile and issues
     // all its loads before any store.  The other threads fill the candidate
@@ -402,6 +389,8 @@ __global__ void __launch_bounds__(kReplayThreads)
   }
   __syncthreads();
 
+  const double sg = (double)*sg_ptr;
+  const double six_sg = 6.0 * sg;
   const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
   const int warp = threadIdx.x >> 5;
   const int rloc = warp * 2 + half;
@@ -414,10 +403,7 @@ __global__ void __launch_bounds__(kReplayThreads)
     const int64_t r = rb + rloc;
     const bool valid = r < d_out;
     // stage the row's batch values
-    {
-      const double* __restrict__ Wt = cp.Wt;
-      for (int c = hl; c < bw; c += 16) row[c] = valid ? Wt[r * d_in + c0 + c] : 0.0;
-    }
+    for (int c = hl; c < bw; c += 16) row[c] = valid ? Wt[r * d_in + c0 + c] : 0.0;
     __syncwarp();
     double rowsum = 0.0;
 
@@ -429,7 +415,7 @@ __global__ void __launch_bounds__(kReplayThreads)
         v[i] = row[16 * b + i];
         amax = fmax(amax, fabs(v[i]));
       }
-      const int k0 = max(e4m3_code_rn(amax / cp.six_sg), 1);
+      const int k0 = max(e4m3_code_rn(amax / six_sg), 1);
       const int lo = min(max(k0 - 8, 1), 127 - kCand);
       const double s = s_tab[lo + hl];   // e4m3_value * s_g, exact: 4 + 24 significant bits
       const double inv_s = inv_tab[lo + hl];
@@ -495,9 +481,9 @@ __global__ void __launch_bounds__(kReplayThreads)
           hi_w |= __shfl_xor_sync(FULL, hi_w, o, 16);
         }
         if (valid && hl == 0) {
-          *reinterpret_cast<uint2*>(cp.codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
+          *reinterpret_cast<uint2*>(codes + r * (d_in / 2) + (c0 + 16 * b) / 2) =
               make_uint2(lo_w, hi_w);
-          cp.scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
+          scales[r * (d_in / kBlock) + (c0 / kBlock) + b] = (uint8_t)(live ? lo + bl : 0);
         }
       }
       // later columns of the batch absorb the chosen block's deltas
@@ -520,15 +506,13 @@ __global__ void __launch_bounds__(kReplayThreads)
       __syncwarp();
     }
     if (valid) {
-      float* __restrict__ Dh = cp.Dh;
-      float* __restrict__ Dl = cp.Dl;
       for (int c = hl; c < bw; c += 16) {
         const double x = row[c];
         const float h = sm100::tf32_rn((float)x);
         Dh[r * ldD + kofs + c] = h;
         Dl[r * ldD + kofs + c] = (float)(x - (double)h);
       }
-      if (hl == 0) cp.rowerr[r] += rowsum;
+      if (hl == 0) rowerr[r] += rowsum;
     }
     __syncwarp();
   }

@@ -294,18 +294,28 @@ def test_quantize_empty_rows():
 
 def test_quantize_errors():
     U = torch.eye(32, dtype=torch.float32, device=DEV)
-    W = torch.zeros((4, 24), dtype=torch.float32, device=DEV)
     codes = torch.empty((4, 16), dtype=torch.uint8, device=DEV)
     scales = torch.empty((4, 2), dtype=torch.uint8, device=DEV)
     sg = torch.empty(1, dtype=torch.float32, device=DEV)
     ws = B.workspace(B.nvfp4_quantize_workspace_size(4, 32), DEV)
+    # d_in not a multiple of 16: the library's shape check (buffers sized to
+    # match, so the binding's own checks pass)
+    W24 = torch.zeros((4, 24), dtype=torch.float32, device=DEV)
+    U24 = torch.eye(24, dtype=torch.float32, device=DEV)
+    c24 = torch.empty((4, 12), dtype=torch.uint8, device=DEV)
+    s24 = torch.empty((4, 1), dtype=torch.uint8, device=DEV)
     with pytest.raises(B.Nvfp4Error) as e:
-        B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws)
+        B.nvfp4_gptq_schur_replay_quantize(W24, U24, c24, s24, sg, None, None, ws)
     assert e.value.code == 2
+    # a U of the wrong shape: rejected by the binding before any launch
     W = torch.zeros((4, 32), dtype=torch.float32, device=DEV)
+    n0 = B.lib().nvfp4_launch_count()
+    with pytest.raises(B.Nvfp4Error) as e:
+        B.nvfp4_gptq_schur_replay_quantize(W, U24, codes, scales, sg, None, None, ws)
+    assert e.value.code == 1 and B.lib().nvfp4_launch_count() == n0
     with pytest.raises(B.Nvfp4Error) as e:
         B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws[:64])
-    assert e.value.code == 3
+    assert e.value.code == 1   # the binding sees the short workspace first
     W[1, 3] = float("nan")
     B.nvfp4_gptq_schur_replay_quantize(W, U, codes, scales, sg, None, None, ws)
     assert B.nvfp4_workspace_status(ws) == 4
