@@ -51,10 +51,10 @@ __device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, vo
   }
 }
 
-// Problem blockIdx.y of a group.  Each thread step takes four consecutive
-// 16-weight blocks (32 code bytes + 4 scale bytes in, their 64 values out),
-// all loads issued before any use; a tail of fewer than four blocks goes one
-// block per thread.
+// Problem blockIdx.y of a group.  Each thread step takes four 16-weight blocks
+// one grid stride apart (so that every load instruction of a warp reads 32
+// consecutive blocks' bytes), all loads issued before any use; the output of
+// a warp's blocks is one contiguous run per store pair.
 template <bool kBF16>
 __global__ void dequant_kernel(PtrArr<const uint8_t*> codes_a, PtrArr<const uint8_t*> scales_a,
                                PtrArr<const float*> sg_a, PtrArr<void*> out_a,
@@ -65,21 +65,20 @@ __global__ void dequant_kernel(PtrArr<const uint8_t*> codes_a, PtrArr<const uint
   uint8_t* out = static_cast<uint8_t*>(out_a.p[pb]);
   constexpr int kOut = kBF16 ? 32 : 64;   // output bytes per block
   const float sg = *sg_a.p[pb];
-  const int64_t nq = nblocks / 4;
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
   const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t step = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t q = t0; q < nq; q += step) {
+  int64_t b = t0;
+  for (; b + 3 * T < nblocks; b += 4 * T) {
     uint2 c[4];
     uint32_t sc[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) c[k] = codes[4 * q + k];
+    for (int k = 0; k < 4; ++k) c[k] = codes[b + k * T];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) sc[k] = scales[4 * q + k];
+    for (int k = 0; k < 4; ++k) sc[k] = scales[b + k * T];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) dequant_block<kBF16>(c[k], sc[k], sg, out + (4 * q + k) * kOut);
+    for (int k = 0; k < 4; ++k) dequant_block<kBF16>(c[k], sc[k], sg, out + (b + k * T) * kOut);
   }
-  for (int64_t b = 4 * nq + t0; b < nblocks; b += step)
-    dequant_block<kBF16>(codes[b], scales[b], sg, out + b * kOut);
+  for (; b < nblocks; b += T) dequant_block<kBF16>(codes[b], scales[b], sg, out + b * kOut);
 }
 
 // Et = (W - Q)^T in fp32 (W bf16 or fp32) for a 64 x 64 tile of W: one

@@ -13,8 +13,9 @@ dequantizations.  Checked:
   delta^2 of all 384 weight matrices);
 * every expert's two Hessians against the oracle's fp64 ones (1e-4 relative
   Frobenius);
-* a spread of experts over the token range against the oracle's whole solve
-  from the same tokens, 128 sampled rows of each of gate, up and down, under
+* a spread of experts over the token range (every 8th and the last) against
+  the oracle's whole solve from the same tokens, 64 sampled rows of each of
+  gate, up and down, under
   the near-tie rule of parity.py, plus the rows' layer error within 1e-4:
   end to end (the library's Hessian and factor) where the Hessian has full
   rank (at least as many tokens as channels); where it has not, the solve is
@@ -40,8 +41,10 @@ from parity import classify, report, unpack_codes
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 N_EXPERTS = 128
-ORACLE_EXPERTS = (0, 6, 20, 50, 90, 127)   # 4096 ... 97 tokens
-ROWS = 128
+# every 8th expert and the last (4096 ... 97 tokens): 17 experts, their gate,
+# up and down projections each on 64 seeded rows
+ORACLE_EXPERTS = tuple(range(0, 128, 8)) + (127,)
+ROWS = 64
 
 
 def rel_frob(a, b):
