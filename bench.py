@@ -308,8 +308,9 @@ class DenseDecoder:
 
 class MoELayer:
     """128 experts (gate/up 4096 -> 1536, down 1536 -> 4096), Zipf(1.1)
-    routed token counts 64..4096 (65536 in total); every phase one batched
-    call over all experts."""
+    routed token counts 64..4096 (65536 in total); every phase (Hessian,
+    prepare, quantize, dequant, layer error) one batched call over all
+    experts."""
 
     def __init__(self, dev):
         import torch
@@ -338,7 +339,7 @@ class MoELayer:
         self.solver.step(self.Wd, self.Xd)
 
     def status_ok(self):
-        return self.solver.status() == (0, 0, 0)
+        return self.solver.status() == (0, 0, 0, 0)
 
 
 WORKLOADS = {

@@ -439,6 +439,19 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize_batched(
     float* const* global_scale, double* const* err_out, void* ws, size_t ws_bytes,
     nvfp4_stream_t stream);
 
+/* The layer error of every problem (H: each problem's undamped d_in x d_in
+ * Hessian; err_out: each problem's device fp64 scalar).  Scratch: one
+ * workspace of nvfp4_layer_error_batched_workspace_size() bytes; a timed-out
+ * wait of a launch is reported for every problem of that launch's shape. */
+size_t nvfp4_layer_error_batched_workspace_size(int count, const int64_t* d_out,
+                                                const int64_t* d_in);
+nvfp4_status nvfp4_layer_error_batched(int count, const void* const* W, nvfp4_dtype w_dtype,
+                                       const uint8_t* const* codes, const uint8_t* const* scales,
+                                       const float* const* global_scale, const float* const* H,
+                                       const int64_t* d_out, const int64_t* d_in,
+                                       double* const* err_out, void* ws, size_t ws_bytes,
+                                       nvfp4_stream_t stream);
+
 /* No workspace. */
 nvfp4_status nvfp4_dequant_batched(int count, const uint8_t* const* codes,
                                    const uint8_t* const* scales,

@@ -87,6 +87,9 @@ def lib():
                 [i32, vp, i32, vp, vp, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
                  sz, vp], i32),
             "nvfp4_dequant_batched": ([i32, vp, vp, vp, vp, vp, vp, i32, vp], i32),
+            "nvfp4_layer_error_batched_workspace_size": ([i32, vp, vp], sz),
+            "nvfp4_layer_error_batched": ([i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+                                          i32),
             "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
                                    vp], i32),
             "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
@@ -555,3 +558,33 @@ def nvfp4_set_wait_limit_ns(ns: int) -> None:
     """Pipeline-wait limit of the library's tensor-core kernels on the
     current device (0: the default 4 s); for testing the timeout path."""
     _check("nvfp4_set_wait_limit_ns", lib().nvfp4_set_wait_limit_ns(int(ns)))
+
+
+def nvfp4_layer_error_batched_workspace_size(shapes) -> int:
+    """shapes: [(d_out, d_in)] of the problems."""
+    return int(lib().nvfp4_layer_error_batched_workspace_size(
+        len(shapes), _i64s([s[0] for s in shapes]), _i64s([s[1] for s in shapes])))
+
+
+def nvfp4_layer_error_batched(Ws, codes, scales, global_scales, Hs, errs, ws, stream=None):
+    """Every problem's tr((W - Q) H (W - Q)^T) in one call (one workspace)."""
+    call = "nvfp4_layer_error_batched"
+    n = len(Ws)
+    _each(call, n, {"codes": codes, "scales": scales, "global_scale": global_scales, "H": Hs,
+                    "err_out": errs})
+    if len({w.dtype for w in Ws}) > 1:
+        raise Nvfp4Error(call, NVFP4_ERR_INVALID_ARG, "all W must share one dtype")
+    shapes = []
+    for i in range(n):
+        d_out, d_in = _matrix(call, Ws[i], f"W[{i}]", _IO_DTYPES)
+        _need(call, codes[i], f"codes[{i}]", (d_out, d_in // 2), _U8)
+        _need(call, scales[i], f"scales[{i}]", (d_out, d_in // 16), _U8)
+        _need(call, global_scales[i], f"global_scale[{i}]", (1,), _F32)
+        _need(call, Hs[i], f"H[{i}]", (d_in, d_in), _F32)
+        _need(call, errs[i], f"err_out[{i}]", (1,), _F64)
+        shapes.append((d_out, d_in))
+    nws = _ws_bytes(call, ws, nvfp4_layer_error_batched_workspace_size(shapes)) if n else 0
+    _check(call, lib().nvfp4_layer_error_batched(
+        n, _ptrs(Ws), _dtype_code(Ws[0]) if n else 0, _ptrs(codes), _ptrs(scales),
+        _ptrs(global_scales), _ptrs(Hs), _i64s([s[0] for s in shapes]),
+        _i64s([s[1] for s in shapes]), _ptrs(errs), _ptr(ws), nws, _stream(stream)))

@@ -59,6 +59,14 @@ size_t prepare_batched_bytes(int count, const int64_t* d) {
   return b;
 }
 
+size_t layer_error_batched_bytes(int count, const int64_t* d_out, const int64_t* d_in) {
+  size_t b = batch_header_bytes(count);
+  for (const auto& g :
+       group_by(count, [&](int i) { return std::make_pair(d_out[i], d_in[i]); }))
+    b += layer_error_group_ws_bytes(d_out[g[0]], d_in[g[0]], (int)g.size());
+  return b;
+}
+
 size_t quantize_batched_bytes(int count, const int64_t* d_out, const int64_t* d_in) {
   size_t b = batch_header_bytes(count);
   for (const auto& g :
@@ -269,6 +277,72 @@ nvfp4_status nvfp4_gptq_schur_replay_quantize_batched(
     s = gather_group_status(bh, reinterpret_cast<const int*>(region), ps_, idx, P, st);
     if (s != NVFP4_OK) return s;
     region += quantize_group_ws_bytes(o, n, P);
+  }
+  return NVFP4_OK;
+}
+
+size_t nvfp4_layer_error_batched_workspace_size(int count, const int64_t* d_out,
+                                                const int64_t* d_in) {
+  if (count < 0 || (count > 0 && (!d_out || !d_in))) return 0;
+  for (int i = 0; i < count; ++i)
+    if (d_out[i] < 0 || d_in[i] < 0) return 0;
+  return layer_error_batched_bytes(count, d_out, d_in);
+}
+
+nvfp4_status nvfp4_layer_error_batched(int count, const void* const* W, nvfp4_dtype w_dtype,
+                                       const uint8_t* const* codes, const uint8_t* const* scales,
+                                       const float* const* global_scale, const float* const* H,
+                                       const int64_t* d_out, const int64_t* d_in,
+                                       double* const* err_out, void* ws, size_t ws_bytes,
+                                       nvfp4_stream_t stream) {
+  if (count < 0 || (count > 0 && (!W || !codes || !scales || !global_scale || !H || !d_out ||
+                                  !d_in || !err_out)))
+    return NVFP4_ERR_INVALID_ARG;
+  if (w_dtype != NVFP4_BF16 && w_dtype != NVFP4_F32) return NVFP4_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (d_out[i] < 0 || d_in[i] < 0 || !err_out[i]) return NVFP4_ERR_INVALID_ARG;
+    if (d_out[i] > 0 && d_in[i] > 0 &&
+        (!W[i] || !codes[i] || !scales[i] || !global_scale[i] || !H[i]))
+      return NVFP4_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(codes[i]) & 7) return NVFP4_ERR_INVALID_ARG;
+    if (d_in[i] % 16 || d_in[i] > (1 << 17) || d_out[i] > (1 << 22)) return NVFP4_ERR_SHAPE;
+  }
+  if (count == 0) return NVFP4_OK;
+  if (!ws || !aligned256(ws) || ws_bytes < layer_error_batched_bytes(count, d_out, d_in))
+    return NVFP4_ERR_WORKSPACE;
+  cudaStream_t st = as_cuda(stream);
+  int* bh = static_cast<int*>(ws);
+  NVFP4_CUDA_TRY(cudaMemsetAsync(bh, 0, batch_header_bytes(count), st));
+  char* region = static_cast<char*>(ws) + batch_header_bytes(count);
+  for (const auto& g :
+       group_by(count, [&](int i) { return std::make_pair(d_out[i], d_in[i]); })) {
+    const int P = (int)g.size();
+    const int64_t o = d_out[g[0]], n = d_in[g[0]];
+    PtrArr<const void*> w;
+    PtrArr<const uint8_t*> c, sc;
+    PtrArr<const float*> gs, h;
+    PtrArr<double*> e;
+    for (int k = 0; k < P; ++k) {
+      const int i = g[k];
+      w.p[k] = W[i];
+      c.p[k] = codes[i];
+      sc.p[k] = scales[i];
+      gs.p[k] = global_scale[i];
+      h.p[k] = H[i];
+      e.p[k] = err_out[i];
+    }
+    nvfp4_status s =
+        launch_layer_error_group(P, w, w_dtype, c, sc, gs, h, o, n, e, region, st);
+    if (s != NVFP4_OK) return s;
+    PtrArr<const int*> ps_;
+    PtrArr<int> idx;
+    for (int k = 0; k < P; ++k) {
+      ps_.p[k] = reinterpret_cast<const int*>(region);   // one status word per group
+      idx.p[k] = g[k];
+    }
+    s = gather_group_status(bh, reinterpret_cast<const int*>(region), ps_, idx, P, st);
+    if (s != NVFP4_OK) return s;
+    region += layer_error_group_ws_bytes(o, n, P);
   }
   return NVFP4_OK;
 }

@@ -236,6 +236,13 @@ nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* co
                                 int64_t d_out, int64_t d_in, double* err, void* ws,
                                 cudaStream_t st);
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in);
+size_t layer_error_group_ws_bytes(int64_t d_out, int64_t d_in, int P);
+nvfp4_status launch_layer_error_group(int P, const PtrArr<const void*>& W, nvfp4_dtype wt,
+                                      const PtrArr<const uint8_t*>& codes,
+                                      const PtrArr<const uint8_t*>& scales,
+                                      const PtrArr<const float*>& sg,
+                                      const PtrArr<const float*>& H, int64_t d_out, int64_t d_in,
+                                      const PtrArr<double*>& err, void* ws, cudaStream_t st);
 
 // Programmatic dependent launch.  The kernels of a serial chain (panel ->
 // update -> panel, replay -> update -> replay) are launched with

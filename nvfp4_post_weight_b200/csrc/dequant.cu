@@ -86,14 +86,21 @@ __global__ void dequant_kernel(PtrArr<const uint8_t*> codes_a, PtrArr<const uint
 // rounding each, the tile is transposed through shared memory, and Et's rows
 // (ldE >= d_out apart) are written whole -- already split for the 3xTF32
 // Gram product: Eh = tf32(Et), El = Et - Eh (exact).
+// Problem blockIdx.z of a group: its Eh/El a whole ldE x d_in array after the
+// previous problem's.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    error_t_kernel(const T* __restrict__ W, const uint8_t* __restrict__ codes,
-                   const uint8_t* __restrict__ scales, const float* __restrict__ sg_ptr,
-                   int64_t d_out, int64_t d_in, float* __restrict__ Eh, float* __restrict__ El,
-                   int64_t ldE) {
+    error_t_kernel(PtrArr<const void*> Ws, PtrArr<const uint8_t*> codes_a,
+                   PtrArr<const uint8_t*> scales_a, PtrArr<const float*> sg_a, int64_t d_out,
+                   int64_t d_in, float* __restrict__ Eh, float* __restrict__ El, int64_t ldE) {
   __shared__ float tile[64][65];
-  const float sg = *sg_ptr;
+  const int pb = blockIdx.z;
+  const T* __restrict__ W = static_cast<const T*>(Ws.p[pb]);
+  const uint8_t* __restrict__ codes = codes_a.p[pb];
+  const uint8_t* __restrict__ scales = scales_a.p[pb];
+  Eh += (int64_t)pb * ldE * d_in;
+  El += (int64_t)pb * ldE * d_in;
+  const float sg = *sg_a.p[pb];
   const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
   const int t = threadIdx.x, row = t >> 2, blk = t & 3;
   const int64_t r = r0 + row, cb = c0 + 16 * blk;
@@ -136,9 +143,16 @@ __global__ void __launch_bounds__(256)
 // and step (d and the tile edges are multiples of 4), read as float4 when H
 // is 16-byte aligned (vec; G is workspace), so that several loads are in
 // flight per thread.
-__global__ void sym_tile_dot_kernel(const float* __restrict__ H, const float* __restrict__ G,
-                                    int64_t d, double* __restrict__ partial, int vec) {
+// Problem blockIdx.y of a group: its G a d x d array after the previous
+// problem's, its partial sums gridDim.x doubles after.
+__global__ void sym_tile_dot_kernel(PtrArr<const float*> Hs, const float* __restrict__ G,
+                                    int64_t d, double* __restrict__ partial) {
   __shared__ double part[32];
+  const int pb = blockIdx.y;
+  const float* __restrict__ H = Hs.p[pb];
+  G += (int64_t)pb * d * d;
+  partial += (int64_t)pb * gridDim.x;
+  const bool vec = (reinterpret_cast<uintptr_t>(H) & 15) == 0;
   double s = 0.0;
   for (int64_t i = blockIdx.x; i < d; i += gridDim.x) {
     const int64_t jdiag = (i / 128) * 128;
@@ -169,8 +183,11 @@ __global__ void sym_tile_dot_kernel(const float* __restrict__ H, const float* __
   }
 }
 
-// The partial sums added by one warp in a fixed order (deterministic).
-__global__ void sum_partials_kernel(const double* __restrict__ p, int n, double* __restrict__ out) {
+// The partial sums added by one warp in a fixed order (deterministic); one
+// CTA per problem of a group.
+__global__ void sum_partials_kernel(const double* __restrict__ p, int n, PtrArr<double*> outs) {
+  double* out = outs.p[blockIdx.x];
+  p += (int64_t)blockIdx.x * n;
   double s = 0.0;
   for (int i = threadIdx.x; i < n; i += 32) s += p[i];
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -253,52 +270,77 @@ nvfp4_status launch_scales_tiled(const uint8_t* scales, int64_t rows, int64_t d_
   return NVFP4_OK;
 }
 
+size_t layer_error_group_ws_bytes(int64_t d_out, int64_t d_in, int P) {
+  return kWsHeader + 2 * align256(sizeof(float) * et_ld(d_out) * d_in * P) +
+         align256(sizeof(float) * d_in * d_in * P) + align256(sizeof(double) * kDotBlocks * P);
+}
+
 size_t layer_error_ws_bytes(int64_t d_out, int64_t d_in) {
-  return kWsHeader + 2 * align256(sizeof(float) * et_ld(d_out) * d_in) +
-         align256(sizeof(float) * d_in * d_in) + align256(sizeof(double) * kDotBlocks);
+  return layer_error_group_ws_bytes(d_out, d_in, 1);
 }
 
 // tr(E H E^T) = <H, E^T E>: the Gram matrix G = E^T E is a symmetric
 // product, so only its tiles on or below the diagonal are formed (half the
-// flops of E H), on the tensor cores (3xTF32), then dotted with H.
-nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* codes,
-                                const uint8_t* scales, const float* sg, const float* H,
-                                int64_t d_out, int64_t d_in, double* err, void* ws,
-                                cudaStream_t st) {
+// flops of E H), on the tensor cores (3xTF32), then dotted with H.  For a
+// group of P problems of one shape every launch covers all P (the GEMM a batch
+// of P); ws is the group region, its first int the status word.
+nvfp4_status launch_layer_error_group(int P, const PtrArr<const void*>& W, nvfp4_dtype wt,
+                                      const PtrArr<const uint8_t*>& codes,
+                                      const PtrArr<const uint8_t*>& scales,
+                                      const PtrArr<const float*>& sg,
+                                      const PtrArr<const float*>& H, int64_t d_out, int64_t d_in,
+                                      const PtrArr<double*>& err, void* ws, cudaStream_t st) {
+  if (P < 1 || P > kMaxGroup) return NVFP4_ERR_INVALID_ARG;
+  int* status = static_cast<int*>(ws);
+  NVFP4_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  if (d_out == 0 || d_in == 0) {
+    for (int i = 0; i < P; ++i)
+      NVFP4_CUDA_TRY(cudaMemsetAsync(err.p[i], 0, sizeof(double), st));
+    return NVFP4_OK;
+  }
   char* p = static_cast<char*>(ws) + kWsHeader;
   const int64_t ldE = et_ld(d_out);
-  const size_t et_bytes = align256(sizeof(float) * ldE * d_in);
+  const size_t et_bytes = align256(sizeof(float) * ldE * d_in * P);
   float* Eh = reinterpret_cast<float*>(p);
   float* El = reinterpret_cast<float*>(p + et_bytes);
   float* G = reinterpret_cast<float*>(p + 2 * et_bytes);
   double* part =
-      reinterpret_cast<double*>(p + 2 * et_bytes + align256(sizeof(float) * d_in * d_in));
-  if (d_out == 0 || d_in == 0) {
-    NVFP4_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(double), st));
-    return NVFP4_OK;
-  }
-  const dim3 tgrid((unsigned)((d_in + 63) / 64), (unsigned)((d_out + 63) / 64));
+      reinterpret_cast<double*>(p + 2 * et_bytes + align256(sizeof(float) * d_in * d_in * P));
+  const dim3 tgrid((unsigned)((d_in + 63) / 64), (unsigned)((d_out + 63) / 64), (unsigned)P);
   if (wt == NVFP4_BF16)
-    error_t_kernel<uint16_t><<<tgrid, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes,
-                                                    scales, sg, d_out, d_in, Eh, El, ldE);
+    error_t_kernel<uint16_t><<<tgrid, 256, 0, st>>>(W, codes, scales, sg, d_out, d_in, Eh, El, ldE);
   else
-    error_t_kernel<float><<<tgrid, 256, 0, st>>>(static_cast<const float*>(W), codes, scales,
-                                                 sg, d_out, d_in, Eh, El, ldE);
+    error_t_kernel<float><<<tgrid, 256, 0, st>>>(W, codes, scales, sg, d_out, d_in, Eh, El, ldE);
   NVFP4_LAUNCH_CHECK();
   count_launches(1);
-  int* status = static_cast<int*>(ws);
-  NVFP4_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  // G = Et Et^T (d_in x d_in, K = d_out), lower tiles only
-  nvfp4_status s = gemm_nt_tc_split((int)d_in, (int)d_in, (int)d_out, 1.f, Eh, El, ldE, 0, Eh,
-                                    El, ldE, 0, 0.f, G, d_in, 0, nullptr, 0, 0, 1, 1, status, st);
+  // G = Et Et^T (d_in x d_in, K = d_out), lower tiles only, one batch entry per problem
+  nvfp4_status s = gemm_nt_tc_split((int)d_in, (int)d_in, (int)d_out, 1.f, Eh, El, ldE,
+                                    ldE * d_in, Eh, El, ldE, ldE * d_in, 0.f, G, d_in, d_in * d_in,
+                                    nullptr, 0, 0, P, 1, status, st);
   if (s != NVFP4_OK) return s;
-  sym_tile_dot_kernel<<<kDotBlocks, 256, 0, st>>>(H, G, d_in, part,
-                                                  (reinterpret_cast<uintptr_t>(H) & 15) == 0);
+  sym_tile_dot_kernel<<<dim3(kDotBlocks, P), 256, 0, st>>>(H, G, d_in, part);
   NVFP4_LAUNCH_CHECK();
-  sum_partials_kernel<<<1, 32, 0, st>>>(part, kDotBlocks, err);
+  sum_partials_kernel<<<P, 32, 0, st>>>(part, kDotBlocks, err);
   NVFP4_LAUNCH_CHECK();
   count_launches(2);
   return NVFP4_OK;
+}
+
+nvfp4_status launch_layer_error(const void* W, nvfp4_dtype wt, const uint8_t* codes,
+                                const uint8_t* scales, const float* sg, const float* H,
+                                int64_t d_out, int64_t d_in, double* err, void* ws,
+                                cudaStream_t st) {
+  PtrArr<const void*> w;
+  PtrArr<const uint8_t*> c, sc;
+  PtrArr<const float*> g, h;
+  PtrArr<double*> e;
+  w.p[0] = W;
+  c.p[0] = codes;
+  sc.p[0] = scales;
+  g.p[0] = sg;
+  h.p[0] = H;
+  e.p[0] = err;
+  return launch_layer_error_group(1, w, wt, c, sc, g, h, d_out, d_in, e, ws, st);
 }
 
 }  // namespace nvfp4

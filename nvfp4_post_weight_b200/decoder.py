@@ -187,8 +187,17 @@ class MoELayerSolver:
         self.ws_quant = _flat(B.nvfp4_quantize_batched_workspace_size(self.wshape, self.params),
                               dev)
         self.Q = [torch.empty(s, dtype=out_dtype, device=dev) for s in self.wshape]
+        self.layer_err = [torch.empty(1, dtype=torch.float64, device=dev) for _ in self.wshape]
+        # the layer-error scratch reuses the prepare workspace behind its status
+        # header (the per-problem status words the prepare leaves there stay
+        # readable): the calls run one after another on one stream, and the
+        # factors are done before the scratch is used
+        n_err = B.nvfp4_layer_error_batched_workspace_size(self.wshape)
+        hdr = (4 * (1 + len(self.dims)) + 255) // 256 * 256
+        self.ws_err = (self.ws_prep[hdr:hdr + n_err] if hdr + n_err <= self.ws_prep.numel()
+                       else _flat(n_err, dev))
 
-    def step(self, Ws, Xs, stream=None):
+    def step(self, Ws, Xs, stream=None, with_error=True):
         """Ws: [gate_0, up_0, down_0, ...] device weights; Xs: [X_in_0,
         X_mid_0, X_in_1, ...] device tokens."""
         B.nvfp4_hessian_accumulate_batched(self.H, Xs, 0, stream)
@@ -197,10 +206,15 @@ class MoELayerSolver:
             Ws, [self.U[f] for f in self.wfac], self.codes, self.scales, self.s_g, self.err,
             ws=self.ws_quant, params=self.params, stream=stream)
         B.nvfp4_dequant_batched(self.codes, self.scales, self.s_g, self.Q, stream)
+        if with_error:
+            B.nvfp4_layer_error_batched(Ws, self.codes, self.scales, self.s_g,
+                                        [self.H[f] for f in self.wfac], self.layer_err,
+                                        self.ws_err, stream)
 
     def status(self, stream=None):
-        """(prepare status, quantize status, Hessian status): the first non-OK
+        """(prepare, quantize, layer-error, Hessian status): the first non-OK
         status of any problem of each batched call."""
         return (B.nvfp4_workspace_status(self.ws_prep, stream),
                 B.nvfp4_workspace_status(self.ws_quant, stream),
+                B.nvfp4_workspace_status(self.ws_err, stream),
                 B.nvfp4_hessian_status(stream))

@@ -71,6 +71,8 @@ def moe():
     n0 = B.lib().nvfp4_launch_count()
     B.nvfp4_gptq_prepare_batched(Hs, 0.01, Us, ws=wsp)
     launches["prepare"] = B.lib().nvfp4_launch_count() - n0
+    status = [B.nvfp4_batched_workspace_status(wsp, len(Hs))]
+    del wsp   # (each call's workspace is freed before the next one is made)
     Ws = [ex[e][name].to(DEV) for e, name, _ in mats]
     Uq = [Us[hi] for _, _, hi in mats]
     codes = [torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=DEV) for w in Ws]
@@ -83,17 +85,25 @@ def moe():
     n0 = B.lib().nvfp4_launch_count()
     B.nvfp4_gptq_schur_replay_quantize_batched(Ws, Uq, codes, scales, sgs, errs, ws=wsq)
     launches["quantize"] = B.lib().nvfp4_launch_count() - n0
+    status.append(B.nvfp4_batched_workspace_status(wsq, len(Ws)))
+    del wsq
     Q = [torch.empty(w.shape, dtype=torch.float32, device=DEV) for w in Ws]
     n0 = B.lib().nvfp4_launch_count()
     B.nvfp4_dequant_batched(codes, scales, sgs, Q)
     launches["dequant"] = B.lib().nvfp4_launch_count() - n0
+    Hq = [Hs[hi] for _, _, hi in mats]
+    Ls = [torch.empty(1, dtype=torch.float64, device=DEV) for _ in Ws]
+    wse = B.workspace(B.nvfp4_layer_error_batched_workspace_size([tuple(w.shape) for w in Ws]),
+                      DEV)
+    n0 = B.lib().nvfp4_launch_count()
+    B.nvfp4_layer_error_batched(Ws, codes, scales, sgs, Hq, Ls, wse)
+    launches["layer_error"] = B.lib().nvfp4_launch_count() - n0
     torch.cuda.synchronize()
-    status = (B.nvfp4_batched_workspace_status(wsp, len(Hs)),
-              B.nvfp4_batched_workspace_status(wsq, len(Ws)))
-    del wsp, wsq
+    status.append(B.nvfp4_batched_workspace_status(wse, len(Ws)))
+    del wse
     return dict(counts=counts, ex=ex, Xs=Xs, Xd=Xd, Hs=Hs, Us=Us, mats=mats, Ws=Ws, Uq=Uq,
-                codes=codes, scales=scales, sgs=sgs, errs=errs, Q=Q, status=status,
-                hstatus=B.nvfp4_hessian_status(), launches=launches)
+                codes=codes, scales=scales, sgs=sgs, errs=errs, Q=Q, Hq=Hq, Ls=Ls,
+                status=status, hstatus=B.nvfp4_hessian_status(), launches=launches)
 
 
 def test_every_problem_status_ok(moe):
@@ -159,6 +169,33 @@ def test_batched_equals_single_calls_every_problem(moe):
         torch.cuda.synchronize()
         assert torch.equal(c, moe["codes"][i]) and torch.equal(s, moe["scales"][i]), i
         assert g.item() == moe["sgs"][i].item() and err.item() == moe["errs"][i].item(), i
+
+
+def test_batched_layer_error_equals_single_calls(moe):
+    assert moe["launches"]["layer_error"] <= 2 * 6   # a few launches per shape
+    for i, W in enumerate(moe["Ws"]):
+        d_out, d_in = W.shape
+        L = torch.empty(1, dtype=torch.float64, device=DEV)
+        ws = B.workspace(B.nvfp4_layer_error_workspace_size(d_out, d_in), DEV)
+        B.nvfp4_layer_error(W, moe["codes"][i], moe["scales"][i], moe["sgs"][i], moe["Hq"][i],
+                            L, ws)
+        torch.cuda.synchronize()
+        assert L.item() == moe["Ls"][i].item(), i
+
+
+@pytest.mark.parametrize("e", (0, 64, 127))
+def test_batched_layer_error_against_the_oracle(moe, e):
+    """The library's tr((W - Q) H (W - Q)^T) of expert e's three tensors
+    against the same quantity evaluated in fp64 on the host from the GPU's
+    codes and the oracle's fp64 Hessian."""
+    for i, (ee, name, hi) in enumerate(moe["mats"]):
+        if ee != e:
+            continue
+        W64 = moe["ex"][e][name].double().numpy()
+        H = O.hessian(moe["Xs"][hi].double().numpy())
+        Q = moe["Q"][i].cpu().numpy().astype(np.float64)
+        L = O.layer_error(W64, Q, H)
+        assert abs(moe["Ls"][i].item() - L) <= 1e-4 * L, (e, name)
 
 
 def test_every_expert_hessian(moe):
