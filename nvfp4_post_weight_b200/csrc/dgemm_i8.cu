@@ -126,6 +126,15 @@ __device__ __forceinline__ void tmem_ld64_raw(uint32_t taddr, uint32_t (&r)[64])
       : "memory");
 }
 
+// The int32 v as a double, exactly, on the integer and fp64 pipes instead of
+// the slower conversion unit: the double with high word 0x43300000 and low
+// word v + 2^31 (as unsigned) is 2^52 + 2^31 + v, an integer below 2^53, and
+// subtracting 2^52 + 2^31 leaves v without rounding.
+__device__ __forceinline__ double i32_to_f64(uint32_t v) {
+  return __dsub_rn(__hiloint2double(0x43300000, (int)(v ^ 0x80000000u)),
+                   4503601774854144.0 /* 2^52 + 2^31 */);
+}
+
 // D = s32, A and B signed 8-bit, both K-major, M = 128, N = n (a multiple of
 // 16 up to kMaxN).
 constexpr int kMaxN = 256;
@@ -422,7 +431,7 @@ __global__ void __launch_bounds__(kIThreads, 1)
           tmem_ld64_raw(tmem + ((uint32_t)(q * 32) << 16) + l * IN, v);
 #pragma unroll
           for (int j = 0; j < IN; ++j)
-            acc[j] = fma(acc[j], 0.0078125 /* 2^-7 */, (double)(int)v[j]);
+            acc[j] = fma(acc[j], 0.0078125 /* 2^-7 */, i32_to_f64(v[j]));
         }
       }
       tc_fence_before();

@@ -71,27 +71,36 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Output tiles.  A full result goes in groups of kGroupTiles tile rows: group
+// by group, inside a group column by column, so that the CTAs of a wave read
+// a few A row slabs and a short run of B slabs, which stay in L2 while they
+// walk K at the same pace (row-major order re-reads every B slab of a wide
+// output from DRAM once per wave).  A lower result (the Gram product) is
+// taken row-major over the tiles on or below the diagonal.
+constexpr int kGroupTiles = 16;
 struct TileSpace {
   int mt, nt, batch, lower;
-  __device__ int count() const {
-    const int per = lower ? mt * (mt + 1) / 2 : mt * nt;
-    return per * batch;
-  }
+  __device__ int per() const { return lower ? mt * (mt + 1) / 2 : mt * nt; }
+  __device__ int count() const { return per() * batch; }
   __device__ void get(int t, int& tm, int& tn, int& b) const {
-    const int per = lower ? mt * (mt + 1) / 2 : mt * nt;
-    b = t / per;
-    t -= b * per;
-    if (lower) {   // row-major over the lower triangle of tiles
+    const int p = per();
+    b = t / p;
+    t -= b * p;
+    if (lower) {
       tm = 0;
       while (t > tm) {
         t -= tm + 1;
         ++tm;
       }
       tn = t;
-    } else {
-      tm = t / nt;
-      tn = t - tm * nt;
+      return;
     }
+    constexpr int G = kGroupTiles;
+    const int g = t / (G * nt);
+    t -= g * G * nt;
+    const int r = (mt - g * G) < G ? (mt - g * G) : G;
+    tn = t / r;
+    tm = g * G + t % r;
   }
 };
 
@@ -398,8 +407,9 @@ nvfp4_status launch_gemm(int M, int N, int K, float alpha, const float* P, const
     mql = mq;
   }
   TileSpace ts{(M + GM - 1) / GM, (N + GN - 1) / GN, batch, lower};
-  const int per = lower ? ts.mt * (ts.mt + 1) / 2 : ts.mt * ts.nt;
-  const int n_tiles = per * batch;
+  const int64_t per = lower ? (int64_t)ts.mt * (ts.mt + 1) / 2 : (int64_t)ts.mt * ts.nt;
+  if (per * batch > (1ll << 30) || (lower && M != N)) return NVFP4_ERR_INVALID_ARG;
+  const int n_tiles = (int)(per * batch);
   const int sms = num_sms();
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_nt_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));

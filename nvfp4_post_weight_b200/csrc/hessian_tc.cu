@@ -19,10 +19,13 @@
 // Accuracy: the tensor cores' fp32 accumulation drops low bits (measured on
 // the 4096-token workload: a 1.3e-5 relative, one-sided error in H when all
 // tokens go into one accumulator).  So each accumulator only sums a chunk of
-// 128 tokens; the epilogue adds the chunk sums into fp32 registers with
-// round-to-nearest adds, then stores the upper part H[i][j>=i] and its mirror
-// H[j][i].  Only 128x256 tiles that touch the upper triangle are computed
-// (J >= I/2); each H element is produced by exactly one tile.
+// 256 tokens; the epilogue adds the chunk sums into fp32 registers with
+// round-to-nearest adds (H within 4e-7 relative Frobenius of the exact sum on
+// 16384 lognormal-scaled tokens; 128-token chunks give 2.4e-7 but drain the
+// accumulators twice as often and are 11% slower), then stores the upper
+// part H[i][j>=i] and its mirror H[j][i].  Only 128x256 tiles that touch the
+// upper triangle are computed (J >= I/2); each H element is produced by
+// exactly one tile.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -44,7 +47,7 @@ constexpr uint32_t kABytes = BM / kBox * kBoxBytes;
 constexpr uint32_t kBBytes = BN / kBox * kBoxBytes;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;  // 48 KB
 constexpr int kThreads = 320;
-constexpr int kChunkStages = 2;              // 128 tokens per accumulator
+constexpr int kChunkStages = 4;              // 256 tokens per accumulator
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr size_t kSmem = kStages * kStageBytes + 1024 + 256;
 
@@ -62,21 +65,53 @@ struct HessGroup {
   int P;
 };
 
-struct BandTiles {   // 128 x 256 tiles (I, J) with J >= I / 2, row-major
-  int nI, nJ;
-  __host__ __device__ int row_count(int I) const { return nJ - (I >> 1); }
-  __host__ __device__ int total() const {
-    int n = 0;
-    for (int I = 0; I < nI; ++I) n += row_count(I);
-    return n;
+// 128 x 256 tiles (I, J) with J >= I / 2 (I.e. I <= 2 J + 1), in groups of
+// kGroupRows tile rows: group by group, inside a group column by column, and
+// inside a column row by row.  The CTAs of one wave then hold a few A slabs
+// (the group's rows) and a short run of B slabs, which the L2 keeps for all
+// of them while they walk the tokens at the same pace; a row-major order
+// would read every B slab of the layer from DRAM once per wave.
+constexpr int kGroupRows = 16;
+constexpr int kMaxBandGroups = 64;          // d up to 64 * 16 * 128 = 131072
+struct BandTiles {
+  int nI, nJ, n_groups, per;
+  int start[kMaxBandGroups + 1];             // first tile of each group
+  // tile rows of group g present in column J
+  __host__ __device__ int col_rows(int g, int J) const {
+    const int i0 = g * kGroupRows;
+    int i1 = i0 + kGroupRows - 1;
+    if (i1 > nI - 1) i1 = nI - 1;
+    if (i1 > 2 * J + 1) i1 = 2 * J + 1;
+    return i1 >= i0 ? i1 - i0 + 1 : 0;
   }
-  __device__ void get(int t, int& I, int& J) const {
-    I = 0;
-    while (t >= row_count(I)) {
-      t -= row_count(I);
-      ++I;
+  __host__ bool init(int64_t d) {
+    nI = (int)((d + BM - 1) / BM);
+    nJ = (int)((d + BN - 1) / BN);
+    n_groups = (nI + kGroupRows - 1) / kGroupRows;
+    if (n_groups > kMaxBandGroups) return false;
+    per = 0;
+    for (int g = 0; g < n_groups; ++g) {
+      start[g] = per;
+      for (int J = (g * kGroupRows) >> 1; J < nJ; ++J) per += col_rows(g, J);
     }
-    J = (I >> 1) + t;
+    start[n_groups] = per;
+    return true;
+  }
+  // the first columns of a group are short (rows I <= 2 J + 1); the rest
+  // hold all of the group's rows
+  __device__ void get(int t, int& I, int& J) const {
+    int g = 0;
+    while (t >= start[g + 1]) ++g;
+    t -= start[g];
+    J = (g * kGroupRows) >> 1;
+    const int full = col_rows(g, nJ - 1);
+    int c = col_rows(g, J);
+    while (c < full && t >= c) {
+      t -= c;
+      c = col_rows(g, ++J);
+    }
+    J += t / full;
+    I = g * kGroupRows + t % full;
   }
 };
 
@@ -106,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(tiles + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = band.total();
+  const int per = band.per;
   const int n_tiles = per * grp.P;
   auto nk_of = [&](int pb) { return (grp.n_tok[pb] + BK - 1) / BK; };
 
@@ -326,8 +361,9 @@ nvfp4_status launch_hessian_tc_group(int P, float* const* H, const void* const* 
       order[j] = order[j - 1];
       order[j - 1] = t;
     }
-  BandTiles band{(int)((d + BM - 1) / BM), (int)((d + BN - 1) / BN)};
-  const int per = band.total();
+  BandTiles band;
+  if (!band.init(d)) return NVFP4_ERR_SHAPE;
+  const int per = band.per;
   const int sms = num_sms();
   NVFP4_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
