@@ -406,12 +406,15 @@ def scales_to_tiled(scales):
 def round_to_bf16(x):
     """Round fp64 values to bf16 (RN-even, one rounding straight from fp64),
     returned as float32 arrays holding the bf16 values.  Going through fp32
-    first would round twice."""
+    first would round twice.  bf16 has fp32's exponent range: 8 significant
+    bits in the binades from 2^-126 up, below that the fixed spacing 2^-133 of
+    its subnormals; values from (2 - 2^-8) 2^127 up round to infinity."""
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)                      # x = m * 2**e, 0.5 <= |m| < 1
-    scaled = np.ldexp(m, 8)                 # 8 significant bits kept
-    r = np.rint(scaled)                     # ties to even
-    return np.ldexp(r, e - 8).astype(np.float32)
+    e = np.maximum(e, -125)                 # spacing 2^(e - 8) >= 2^-133
+    r = np.rint(np.ldexp(x, 8 - e))         # ties to even
+    with np.errstate(over="ignore"):
+        return np.ldexp(r, e - 8).astype(np.float32)
 
 
 def layer_error(W, Q, H):

@@ -332,6 +332,47 @@ def test_round_to_bf16_matches_ml_dtypes_on_fp32_values():
     x = (rng.standard_normal(10000) * 10 ** rng.uniform(-5, 3, 10000)).astype(np.float32)
     np.testing.assert_array_equal(O.round_to_bf16(x.astype(np.float64)),
                                   x.astype(md.bfloat16).astype(np.float32))
+    # the ends of the range: bf16 subnormals (below 2^-126) and overflow
+    lo = (rng.standard_normal(10000) * 10 ** rng.uniform(-44.5, -36, 10000)).astype(np.float32)
+    hi = (rng.standard_normal(10000) * 10 ** rng.uniform(37, 38.5, 10000)).astype(np.float32)
+    for v in (lo, hi):
+        with np.errstate(over="ignore"):
+            want = v.astype(md.bfloat16).astype(np.float32)
+        np.testing.assert_array_equal(O.round_to_bf16(v.astype(np.float64)), want)
+
+
+def test_round_to_bf16_is_the_nearest_bf16_value():
+    """Brute force over the whole bf16 grid: every finite bf16 value (all
+    65536 bit patterns, the subnormals included), the nearest one to x, ties
+    to the even bit pattern, overflow past the largest finite value plus half
+    its spacing to infinity.  Inputs: exact products with up to 30
+    significant bits (the dequant's e2m1 * e4m3 * s_g) across the range."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        vals = (bits << 16).view(np.float32).astype(np.float64)
+    fin = np.isfinite(vals) & (bits < 0x8000)           # non-negative finite values
+    grid, gbits = vals[fin], bits[fin]
+    order = np.argsort(grid, kind="stable")
+    grid, gbits = grid[order], gbits[order]
+    big = (2.0 - 2.0 ** -7) * 2.0 ** 127
+    rng = np.random.default_rng(41)
+    mant = rng.integers(1 << 29, 1 << 30, 3000).astype(np.float64)
+    ex = rng.integers(-165, 100, 3000)
+    xs = np.concatenate([np.ldexp(mant, ex - 29), np.ldexp(mant[:200], rng.integers(127, 130, 200) - 29),
+                         grid[:40] + np.ldexp(1.0, -134), [0.0, big, big * (1 + 2.0 ** -9)]])
+    got = O.round_to_bf16(xs)
+    for x, g in zip(xs, got):
+        i = np.searchsorted(grid, x)
+        cands = [j for j in (i - 1, i) if 0 <= j < len(grid)]
+        dist = [abs(grid[j] - x) for j in cands]
+        best = min(dist)
+        near = [j for j, dd in zip(cands, dist) if dd == best]
+        j = near[0] if len(near) == 1 else min(near, key=lambda k: (int(gbits[k]) & 1, k))
+        want = grid[j]
+        if x >= big + 2.0 ** 119:   # half the top spacing past the largest value
+            want = np.inf
+        assert g == np.float32(want), (x, g, want)
+        assert O.round_to_bf16(-x) == -g
 
 
 def test_all_zero_row_and_block():
