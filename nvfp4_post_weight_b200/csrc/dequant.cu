@@ -19,15 +19,32 @@ namespace {
 
 __device__ __forceinline__ uint16_t bf16_of_product(float cs, float sg) {
   float hi = __fmul_rz(cs, sg);
-  const float lo = fmaf(cs, sg, -hi);  // exact residual
+  const float lo = fmaf(cs, sg, -hi);  // exact residual (normal products)
   if (lo != 0.f) hi = __uint_as_float(__float_as_uint(hi) | 1u);
   return __bfloat16_as_ushort(__float2bfloat16_rn(hi));
 }
 
+// bf16 bits of p, an exact product (cs * sg: 6 + 24 significant bits, exact in
+// fp64), rounded once to nearest-even on bf16's grid: spacing 2^(e - 7) in
+// the binade 2^e, 2^-133 below the normal range, overflow to infinity.  Used
+// for products outside the normal fp32 range, where the fp32 residual of
+// bf16_of_product is no longer exact.
+__device__ __forceinline__ uint16_t bf16_of_exact(double p) {
+  const double a = fabs(p);
+  const uint32_t sign = (uint32_t)(__double2hiint(p) >> 31) << 15;
+  if (a == 0.0) return (uint16_t)sign;
+  int e = ilogb(a);
+  e = e < -126 ? -126 : e;
+  const double M = scalbn(1.5, e + 45);          // unit in the last place 2^(e - 7)
+  const float r = (float)__dsub_rn(__dadd_rn(a, M), M);   // on bf16's grid: exact (or inf)
+  return (uint16_t)((__float_as_uint(r) >> 16) | sign);
+}
+
 // The 16 dequantized values of one block: code bytes c (low nibble first),
-// scale code sc, written to o (16 bf16 = 32 bytes, or 16 fp32 = 64 bytes).
+// scale code sc, written to o (16 bf16 = 32 bytes, or 16 fp32 = 64 bytes),
+// one product and one rounding per element.
 template <bool kBF16>
-__device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, void* o) {
+__device__ __forceinline__ void dequant_block_exact(uint2 c, uint32_t sc, float sg, void* o) {
   const float sb = (float)e4m3_value(sc & 0x7F);
   const uint64_t p = ((uint64_t)c.y << 32) | c.x;
   float cs[16];
@@ -37,8 +54,8 @@ __device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, vo
     uint32_t h[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      h[j] = (uint32_t)bf16_of_product(cs[2 * j], sg) |
-             ((uint32_t)bf16_of_product(cs[2 * j + 1], sg) << 16);
+      h[j] = (uint32_t)bf16_of_exact((double)cs[2 * j] * (double)sg) |
+             ((uint32_t)bf16_of_exact((double)cs[2 * j + 1] * (double)sg) << 16);
     uint4* q = reinterpret_cast<uint4*>(o);
     q[0] = make_uint4(h[0], h[1], h[2], h[3]);
     q[1] = make_uint4(h[4], h[5], h[6], h[7]);
@@ -49,6 +66,65 @@ __device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, vo
       q[k] = make_float4(cs[4 * k] * sg, cs[4 * k + 1] * sg, cs[4 * k + 2] * sg,
                          cs[4 * k + 3] * sg);
   }
+}
+
+// bf16 output by table.  An E2M1 magnitude is 1 or 3 times a power of two
+// (0.5, 1, 2, 4 and 1.5, 3, 6), so every element of a block is
+// 2^k bf16(sb sg) or 2^k bf16(3 sb sg): the block takes two correctly rounded
+// products, and scaling a normal bf16 by 2^k is exact (an add to its exponent
+// field).  The eight magnitudes' bf16 bits form a table whose low and high
+// bytes sit in two register pairs; one byte permutation per register pair
+// looks up four elements at once (selector = the 3-bit magnitudes), a third
+// interleaves low and high bytes, and the sign bits come from the code bits
+// by a fourth.  Blocks whose products come near either end of the normal
+// range take the exact path; a scale code of 0 gives a table of zeros.
+__device__ __forceinline__ void dequant_block_bf16(uint2 c, uint32_t sc, float sg, void* o) {
+  const uint32_t s7 = sc & 0x7F;
+  // e4m3 value: (8 + m) 2^(e - 10) for e >= 1 (as fp32 bits), m 2^-9 for e == 0
+  const float sb =
+      (s7 & 0x78) ? __uint_as_float((s7 << 20) + 0x3C000000u) : (float)s7 * 0x1p-9f;
+  const uint32_t b1 = bf16_of_product(sb, sg), b3 = bf16_of_product(3.f * sb, sg);
+  const uint32_t e1 = (b1 >> 7) & 0xFF, e3 = (b3 >> 7) & 0xFF;
+  // b1 and b3 are exact through the fp32 residual while every bit of the
+  // product is at or above 2^-149 (products from 2^-118 up: e1 >= 10), and
+  // 2^-1 b1 ... 2 b3 stay normal and finite for e1 >= 10, e3 <= 252
+  if (s7 != 0 && (e1 < 10 || e3 > 252)) {
+    dequant_block_exact<true>(c, sc, sg, o);
+    return;
+  }
+  const uint32_t z = s7 ? 0xFFFFFFFFu : 0u;
+  // magnitudes 0, 1/2, 1, 3/2 | 2, 3, 4, 6 as bf16 bits, two per word
+  const uint32_t t01 = ((b1 - 0x80u) << 16) & z;
+  const uint32_t t23 = (b1 | ((b3 - 0x80u) << 16)) & z;
+  const uint32_t t45 = ((b1 + 0x80u) | (b3 << 16)) & z;
+  const uint32_t t67 = ((b1 + 0x100u) | ((b3 + 0x80u) << 16)) & z;
+  const uint32_t L0 = __byte_perm(t01, t23, 0x6420), H0 = __byte_perm(t01, t23, 0x7531);
+  const uint32_t L1 = __byte_perm(t45, t67, 0x6420), H1 = __byte_perm(t45, t67, 0x7531);
+  uint32_t h[8];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint32_t w = q ? c.y : c.x;   // eight code nibbles
+    const uint32_t m0 = w & 0x7777u, m1 = (w >> 16) & 0x7777u;
+    const uint32_t l0 = __byte_perm(L0, L1, m0), h0 = __byte_perm(H0, H1, m0);
+    const uint32_t l1 = __byte_perm(L0, L1, m1), h1 = __byte_perm(H0, H1, m1);
+    // byte k of s4 / s8 carries the sign of element 2k / 2k + 1 in its top bit
+    const uint32_t s4 = (w << 4) & 0x80808080u, s8 = w & 0x80808080u;
+    h[4 * q + 0] = __byte_perm(l0, h0, 0x5140) | (__byte_perm(s4, s8, 0x4400) & 0x80008000u);
+    h[4 * q + 1] = __byte_perm(l0, h0, 0x7362) | (__byte_perm(s4, s8, 0x5511) & 0x80008000u);
+    h[4 * q + 2] = __byte_perm(l1, h1, 0x5140) | (__byte_perm(s4, s8, 0x6622) & 0x80008000u);
+    h[4 * q + 3] = __byte_perm(l1, h1, 0x7362) | (__byte_perm(s4, s8, 0x7733) & 0x80008000u);
+  }
+  uint4* d = reinterpret_cast<uint4*>(o);
+  d[0] = make_uint4(h[0], h[1], h[2], h[3]);
+  d[1] = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
+template <bool kBF16>
+__device__ __forceinline__ void dequant_block(uint2 c, uint32_t sc, float sg, void* o) {
+  if constexpr (kBF16)
+    dequant_block_bf16(c, sc, sg, o);
+  else
+    dequant_block_exact<false>(c, sc, sg, o);
 }
 
 // Problem blockIdx.y of a group.  Each thread step takes four 16-weight blocks
@@ -227,7 +303,11 @@ nvfp4_status launch_dequant_group(int P, const PtrArr<const uint8_t*>& codes,
                                   int64_t d_out, int64_t d_in, nvfp4_dtype ot, cudaStream_t st) {
   const int64_t nb = d_out * (d_in / kBlock);
   if (nb == 0 || P < 1) return NVFP4_OK;
-  int g = grid_for((nb + 3) / 4, 256) / P;
+  // many resident CTAs: each thread keeps four blocks' loads in flight, and
+  // the write-heavy stream wants every SM's load/store queues full
+  int64_t g = ((nb + 3) / 4 + 255) / 256;
+  if (g > 32 * kNumSMs) g = 32 * kNumSMs;
+  g /= P;
   const dim3 grid((unsigned)(g < 1 ? 1 : g), (unsigned)P);
   if (ot == NVFP4_BF16)
     dequant_kernel<true><<<grid, 256, 0, st>>>(codes, scales, sg, out, nb);

@@ -70,8 +70,10 @@ def test_dequant_bitexact(d_out, d_in, out):
     rng = np.random.default_rng(d_out * 7 + d_in)
     codes = rng.integers(0, 16, size=(d_out, d_in))
     scales = rng.integers(0, 127, size=(d_out, d_in // 16))
+    # 1e-30 and 1.1e35 put products at the bottom and top of the normal range
+    # (the bf16 path's exact fallback and the edge of its table)
     for sg in (np.float32(1.0), np.float32(3.7e-5), np.float32(rng.uniform(1e-6, 1e3)),
-               np.float32(1e-30)):
+               np.float32(1e-30), np.float32(1.1e35), np.float32(7.1e-36)):
         c = torch.from_numpy(pack_codes(codes)).to(DEV)
         s = torch.from_numpy(scales.astype(np.uint8)).to(DEV)
         g = torch.tensor([sg], dtype=torch.float32, device=DEV)
