@@ -16,7 +16,10 @@
 //               then split once instead of once per tile, and the shared
 //               memory traffic of the split is gone.
 //   warp 1      MMA issuer: per K step of 8, main += Ph Qh and
-//               cross += Ph Ql + Pl Qh (kind::tf32, M=128 N=128)
+//               cross += Ph Ql + Pl Qh (kind::tf32, M=128): Qh and Ql lie
+//               next to each other in the stage and the cross accumulator
+//               next to main in TMEM, so Ph [Qh; Ql] is one N=256 MMA (Ph is
+//               read once for both), then Pl Qh an N=128 one
 //   warps 6-13  epilogue (two warps per TMEM lane quarter, 64 columns each):
 //               every 128 K values the two accumulators are read out of TMEM
 //               and added, with round-to-nearest fp32 adds, into register sums
@@ -37,7 +40,7 @@ constexpr int GM = 128, GN = 128, GK = 32;
 constexpr int kStages = 3;
 constexpr int kChunkSteps = 4;                     // K = 128 per accumulator
 constexpr uint32_t kTile = GM * GK * 4;            // 16 KB (P or Q, raw/hi or lo)
-constexpr uint32_t kStageBytes = 4 * kTile;        // Ph, Qh, Pl, Ql
+constexpr uint32_t kStageBytes = 4 * kTile;        // Ph, Pl, Qh, Ql
 constexpr int kThreads = 448;                      // 14 warps
 constexpr int kEpiCols = GN / 2;                   // columns per epilogue thread
 constexpr uint32_t kBufCols = 2 * GN;              // main + cross
@@ -162,11 +165,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&sm->full[s], (presplit ? 4 : 2) * kTile);
+        // stage: Ph, Pl, Qh, Ql (Qh and Ql adjacent: one 256-row B operand)
         uint8_t* st = ring + s * kStageBytes;
         tma_load_3d(st, &tmP, &sm->full[s], kb * GK, tm * GM, b);
-        tma_load_3d(st + kTile, &tmQ, &sm->full[s], kb * GK, tn * GN, b);
+        tma_load_3d(st + 2 * kTile, &tmQ, &sm->full[s], kb * GK, tn * GN, b);
         if (presplit) {
-          tma_load_3d(st + 2 * kTile, &tmPl, &sm->full[s], kb * GK, tm * GM, b);
+          tma_load_3d(st + kTile, &tmPl, &sm->full[s], kb * GK, tm * GM, b);
           tma_load_3d(st + 3 * kTile, &tmQl, &sm->full[s], kb * GK, tn * GN, b);
         }
         ++issued;
@@ -198,10 +202,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        float4* hi = reinterpret_cast<float4*>(ring + s * kStageBytes);
-        float4* lo = reinterpret_cast<float4*>(ring + s * kStageBytes + 2 * kTile);
+        // raw P at Ph and raw Q at Qh; each tile's lo part goes kTile after it
+        uint8_t* stg = ring + s * kStageBytes;
 #pragma unroll 4
-        for (int i = tid; i < (int)(2 * kTile / 16); i += 128) {
+        for (int e = tid; e < (int)(2 * kTile / 16); e += 128) {
+          const int i = e & (int)(kTile / 16 - 1);
+          float4* hi = reinterpret_cast<float4*>(stg + (e >= (int)(kTile / 16) ? 2 * kTile : 0));
+          float4* lo = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(hi) + kTile);
           float4 x = hi[i];
           float4 h = make_float4(tf32_rn(x.x), tf32_rn(x.y), tf32_rn(x.z),
                                  tf32_rn(x.w));
@@ -219,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = instr_desc(2 /*tf32*/, 0, 0, GM, GN);
+    constexpr uint32_t idesc2 = instr_desc(2 /*tf32*/, 0, 0, GM, 2 * GN);
     int s = 0, g = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -241,17 +249,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t ph_ = smem_u32(ring + s * kStageBytes);
-          const uint32_t qh = ph_ + kTile, pl = ph_ + 2 * kTile, ql = ph_ + 3 * kTile;
+          const uint32_t pl = ph_ + kTile, qh = ph_ + 2 * kTile;
 #pragma unroll
           for (int k = 0; k < GK / 8; ++k) {
             const uint64_t dph = smem_desc_sw128(ph_ + 32 * k, 16, 1024);
-            const uint64_t dqh = smem_desc_sw128(qh + 32 * k, 16, 1024);
             const uint64_t dpl = smem_desc_sw128(pl + 32 * k, 16, 1024);
-            const uint64_t dql = smem_desc_sw128(ql + 32 * k, 16, 1024);
+            const uint64_t dq = smem_desc_sw128(qh + 32 * k, 16, 1024);   // Qh then Ql rows
             const uint32_t first = (kb != kb0) | (k != 0);
-            mma_tf32(mainc, dph, dqh, idesc, first);
-            mma_tf32(cross, dph, dql, idesc, first);
-            mma_tf32(cross, dpl, dqh, idesc, 1);
+            // Ph [Qh; Ql]^T: main += Ph Qh^T in columns 0..127 and cross +=
+            // Ph Ql^T in 128..255 (the cross accumulator sits right after
+            // main), one operand read of Ph; then cross += Pl Qh^T
+            mma_tf32(mainc, dph, dq, idesc2, first);
+            mma_tf32(cross, dpl, dq, idesc, 1);
           }
           mma_commit(&sm->empty[s]);
           if (++s == kStages) {
