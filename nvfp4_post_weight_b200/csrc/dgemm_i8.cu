@@ -252,9 +252,11 @@ __global__ void __launch_bounds__(256) slice_rows_kernel(const double* __restric
 // row tm holds min(2 tm + 2, nt) of them and starts at tm (tm + 1)).  A full
 // result is ordered by tile row first, then batch entry and column, with the
 // rows of a triangular P in the order of falling K range (ktri 1: ascending,
-// ktri 2: descending), so that the work per tile never grows along the order.
+// ktri 2: descending), so that the work per tile never grows along the order;
+// where the B slices are far larger than L2, by groups of tile rows (below).
+constexpr int kGroupRows = 16;
 struct ITiles {
-  int mt, nt, batch, lower, ktri;
+  int mt, nt, batch, lower, ktri, grouped;
   __device__ int per() const {
     if (!lower) return mt * nt;
     return mt * (mt + 1) - (nt < 2 * mt ? 2 * mt - nt : 0);   // the last row may be short
@@ -270,12 +272,27 @@ struct ITiles {
       while (r * (r + 1) > t) --r;
       tm = r;
       tn = t - r * (r + 1);
-    } else {
+    } else if (!grouped) {
       const int row = nt * batch;
       const int i = t / row;
       t -= i * row;
       b = t / nt;
       tn = t - b * nt;
+      tm = ktri == 2 ? mt - 1 - i : i;
+    } else {
+      // B slices far beyond L2: groups of kGroupRows tile rows, inside a group
+      // batch entry by batch entry and column by column, so that the CTAs of
+      // a round share a few A row slabs and a short run of B column slabs in
+      // L2 (row-major order would stream every B slab from DRAM once per
+      // round); the groups keep the falling K-range order
+      const int pg = kGroupRows * nt * batch;
+      const int g = t / pg;
+      t -= g * pg;
+      const int r = (mt - g * kGroupRows) < kGroupRows ? (mt - g * kGroupRows) : kGroupRows;
+      b = t / (r * nt);
+      t -= b * r * nt;
+      tn = t / r;
+      const int i = g * kGroupRows + t % r;
       tm = ktri == 2 ? mt - 1 - i : i;
     }
   }
@@ -574,7 +591,9 @@ nvfp4_status dgemm_i8(int M, int N, int K, double alpha, const double* P, int64_
   if (!encode_slices(&ma, A, K, (int64_t)batch * M, kp, planeA, IM) ||
       !encode_slices(&mb, Bsrc, K, (int64_t)batch * N, kp, same ? planeA : planeB, IN))
     return NVFP4_ERR_CUDA;
-  const ITiles ts{(M + IM - 1) / IM, (N + IN - 1) / IN, batch, lower, ktri};
+  // B slices past 256 MB (twice L2): group the tile rows
+  const int grouped = !lower && (int64_t)S * batch * N * kp > (int64_t(256) << 20);
+  const ITiles ts{(M + IM - 1) / IM, (N + IN - 1) / IN, batch, lower, ktri, grouped};
   const int64_t n_tiles =
       (int64_t)(lower ? (int64_t)ts.mt * (ts.mt + 1) : (int64_t)ts.mt * ts.nt) * batch;
   if (n_tiles > (1ll << 30)) return NVFP4_ERR_SHAPE;
