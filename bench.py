@@ -43,10 +43,20 @@ N_PHASES = 9                # the library's profiling phases (nvfp4pw.h)
 E2E_CHUNK_TOK = 1024        # tokens per host-to-device chunk of the end-to-end step
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor rates
 INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
-# DRAM bytes (read + write) of one launch of a phase's kernel, from an ncu
-# capture of the current kernel source (the launch named); a phase without an
-# entry reports null, and an entry is dropped when its kernel changes
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of a phase's kernel, from an ncu
+# capture of the current kernel source (what was averaged is named); a phase
+# without an entry reports null, and an entry is dropped when its kernel
+# changes.  factor_i8: ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum
+# over the 146 dgemm_i8_kernel launches of one 70B-decoder step (192.4 GB read,
+# 70.5 GB written; about 150 GB if every byte moved once: 127 GB of it the fp64
+# C of the trailing updates read and written, the rest slices and the
+# doubling levels' blocks).
+NCU_TRAFFIC = {
+    "factor_i8": {
+        "bytes": (192.4e9 + 70.5e9) / 146,
+        "launch": "mean over the 146 dgemm_i8_kernel launches of one dense_decoder_70b step",
+    },
+}
 I8_PAIRS = 21               # int8 slice products per fp64 MAC in the int8-slice GEMM (6 slices)
 FP64_LANES_PER_SM = 64      # B200: 64 FP64 FMA lanes per SM
 PHASE_NAMES = ["hessian", "prepare", "replay", "update", "dequant", "other", "factor_gemm",
