@@ -22,14 +22,17 @@
 // The levels are combined in fp64 in the epilogue.
 //
 // Persistent kernel, one CTA per SM, 128 x 64 output tiles:
-//   warp 0     TMA producer: a 4-stage ring, each stage 32 K-bytes of all S
+//   warp 0     TMA producer: a 2-stage ring, each stage 64 K-bytes of all S
 //              slices of A (128 rows) and B (64 rows), one 3-D load per
-//              operand (SWIZZLE_32B: one MMA's K per row)
+//              operand (SWIZZLE_64B: two MMAs' K per 64-byte row; rows of
+//              32 bytes took twice the TMA requests per byte and ran 6-8%
+//              slower even with a deeper ring)
 //   warp 1     MMA issuer.  The B slices of a stage lie one after another and
 //              so do the S level accumulators in TMEM (64 columns each), so
 //              A_t times the stacked B_0 .. B_{S-1-t} adds A_t B_u^T to level
 //              t + u for all u in one MMA of N = 64 (S - t) (cut at 256): 8
-//              MMAs per K step instead of S (S + 1) / 2 = 21 narrow ones
+//              MMAs per 32-byte K step instead of S (S + 1) / 2 = 21 narrow
+//              ones
 //   warps 2-5  epilogue: levels summed in fp64 straight out of TMEM, TMEM
 //              handed back (the next tile's MMAs start), then the tile is
 //              scaled by the row and column exponents and written through a
@@ -52,8 +55,8 @@ using namespace sm100;
 
 constexpr int S = 6;                     // slices per value
 constexpr int IM = 128, IN = 64;         // output tile
-constexpr int KC = 32;                   // K bytes (int8 values) per stage: one MMA's K
-constexpr int kIStages = 4;
+constexpr int KC = 64;                   // K bytes (int8 values) per stage: two MMAs' K
+constexpr int kIStages = 2;
 constexpr uint32_t kASlice = IM * KC;    // 4 KB
 constexpr uint32_t kBSlice = IN * KC;    // 2 KB
 constexpr uint32_t kIStage = S * (kASlice + kBSlice);   // 36 KB
@@ -78,15 +81,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// K-major operand in the canonical 32-byte-swizzled layout: rows of 32 bytes
-// (one MMA's K), 8-row groups 256 bytes apart.
-__device__ __forceinline__ uint64_t desc_sw32(uint32_t saddr) {
+// K-major operand in the canonical 64-byte-swizzled layout: rows of 64 bytes
+// (two MMAs' K; the second MMA's operand starts 32 bytes into the row),
+// 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
   d |= (uint64_t)1 << 16;             // leading byte offset (unused when K fits a row)
-  d |= (uint64_t)(256 >> 4) << 32;    // stride byte offset: 8 rows x 32 B
+  d |= (uint64_t)(512 >> 4) << 32;    // stride byte offset: 8 rows x 64 B
   d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
-  d |= (uint64_t)6 << 61;             // SWIZZLE_32B
+  d |= (uint64_t)4 << 61;             // SWIZZLE_64B
   return d;
 }
 
@@ -403,12 +407,15 @@ __global__ void __launch_bounds__(kIThreads, 1)
         // slices lie one after another in the stage and so do the level
         // accumulators in TMEM
 #pragma unroll
+        for (int kk = 0; kk < KC / 32; ++kk)
+#pragma unroll
         for (int t = 0; t < S; ++t)
 #pragma unroll
           for (int c0 = 0; c0 < IN * (S - t); c0 += kMaxN)
-            mma_i8(tmem + IN * t + c0, desc_sw32(a0 + t * kASlice), desc_sw32(b0 + c0 * KC),
+            mma_i8(tmem + IN * t + c0, desc_sw64(a0 + t * kASlice + 32 * kk),
+                   desc_sw64(b0 + c0 * KC + 32 * kk),
                    idesc_i8(IN * (S - t) - c0 < kMaxN ? IN * (S - t) - c0 : kMaxN),
-                   (i > 0 || t > 0) ? 1u : 0u);
+                   (i > 0 || t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm->empty[s]);
       }
       mma_commit(&sm->acc_full);   // arrives when this tile's MMAs are done (also if nk == 0)
@@ -526,7 +533,7 @@ bool encode_slices(CUtensorMap* map, const int8_t* base, int64_t K, int64_t tota
   const uint64_t strides[2] = {(uint64_t)kp, (uint64_t)plane};
   const uint32_t box[3] = {(uint32_t)KC, (uint32_t)box_rows, (uint32_t)S};
   return encode_tmap_nd(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, dims, strides, box,
-                        CU_TENSOR_MAP_SWIZZLE_32B);
+                        CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 nvfp4_status slice(const double* X, int64_t rows, int64_t K, int64_t ld, int64_t stride,
@@ -544,7 +551,7 @@ nvfp4_status slice(const double* X, int64_t rows, int64_t K, int64_t ld, int64_t
 }  // namespace
 
 size_t dgemm_i8_scratch_bytes(int64_t M, int64_t N, int64_t K, int batch) {
-  const int64_t kp = (K + 15) / 16 * 16;
+  const int64_t kp = (K + 63) / 64 * 64;
   return align256((size_t)S * batch * M * kp) + align256((size_t)S * batch * N * kp) +
          align256(sizeof(int) * batch * (M + N));
 }
@@ -568,7 +575,7 @@ nvfp4_status dgemm_i8(int M, int N, int K, double alpha, const double* P, int64_
       f = 2.0 * N * ((double)M * (M + 1) / 2 + (double)M * (K - M) * (ktri == 1));
     add_phase_work(f * batch);
   }
-  const int64_t kp = (K + 15) / 16 * 16;
+  const int64_t kp = (K + 63) / 64 * 64;
   const int64_t planeA = (int64_t)batch * M * kp, planeB = (int64_t)batch * N * kp;
   char* p = static_cast<char*>(scratch);
   int8_t* A = reinterpret_cast<int8_t*>(p);
