@@ -47,13 +47,13 @@ INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
 # capture of the current kernel source (what was averaged is named); a phase
 # without an entry reports null, and an entry is dropped when its kernel
 # changes.  factor_i8: ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum
-# over the 146 dgemm_i8_kernel launches of one 70B-decoder step (192.4 GB read,
-# 70.5 GB written; about 150 GB if every byte moved once: 127 GB of it the fp64
+# over the 146 dgemm_i8_kernel launches of one 70B-decoder step (194.2 GB read,
+# 70.4 GB written; about 150 GB if every byte moved once: 127 GB of it the fp64
 # C of the trailing updates read and written, the rest slices and the
 # doubling levels' blocks).
 NCU_TRAFFIC = {
     "factor_i8": {
-        "bytes": (192.4e9 + 70.5e9) / 146,
+        "bytes": (194.2e9 + 70.4e9) / 146,
         "launch": "mean over the 146 dgemm_i8_kernel launches of one dense_decoder_70b step",
     },
 }

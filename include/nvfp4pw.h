@@ -52,7 +52,9 @@ typedef enum {
   NVFP4_ERR_NOT_PD = 5,      /* damped H not positive definite (device)      */
   NVFP4_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (device)       */
   NVFP4_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed         */
-  NVFP4_ERR_UNSUPPORTED = 8  /* parameter value this build does not support  */
+  NVFP4_ERR_UNSUPPORTED = 8, /* parameter value this build does not support  */
+  NVFP4_ERR_BOUNDS = 9       /* debug build only: a kernel's tile or index
+                                left its array; the access was skipped (device) */
 } nvfp4_status;
 
 /* Element type of an input or output array. */
@@ -478,6 +480,17 @@ nvfp4_status nvfp4_gemm_nt_f32(int64_t M, int64_t N, int64_t K, float alpha, con
 /* Number of kernels this library has launched since it was loaded (all
  * threads, all devices).  Host-only; never fails. */
 long long nvfp4_launch_count(void);
+
+/* Debugging support (the paper has no counterpart; it stands in for a memory
+ * checker).  The library is also built as libnvfp4pw_debug.so with
+ * NVFP4_DEBUG defined: there every kernel checks the tile and index
+ * arithmetic it derives from the call's shapes (a tile decomposition that
+ * leaves its output, a row or column past the array) before each access; a
+ * failed check skips the access and records NVFP4_ERR_BOUNDS in the call's
+ * status word (for the tensor-core Hessian: the status nvfp4_hessian_status
+ * reads).  Results are otherwise identical to the release build.  Returns 1
+ * in the debug build, 0 in the release build.  Host-only; never fails. */
+int nvfp4_debug_build(void);
 
 /* Failure-detection support (the paper has no counterpart).  Sets, for the
  * current device, how long a pipeline wait inside the library's tensor-core

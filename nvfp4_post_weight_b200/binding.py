@@ -12,6 +12,10 @@ import os
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4pw.so")
+# the same library built with NVFP4_DEBUG (kernel index checks, see
+# nvfp4_debug_build in the header); NVFP4PW_DEBUG=1 makes lib() load it
+_LIB_DEBUG_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                               "libnvfp4pw_debug.so")
 
 NVFP4_BF16 = 0
 NVFP4_F32 = 1
@@ -19,7 +23,7 @@ NVFP4_F32 = 1
 _STATUS = {
     0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace",
     4: "non-finite input", 5: "not positive definite", 6: "timeout", 7: "CUDA error",
-    8: "unsupported parameter",
+    8: "unsupported parameter", 9: "index left its array (debug build)",
 }
 
 
@@ -40,72 +44,90 @@ _lib = None
 
 
 def lib():
-    """The loaded library; raises if it has not been built."""
+    """The loaded library (the debug build when NVFP4PW_DEBUG=1); raises if it
+    has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(_LIB_PATH):
-            raise RuntimeError(
-                f"{_LIB_PATH} is missing: build it with `python -m nvfp4_post_weight_b200.build`")
-        L = ctypes.CDLL(_LIB_PATH)
-        vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
-        f32 = ctypes.c_float
-        sig = {
-            "nvfp4_status_string": ([i32], ctypes.c_char_p),
-            "nvfp4_workspace_status": ([vp, vp], i32),
-            "nvfp4_default_params": ([ctypes.POINTER(SolveParams)], None),
-            "nvfp4_hessian_accumulate": ([vp, vp, i32, i64, i64, i32, vp], i32),
-            "nvfp4_hessian_status": ([vp], i32),
-            "nvfp4_hessian_host_workspace_size": ([i64, i64, i32], sz),
-            "nvfp4_hessian_accumulate_host": ([vp, vp, i32, i64, i64, i32, i64, vp, sz, vp],
-                                              i32),
-            "nvfp4_prepare_workspace_size": ([i64], sz),
-            "nvfp4_hessian_f64_workspace_size": ([i64, i64], sz),
-            "nvfp4_hessian_accumulate_f64": ([vp, vp, i32, i64, i64, i32, vp, sz, vp], i32),
-            "nvfp4_gptq_prepare_f64": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
-            "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
-            "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
-            "nvfp4_gptq_schur_replay_quantize": (
-                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, sz,
-                 vp], i32),
-            "nvfp4_gptq_schur_replay_quantize_noalloc": (
-                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
-                 vp], i32),
-            "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
-            "nvfp4_weight_amax": ([vp, i32, i64, i64, vp, vp, vp], i32),
-            "nvfp4_export_scales_size": ([i64, i64], sz),
-            "nvfp4_export_scales": ([vp, i64, i64, vp, vp], i32),
-            "nvfp4_gptq_schur_replay_quantize_rows": (
-                [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, vp,
-                 sz, vp], i32),
-            "nvfp4_hessian_accumulate_batched": ([i32, vp, vp, i32, vp, vp, i32, vp], i32),
-            "nvfp4_prepare_batched_workspace_size": ([i32, vp], sz),
-            "nvfp4_quantize_batched_workspace_size": ([i32, vp, vp, ctypes.POINTER(SolveParams)],
-                                                      sz),
-            "nvfp4_batched_workspace_status": ([vp, i32, vp, vp], i32),
-            "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, sz, vp], i32),
-            "nvfp4_gptq_schur_replay_quantize_batched": (
-                [i32, vp, i32, vp, vp, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
-                 sz, vp], i32),
-            "nvfp4_dequant_batched": ([i32, vp, vp, vp, vp, vp, vp, i32, vp], i32),
-            "nvfp4_layer_error_batched_workspace_size": ([i32, vp, vp], sz),
-            "nvfp4_layer_error_batched": ([i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-                                          i32),
-            "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
-                                   vp], i32),
-            "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
-            "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
-            "nvfp4_launch_count": ([], ctypes.c_longlong),
-            "nvfp4_set_wait_limit_ns": ([ctypes.c_ulonglong], i32),
-            "nvfp4_profile_begin": ([], i32),
-            "nvfp4_profile_end": ([vp, vp, i32], i32),
-            "nvfp4_profile_work": ([vp, i32], i32),
-        }
-        for name, (args, res) in sig.items():
-            fn = getattr(L, name)
-            fn.argtypes = args
-            fn.restype = res
-        _lib = L
+        _lib = _load(_LIB_DEBUG_PATH if os.environ.get("NVFP4PW_DEBUG") == "1" else _LIB_PATH)
     return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib():
+    """The debug build, loaded beside the release one (its calls take the
+    same arguments); raises if it has not been built."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(_LIB_DEBUG_PATH)
+    return _debug_lib
+
+
+def _load(path):
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m nvfp4_post_weight_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+    f32 = ctypes.c_float
+    sig = {
+        "nvfp4_status_string": ([i32], ctypes.c_char_p),
+        "nvfp4_workspace_status": ([vp, vp], i32),
+        "nvfp4_default_params": ([ctypes.POINTER(SolveParams)], None),
+        "nvfp4_hessian_accumulate": ([vp, vp, i32, i64, i64, i32, vp], i32),
+        "nvfp4_hessian_status": ([vp], i32),
+        "nvfp4_hessian_host_workspace_size": ([i64, i64, i32], sz),
+        "nvfp4_hessian_accumulate_host": ([vp, vp, i32, i64, i64, i32, i64, vp, sz, vp],
+                                          i32),
+        "nvfp4_prepare_workspace_size": ([i64], sz),
+        "nvfp4_hessian_f64_workspace_size": ([i64, i64], sz),
+        "nvfp4_hessian_accumulate_f64": ([vp, vp, i32, i64, i64, i32, vp, sz, vp], i32),
+        "nvfp4_gptq_prepare_f64": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
+        "nvfp4_gptq_prepare": ([vp, i64, f32, vp, vp, vp, vp, sz, vp], i32),
+        "nvfp4_quantize_workspace_size": ([i64, i64, ctypes.POINTER(SolveParams)], sz),
+        "nvfp4_gptq_schur_replay_quantize": (
+            [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, sz,
+             vp], i32),
+        "nvfp4_gptq_schur_replay_quantize_noalloc": (
+            [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
+             vp], i32),
+        "nvfp4_dequant": ([vp, vp, vp, i64, i64, vp, i32, vp], i32),
+        "nvfp4_weight_amax": ([vp, i32, i64, i64, vp, vp, vp], i32),
+        "nvfp4_export_scales_size": ([i64, i64], sz),
+        "nvfp4_export_scales": ([vp, i64, i64, vp, vp], i32),
+        "nvfp4_gptq_schur_replay_quantize_rows": (
+            [vp, i32, i64, i64, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp, vp,
+             sz, vp], i32),
+        "nvfp4_hessian_accumulate_batched": ([i32, vp, vp, i32, vp, vp, i32, vp], i32),
+        "nvfp4_prepare_batched_workspace_size": ([i32, vp], sz),
+        "nvfp4_quantize_batched_workspace_size": ([i32, vp, vp, ctypes.POINTER(SolveParams)],
+                                                  sz),
+        "nvfp4_batched_workspace_status": ([vp, i32, vp, vp], i32),
+        "nvfp4_gptq_prepare_batched": ([i32, vp, vp, f32, vp, vp, vp, vp, sz, vp], i32),
+        "nvfp4_gptq_schur_replay_quantize_batched": (
+            [i32, vp, i32, vp, vp, vp, ctypes.POINTER(SolveParams), vp, vp, vp, vp, vp, vp,
+             sz, vp], i32),
+        "nvfp4_dequant_batched": ([i32, vp, vp, vp, vp, vp, vp, i32, vp], i32),
+        "nvfp4_layer_error_batched_workspace_size": ([i32, vp, vp], sz),
+        "nvfp4_layer_error_batched": ([i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+                                      i32),
+        "nvfp4_gemm_nt_f32": ([i64, i64, i64, f32, vp, i64, vp, i64, f32, vp, i64, i32, vp,
+                               vp], i32),
+        "nvfp4_layer_error_workspace_size": ([i64, i64], sz),
+        "nvfp4_layer_error": ([vp, i32, vp, vp, vp, vp, i64, i64, vp, vp, sz, vp], i32),
+        "nvfp4_launch_count": ([], ctypes.c_longlong),
+        "nvfp4_debug_build": ([], i32),
+        "nvfp4_set_wait_limit_ns": ([ctypes.c_ulonglong], i32),
+        "nvfp4_profile_begin": ([], i32),
+        "nvfp4_profile_end": ([vp, vp, i32], i32),
+        "nvfp4_profile_work": ([vp, i32], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
 
 
 def _ptr(t):

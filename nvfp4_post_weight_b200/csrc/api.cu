@@ -51,6 +51,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_TIMEOUT: return "bounded device wait timed out";
     case NVFP4_ERR_CUDA: return "CUDA error";
     case NVFP4_ERR_UNSUPPORTED: return "unsupported parameter value";
+    case NVFP4_ERR_BOUNDS: return "index left its array (debug build check)";
   }
   return "unknown status";
 }

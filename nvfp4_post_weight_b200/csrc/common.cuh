@@ -83,6 +83,16 @@ struct ProfileScope {
   cudaStream_t st;
 };
 
+// Debug-build check (NVFP4_DEBUG): true when cond holds; otherwise records
+// NVFP4_ERR_BOUNDS in *status (first error wins) and yields false, so that
+// the caller skips the access.  In the release build it is the constant true.
+#ifdef NVFP4_DEBUG
+#define NVFP4_DCHECK(cond, status)                                                  \
+  ((cond) ? true : (atomicCAS((status), 0, (int)NVFP4_ERR_BOUNDS), false))
+#else
+#define NVFP4_DCHECK(cond, status) true
+#endif
+
 #define NVFP4_LAUNCH_CHECK()                                   \
   do {                                                         \
     if (cudaPeekAtLastError() != cudaSuccess) {                \

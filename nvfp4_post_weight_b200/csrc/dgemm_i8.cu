@@ -358,6 +358,12 @@ __global__ void __launch_bounds__(kIThreads, 1)
       int tm, tn, bz, kc0, nk;
       ts.get(t, tm, tn, bz);
       k_range(tm, kc0, nk);
+#ifdef NVFP4_DEBUG
+      if (!NVFP4_DCHECK(bz >= 0 && bz < ts.batch && tm >= 0 && tm < ts.mt && tn >= 0 &&
+                            tn < ts.nt && (!ts.lower || tn * IN <= tm * IM + IM - 1),
+                        status))
+        continue;   // debug build: a tile outside the output is skipped by every role
+#endif
       for (int i = 0; i < nk; ++i, ++g) {
         const int s = g % kIStages;
         if ((g >= kIStages && !mbar_wait(&sm->empty[s], ((g / kIStages) - 1) & 1)) ||
@@ -385,6 +391,12 @@ __global__ void __launch_bounds__(kIThreads, 1)
       int tm, tn, bz, kc0, nk;
       ts.get(t, tm, tn, bz);
       k_range(tm, kc0, nk);
+#ifdef NVFP4_DEBUG
+      if (!NVFP4_DCHECK(bz >= 0 && bz < ts.batch && tm >= 0 && tm < ts.mt && tn >= 0 &&
+                            tn < ts.nt && (!ts.lower || tn * IN <= tm * IM + IM - 1),
+                        status))
+        continue;   // debug build: a tile outside the output is skipped by every role
+#endif
       // the epilogue has read the previous tile's accumulators out of TMEM
       if (lt > 0 && !mbar_wait(&sm->acc_empty, (lt - 1) & 1)) {
         atomicExch(&sm->abort, 1);
@@ -441,6 +453,12 @@ __global__ void __launch_bounds__(kIThreads, 1)
       int tm, tn, bz, kc0, nk;
       ts.get(t, tm, tn, bz);
       k_range(tm, kc0, nk);
+#ifdef NVFP4_DEBUG
+      if (!NVFP4_DCHECK(bz >= 0 && bz < ts.batch && tm >= 0 && tm < ts.mt && tn >= 0 &&
+                            tn < ts.nt && (!ts.lower || tn * IN <= tm * IM + IM - 1),
+                        status))
+        continue;   // debug build: a tile outside the output is skipped by every role
+#endif
       const int m0 = tm * IM, n0 = tn * IN;
       const bool mine = __all_sync(0xffffffffu, mbar_wait(&sm->acc_full, lt & 1));
       tc_fence_after();

@@ -107,6 +107,21 @@ struct TileSpace {
   }
 };
 
+#ifdef NVFP4_DEBUG
+// debug build: the tile a loop is about to take lies inside the output
+__device__ bool tile_in_bounds(const TileSpace& ts, int t, int* status) {
+  int tm, tn, b;
+  ts.get(t, tm, tn, b);
+  return NVFP4_DCHECK(b >= 0 && b < ts.batch && tm >= 0 && tm < ts.mt && tn >= 0 &&
+                          tn < ts.nt && (!ts.lower || tn <= tm),
+                      status);
+}
+#define NVFP4_TILE_CHECK(t) \
+  if (!tile_in_bounds(ts, (t), status)) continue;
+#else
+#define NVFP4_TILE_CHECK(t)
+#endif
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nt_tc_kernel(const __grid_constant__ CUtensorMap tmP,
                       const __grid_constant__ CUtensorMap tmQ,
@@ -156,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       int tm, tn, b;
       ts.get(t, tm, tn, b);
       for (int kb = 0; kb < nk; ++kb) {
@@ -196,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait(&sm->full[s], ph)) {
           give_up(sm, status);
@@ -231,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       for (int kb0 = 0; ok && kb0 < nk; kb0 += kChunkSteps, ++g) {
         const int buf = g & 1;
         if (!mbar_wait(&sm->acc_empty[buf], ((g >> 1) & 1) ^ 1)) {
@@ -281,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !__any_sync(0xffffffffu, aborted(sm));
          t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       float sum[kEpiCols];
 #pragma unroll
       for (int k = 0; k < kEpiCols; ++k) sum[k] = 0.f;

@@ -134,6 +134,21 @@ __device__ __forceinline__ bool aborted(Smem* sm) {
   return *reinterpret_cast<volatile int*>(&sm->abort) != 0;
 }
 
+#ifdef NVFP4_DEBUG
+// debug build: the band tile a loop is about to take lies inside H
+__device__ bool band_tile_in_bounds(const BandTiles& band, int per, int P, int t) {
+  const int pb = t / per;
+  int I, J;
+  band.get(t - pb * per, I, J);
+  return NVFP4_DCHECK(pb < P && I >= 0 && I < band.nI && J < band.nJ && J >= (I >> 1),
+                      &g_hessian_status);
+}
+#define NVFP4_TILE_CHECK(t) \
+  if (!band_tile_in_bounds(band, per, grp.P, (t))) continue;
+#else
+#define NVFP4_TILE_CHECK(t)
+#endif
+
 __global__ void __launch_bounds__(kThreads, 1)
     hessian_tc_kernel(const __grid_constant__ HessGroup grp, int d, int beta, BandTiles band) {
   extern __shared__ uint8_t smem_raw[];
@@ -170,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     int issued = 0;
     for (int t = blockIdx.x; t < n_tiles && !aborted(sm); t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       const int pb = t / per;
       const CUtensorMap* tmX = &grp.map[pb];
       const int nk = nk_of(pb);
@@ -212,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;   // chunks issued by this CTA
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !aborted(sm); t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       const int nk = nk_of(t / per);
       for (int kb0 = 0; ok && kb0 < nk; kb0 += kChunkStages, ++g) {
         const int acc = g & 1;
@@ -263,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles && !__any_sync(0xffffffffu, aborted(sm));
          t += gridDim.x) {
+      NVFP4_TILE_CHECK(t)
       const int pb = t / per;
       const int nk = nk_of(pb);
       float* __restrict__ H = grp.H[pb];

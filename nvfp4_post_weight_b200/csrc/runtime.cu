@@ -5,7 +5,10 @@
 // While profiling is on, each launcher's ProfileScope records a CUDA event
 // pair on the launching stream; nvfp4_profile_end() waits for the events and
 // returns, per phase, the summed device time and the number of launches.
+// Every ProfileScope also opens an NVTX range named for its phase (always,
+// profiling on or off), so a tool attached through NVTX sees the phases.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <mutex>
@@ -77,8 +80,18 @@ void add_phase_work(double work) {
   g_phase_work[p] += work;
 }
 
+// NVTX range names of the phases (nvfp4_phase order); a tool that attaches
+// through NVTX sees every call's phases on the host timeline, and without one
+// a push or pop costs a pointer test.
+static const char* const kPhaseRangeNames[] = {
+    "nvfp4 hessian", "nvfp4 prepare", "nvfp4 replay", "nvfp4 update", "nvfp4 dequant",
+    "nvfp4 other",   "nvfp4 factor fp64 gemm", "nvfp4 panel", "nvfp4 factor int8 gemm"};
+
 ProfileScope::ProfileScope(int phase, cudaStream_t s) : slot(-1), prev_phase(t_phase), st(s) {
   t_phase = phase;
+  nvtxRangePushA(phase >= 0 && phase < (int)(sizeof(kPhaseRangeNames) / sizeof(kPhaseRangeNames[0]))
+                     ? kPhaseRangeNames[phase]
+                     : "nvfp4");
   if (!g_profiling.load(std::memory_order_relaxed)) return;
   std::lock_guard<std::mutex> lk(g_mu);
   Record r{phase, get_event(), get_event()};
@@ -92,6 +105,7 @@ ProfileScope::ProfileScope(int phase, cudaStream_t s) : slot(-1), prev_phase(t_p
 }
 
 ProfileScope::~ProfileScope() {
+  nvtxRangePop();
   t_phase = prev_phase;
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -162,6 +176,14 @@ using namespace nvfp4;
 extern "C" {
 
 long long nvfp4_launch_count(void) { return g_launches.load(); }
+
+int nvfp4_debug_build(void) {
+#ifdef NVFP4_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 nvfp4_status nvfp4_set_wait_limit_ns(unsigned long long ns) {
   const unsigned long long v = ns == 0 ? 4000000000ull : ns;

@@ -34,6 +34,17 @@ def test_library_exports_every_declared_function():
     assert not missing, missing
 
 
+def test_debug_library_exports_the_same_calls_and_says_so():
+    """libnvfp4pw_debug.so (NVFP4_DEBUG: kernel index checks) is the same ABI;
+    nvfp4_debug_build tells the two apart."""
+    dbg = ctypes.CDLL(B._LIB_DEBUG_PATH)
+    missing = [n for n in declared_functions() if not hasattr(dbg, n)]
+    assert not missing, missing
+    assert B.debug_lib().nvfp4_debug_build() == 1
+    assert B.lib().nvfp4_debug_build() == 0
+    assert B.lib().nvfp4_status_string(9) == b"index left its array (debug build check)"
+
+
 def test_binding_covers_every_declared_function():
     lib = B.lib()
     for n in declared_functions():
