@@ -40,7 +40,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 N_SM = 148
 N_PHASES = 9                # the library's profiling phases (nvfp4pw.h)
-E2E_CHUNK_TOK = 1024        # tokens per host-to-device chunk of the end-to-end step
+E2E_CHUNK_TOK = 8192        # tokens per host-to-device chunk of the end-to-end step
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor rates
 INT8_PER_BF16 = 4.5 / 2.25  # nominal dense int8 (= fp8) : bf16 tensor rates
 # DRAM bytes (read + write) per launch of a phase's kernel, from an ncu

@@ -90,19 +90,27 @@ class DecoderLayerSolver:
             B.nvfp4_hessian_accumulate(self.H(d), X[x], 0, stream)
             self.solve_group(list(t), W, stream, with_error)
 
-    def step_host(self, W_host, X_host, W_dev, chunk_tok=1024, stream=None, with_error=True,
+    def step_host(self, W_host, X_host, W_dev, chunk_tok=8192, stream=None, with_error=True,
                   out_host=None):
-        """The same solve from host-resident (pinned) inputs: each group's
-        tokens stream into its Hessian chunk by chunk; the group's weights are
-        copied into W_dev (device tensors of the same shapes) on a side stream
-        once its last token chunk is on the device, beside the prepare.  With
-        out_host = {name: (codes_h, scales_h, s_g_h)} the results are read
-        back on the side stream as soon as each quantize has written them; the
-        caller's stream waits for the read-backs at the end."""
+        """The same solve from host-resident (pinned) inputs, pipelined across
+        the groups: the tokens of group g + 1 stream into a second Hessian
+        buffer (the library's host-streamed Hessian, chunk_tok tokens per
+        chunk, on a Hessian stream) while group g is factored and quantized on
+        the caller's stream; a group's weights are copied into W_dev (device
+        tensors of the same shapes) on a side stream once its tokens are on the
+        device, beside its prepare.  With out_host = {name: (codes_h,
+        scales_h, s_g_h)} the results are read back on the side stream as soon
+        as each quantize has written them.  The caller's stream waits for all
+        of it at the end.  (Groups alternate between the two Hessian buffers;
+        H(d) afterwards holds group 0's, 2's, ... Hessian, not necessarily the
+        last one.)"""
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         if not hasattr(self, "_side"):
-            self._side = torch.cuda.Stream(self.device)
+            self._side = torch.cuda.Stream(self.device)   # weights in, results out
+            self._hst = torch.cuda.Stream(self.device)    # tokens into the Hessians
             self._ev = {}
+        if not hasattr(self, "_H2"):
+            self._H2 = torch.empty_like(self._H)
         ev = self._ev
 
         def event(key):
@@ -116,18 +124,38 @@ class DecoderLayerSolver:
                 B.nvfp4_hessian_host_workspace_size(self.dmax, chunk_tok, torch.bfloat16),
                 self.device)
             self._ws_host_key = key
-        for x, t in self.groups:
-            d = next(iter(t.values()))[1]
-            B.nvfp4_hessian_accumulate_host(self.H(d), X_host[x], chunk_tok, self.ws_host, 0, st)
-            event(("x", x)).record(st)
-            self._side.wait_event(event(("x", x)))
+        groups = self.groups
+        dims = [next(iter(t.values()))[1] for _, t in groups]
+        bufs = (self._H, self._H2)
+
+        def hbuf(i):
+            return bufs[i % 2][:dims[i] * dims[i]].view(dims[i], dims[i])
+
+        # the Hessian stream starts after what the caller queued before
+        event("start").record(st)
+        self._hst.wait_event(event("start"))
+
+        def hessian(i):
+            if i >= 2:   # the buffer's last reader: group i - 2's layer errors
+                self._hst.wait_event(event(("done", i - 2)))
+            B.nvfp4_hessian_accumulate_host(hbuf(i), X_host[groups[i][0]], chunk_tok,
+                                            self.ws_host, 0, self._hst)
+            event(("h", i)).record(self._hst)
+
+        hessian(0)
+        for i, (x, t) in enumerate(groups):
+            if i + 1 < len(groups):
+                hessian(i + 1)
+            d = dims[i]
+            H, U = hbuf(i), self.U(d)
+            self._side.wait_event(event(("h", i)))
             with torch.cuda.stream(self._side):
                 for n in t:
                     W_dev[n].copy_(W_host[n], non_blocking=True)
-                event(("w", x)).record(self._side)
-            H, U = self.H(d), self.U(d)
+                event(("w", i)).record(self._side)
+            st.wait_event(event(("h", i)))
             B.nvfp4_gptq_prepare(H, self.damp, U, self.dead[:d], self.lam, self.ws_prep, st)
-            st.wait_event(event(("w", x)))
+            st.wait_event(event(("w", i)))
             for n in t:
                 B.nvfp4_gptq_schur_replay_quantize(W_dev[n], U, self.codes[n], self.scales[n],
                                                    self.s_g[n], self.err[n], self.dead[:d],
@@ -144,9 +172,11 @@ class DecoderLayerSolver:
                 if with_error:
                     B.nvfp4_layer_error(W_dev[n], self.codes[n], self.scales[n], self.s_g[n], H,
                                         self.layer_err[n], self.ws_err, st)
-        if out_host is not None:
-            event("d2h").record(self._side)
-            st.wait_event(event("d2h"))
+            event(("done", i)).record(st)
+        event("side").record(self._side)
+        st.wait_event(event("side"))
+        event("hst").record(self._hst)
+        st.wait_event(event("hst"))
 
     def status(self, stream=None):
         return (B.nvfp4_workspace_status(self.ws_prep, stream),
